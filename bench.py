@@ -1,0 +1,361 @@
+#!/usr/bin/env python
+"""Throughput of the GPT-2 124M training step on B200.
+
+One step = one optimizer step of the pages' headline workload: micro-batch B=16, T=1024,
+32 gradient-accumulation micro-steps (524,288 tokens, loss / 32), then the global-norm
+clip and AdamW at lr = get_lr(1000).  Token streams are seeded synthetic Zipf(1.1) ids
+(the pages' datasets are not available); weights are the random GPT-2 init.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  With N > 1 (launched by torchrun) every rank trains an
+independent replica on its own token stream (the path has no exchange step in this
+build), and value = all ranks' tokens / the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPT-2 124M train tokens/sec (B=16,T=1024, 1 B200); ms/step; MFU vs BF16 peak"
+FLOP_PER_TOKEN = 6 * (12 * 12 * 768 * 768 + 50304 * 768) + 6 * 12 * 1024 * 768   # 798,031,872 (causal attention)
+NOMINAL_BF16_TFLOPS = 2250.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--micro-batch", type=int, default=16)
+    ap.add_argument("--seq", type=int, default=1024)
+    ap.add_argument("--accum", type=int, default=32)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks sampling
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world, backend):
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+
+
+def dist_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def cpu_oracle_sample(seq: int, samples: int = 1):
+    """Times the CPU oracle (fp32, as it stands) on B=1 x `seq` tokens of the same model:
+    forward + backward per sample, plus one clip + AdamW step amortised over the 32
+    micro-steps of an optimizer step."""
+    import torch
+    import oracle as O
+    from decoder_only_transformer_train_b200 import synthetic as S
+    cfg = O.GPT2_124M
+    params = O.init_params(cfg, 1, dtype=torch.float32)
+    x, y = S.token_batch(3, 1, seq, cfg.vocab_size)
+    x, y = torch.from_numpy(x), torch.from_numpy(y)
+    t0 = time.perf_counter()
+    grads = None
+    for _ in range(samples):
+        _, cache = O.forward(params, cfg, x, y)
+        grads = O.backward(params, cfg, cache, grad_scale=1.0 / 32, grads=grads)
+        del cache
+    t_fb = (time.perf_counter() - t0) / samples
+    m = {n: torch.zeros_like(t) for n, t in params.items()}
+    v = {n: torch.zeros_like(t) for n, t in params.items()}
+    t1 = time.perf_counter()
+    O.optimizer_step(params, grads, m, v, 1, cfg, lr=O.get_lr(1000))
+    t_opt = time.perf_counter() - t1
+    per_micro = t_fb + t_opt / 32
+    return seq / per_micro, torch.get_num_threads(), t_fb, t_opt
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, world, rank):
+    """The oracle, as it stands, on the host cores: each step is a bounded sample of the
+    workload (one B=1 x T micro-batch forward + backward, plus 1/32 of an optimizer step)."""
+    if rank != 0:
+        return
+    import torch
+    tok_s, threads, t_fb, t_opt = None, None, None, None
+    rates = []
+    for i in range(args.warmup + args.steps):
+        r, threads, t_fb, t_opt = cpu_oracle_sample(args.seq)
+        if i >= args.warmup:
+            rates.append(r)
+    value = statistics.mean(rates)
+    ms = args.micro_batch * args.seq * args.accum / value * 1000.0
+    line = {
+        "metric": METRIC, "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"GPT-2 124M fp32 CPU oracle, B=1 x T={args.seq} forward+backward "
+                                   f"({t_fb:.2f} s) plus 1/32 of clip+AdamW ({t_opt:.2f} s) per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(args):
+    return {"workload": f"GPT-2 124M training step: B={args.micro_batch} x T={args.seq}, "
+                        f"{args.accum} accumulation micro-steps ({args.micro_batch * args.seq * args.accum} tokens), "
+                        f"global-norm clip 1.0, AdamW at lr=get_lr(1000)",
+            "micro_batch": args.micro_batch, "seq_len": args.seq, "grad_accum_steps": args.accum,
+            "tokens_per_step": args.micro_batch * args.seq * args.accum,
+            "parallelism": "replicas" if args.gpus > 1 else "single-gpu",
+            "l2": "inputs larger than L2 (0.5 GB params + ~6 GB activations per micro-step)"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+    from decoder_only_transformer_train_b200 import binding as BD
+    from decoder_only_transformer_train_b200 import synthetic as S
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    B, T, k = args.micro_batch, args.seq, args.accum
+    cfg = BD.Config(n_layer=12, n_embd=768, n_head=12, block_size=1024, vocab_size=50257, padded_vocab_size=50304,
+                    max_batch=B, grad_accum_steps=k, precision=BD.GPT2_BF16)
+    stream = torch.cuda.Stream(device)
+    model = BD.GPT2(cfg, seed=1, stream=stream.cuda_stream)
+    lr = float(BD.lib().gpt2_lr_cosine(1000, 6e-4, 715, 19073, 0.1))
+    # each rank its own seeded token stream: k micro-batches of B x T (+1 for the targets)
+    run = S.zipf_tokens(3 + rank, k * B * T + 1, 50257)
+    x_host = run[:-1].reshape(k, B, T).astype(np.int32)
+    y_host = run[1:].reshape(k, B, T).astype(np.int32)
+    x_dev = torch.from_numpy(x_host).to(device)
+    y_dev = torch.from_numpy(y_host).to(device)
+
+    def step():
+        model.zero_grad()
+        for i in range(k):
+            model.forward(x_dev[i], y_dev[i], sync_loss=False)
+            model.backward()
+        model.adamw_step(lr, sync_norm=False)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize(device)
+    first_loss = model.get_loss()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize(device)
+    launches0 = int(BD.lib().gpt2_kernel_launches())
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            step()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    launches = int(BD.lib().gpt2_kernel_launches()) - launches0
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    ms_max = dist_max(ms_total, world, device)
+    tokens = world * args.steps * k * B * T
+    value = tokens / (ms_max / 1000.0)
+    last_loss = model.get_loss()
+
+    # per-kernel-class event timing of one more step (roofline of the dominant kernel)
+    with torch.cuda.stream(stream):
+        model.profile_start()
+        step()
+        prof = model.profile_stop()
+    torch.cuda.synchronize(device)
+
+    # end to end through the public API with host buffers: pinned token/target copies in,
+    # loss and grad norm out, every step
+    e2e = None
+    if not args.no_e2e:
+        xp = torch.from_numpy(x_host).pin_memory()
+        yp = torch.from_numpy(y_host).pin_memory()
+
+        def step_host():
+            model.zero_grad()
+            for i in range(k):
+                model.forward_host(xp[i], yp[i], sync_loss=False)
+                model.backward()
+            model.get_loss()
+            return model.adamw_step(lr, sync_norm=True)
+
+        barrier(world)
+        torch.cuda.synchronize(device)
+        t0 = time.perf_counter()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(args.steps):
+                step_host()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        wall = time.perf_counter() - t0
+        ms_e2e = dist_max(max(e0.elapsed_time(e1), wall * 1000.0), world, device)
+        e2e = {"value": tokens / (ms_e2e / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(2 * k * B * T * 4), "d2h_bytes_per_step": 8}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r, threads, t_fb, t_opt = cpu_oracle_sample(T)
+        cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"GPT-2 124M fp32 CPU oracle, B=1 x T={T} forward+backward ({t_fb:.2f} s) plus "
+                         f"1/32 of clip+AdamW ({t_opt:.2f} s)"}
+
+    if rank == 0:
+        pk = peaks()
+        tensor_classes = ("gemm_fwd", "gemm_bwd", "lm_head_fwd", "lm_head_bwd", "attn_fwd", "attn_bwd")
+        dom = max(prof, key=lambda c: prof[c]["ms"])
+        d = prof[dom]
+        if dom in tensor_classes:
+            achieved = d["flops"] / (d["ms"] / 1e3) / 1e12
+            peak = pk["bf16_tflops_sustained"]
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None, "kernel": dom,
+                    "launches": d["launches"], "avg_launch_ms": d["ms"] / max(1, d["launches"]),
+                    "peak_kind": f"{pk['source']} sustained dense bf16"}
+        else:
+            achieved = d["bytes"] / (d["ms"] / 1e3) / 1e9
+            peak = pk["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": None, "kernel": dom, "launches": d["launches"],
+                    "avg_launch_ms": d["ms"] / max(1, d["launches"]), "peak_kind": f"{pk['source']} HBM copy"}
+        step_ms = sum(p["ms"] for p in prof.values())
+        kernels = {}
+        for c, p in prof.items():
+            if p["launches"] == 0:
+                continue
+            ent = {"ms": round(p["ms"], 3), "share": round(p["ms"] / step_ms, 4), "launches": p["launches"]}
+            if p["flops"] > 0:
+                ent["tflops"] = round(p["flops"] / (p["ms"] / 1e3) / 1e12, 1)
+            if p["bytes"] > 0:
+                ent["gbs"] = round(p["bytes"] / (p["ms"] / 1e3) / 1e9, 1)
+            kernels[c] = ent
+        per_gpu = value / world
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(args),
+            "mfu": {"vs_nominal_2250": per_gpu * FLOP_PER_TOKEN / (NOMINAL_BF16_TFLOPS * 1e12),
+                    "vs_measured_sustained": per_gpu * FLOP_PER_TOKEN / (pk["bf16_tflops_sustained"] * 1e12),
+                    "flop_per_token": FLOP_PER_TOKEN},
+            "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clk, "gpu_launches": launches,
+            "loss": {"after_warmup": first_loss, "after_timed": last_loss},
+        }
+        print(json.dumps(line), flush=True)
+    model.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if world > 1:
+        args.gpus = world
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

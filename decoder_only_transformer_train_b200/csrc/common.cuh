@@ -1,0 +1,81 @@
+// Shared device helpers for the GPT-2 training-step kernels (sm_100a).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+typedef __nv_bfloat16 bf16;
+
+// Device-side error word, read by the host at sync points.  Kernels never trap: a
+// failed check records a code here and the kernel skips the offending access.
+enum DeviceError : int {
+  DEVERR_NONE = 0,
+  DEVERR_TOKEN = 1,     // input token id outside [0, vocab_size)
+  DEVERR_TARGET = 2,    // target outside [0, vocab_size) and not the ignore index -1
+  DEVERR_TIMEOUT = 3,   // a bounded wait on an mbarrier gave up
+  DEVERR_INTERNAL = 4,
+};
+
+extern __device__ int g_device_error;
+
+__device__ __forceinline__ void raise_device_error(int code) {
+  atomicCAS(&g_device_error, 0, code);
+}
+
+// ---------------------------------------------------------------- conversions
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f(float x) { return x; }
+  static __device__ __forceinline__ float from_f(float x) { return x; }
+};
+template <> struct Elem<bf16> {
+  static __device__ __forceinline__ float to_f(bf16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ bf16 from_f(float x) { return __float2bfloat16_rn(x); }
+};
+
+template <typename T> __device__ __forceinline__ float ld_f(const T* p) { return Elem<T>::to_f(*p); }
+template <typename T> __device__ __forceinline__ void st_f(T* p, float v) { *p = Elem<T>::from_f(v); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(h);
+}
+
+// ---------------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// ---------------------------------------------------------------- GELU (tanh form)
+// gelu(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))  -- the approximation GPT-2
+// used ("Karpathy's Zero to Hero, Lecture 9" notes, section "1:48:25 – 2:00:19").
+// tanhf is CUDA's, called, not re-implemented.
+#define GELU_A 0.7978845608028654f
+#define GELU_C 0.044715f
+__device__ __forceinline__ float gelu_tanh_f(float x) {
+  float t = tanhf(GELU_A * (x + GELU_C * x * x * x));
+  return 0.5f * x * (1.0f + t);
+}
+__device__ __forceinline__ float gelu_tanh_grad_f(float x) {
+  float t = tanhf(GELU_A * (x + GELU_C * x * x * x));
+  return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * GELU_A * (1.0f + 3.0f * GELU_C * x * x);
+}
+
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+__host__ __device__ __forceinline__ long long cdivll(long long a, long long b) { return (a + b - 1) / b; }

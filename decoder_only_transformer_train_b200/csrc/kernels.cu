@@ -1,0 +1,734 @@
+// Memory-bound kernels of the GPT-2 training step: embedding gather and its
+// deterministic backward, LayerNorm forward/backward, bias-gradient column sums, the
+// cross-entropy finalisation and its logit gradient, the global gradient norm, AdamW and
+// the parameter initialisation.  Rows are handled one warp each with coalesced (or
+// 128-bit) accesses and warp-shuffle reductions; every cross-block reduction is done in
+// a fixed order so that results are bitwise reproducible.
+//
+// Citations name "Karpathy's Zero to Hero, Lecture 9: Reproduce GPT-2 (124M)" notes (L9)
+// and a section on that page.
+#include <float.h>
+#include "common.cuh"
+#include "kernels.h"
+
+__device__ int g_device_error = 0;
+
+#include <atomic>
+static std::atomic<long long> g_kernel_launches{0};
+void note_kernel_launches(int n) { g_kernel_launches.fetch_add(n, std::memory_order_relaxed); }
+long long kernel_launch_count() { return g_kernel_launches.load(std::memory_order_relaxed); }
+
+int read_and_clear_device_error(int* code) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -3;
+  const int zero = 0;
+  if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return -3;
+  *code = v;
+  return 0;
+}
+
+namespace {
+
+// ================================================================ encoder forward
+// x[n, :] = wte[tok[n], :] + wpe[n mod T, :]   (L9, "Code you'll write": forward pass).
+// Out-of-range ids are reported and embed as zeros.
+__global__ void encoder_fwd_kernel(const int* __restrict__ tok, const float4* __restrict__ wte,
+                                   const float4* __restrict__ wpe, float4* __restrict__ x, int N, int T, int C4,
+                                   int V) {
+  const long long total = (long long)N * C4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / C4), c = (int)(i % C4);
+    const int t = n % T;
+    const int id = tok[n];
+    float4 o;
+    if (id < 0 || id >= V) {
+      if (c == 0) raise_device_error(DEVERR_TOKEN);
+      o = make_float4(0.f, 0.f, 0.f, 0.f);
+    } else {
+      const float4 a = wte[(long long)id * C4 + c], b = wpe[(long long)t * C4 + c];
+      o = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+    }
+    x[i] = o;
+  }
+}
+
+// ================================================================ LayerNorm
+// y = (x - mean) * rstd * w + b over the C channels of a row; biased variance, eps 1e-5
+// (nn.LayerNorm defaults, L9 "Code you'll write": Block).  One warp per row; lane l
+// owns channels l + 32k, so every load and store of the warp is one coalesced line.
+template <typename OutT, int CPL>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const float* __restrict__ x, const float* __restrict__ w,
+                                                     const float* __restrict__ b, OutT* __restrict__ y,
+                                                     float* __restrict__ mean, float* __restrict__ rstd, int N) {
+  constexpr int C = CPL * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + warp;
+  if (row >= N) return;
+  const float* xr = x + (long long)row * C;
+  float v[CPL];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    v[k] = xr[lane + 32 * k];
+    s += v[k];
+  }
+  const float mu = warp_sum(s) * (1.0f / C);
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    const float d = v[k] - mu;
+    ss += d * d;
+  }
+  const float r = rsqrtf(warp_sum(ss) * (1.0f / C) + 1e-5f);
+  OutT* yr = y + (long long)row * C;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    const int c = lane + 32 * k;
+    st_f(yr + c, (v[k] - mu) * r * w[c] + b[c]);
+  }
+  if (lane == 0) {
+    mean[row] = mu;
+    rstd[row] = r;
+  }
+}
+
+// dx = rstd * (dxhat - mean(dxhat) - xhat * mean(dxhat * xhat)),  dxhat = dy * w;
+// dres = (accumulate ? dres : 0) + dx, also written in the activation type for the next
+// GEMM.  dw = sum_rows dy * xhat and db = sum_rows dy go to per-block partials in a fixed
+// row order (block b owns rows b*8+warp + k*gridDim*8).
+template <typename ActT, int CPL>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
+                                                     const float* __restrict__ mean, const float* __restrict__ rstd,
+                                                     const float* __restrict__ w, float* __restrict__ dres,
+                                                     ActT* __restrict__ dres_act, int accumulate,
+                                                     float* __restrict__ part, int N) {
+  constexpr int C = CPL * 32;
+  extern __shared__ float red[];   // [8][2C]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float wv[CPL], dwa[CPL], dba[CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    wv[k] = w[lane + 32 * k];
+    dwa[k] = 0.f;
+    dba[k] = 0.f;
+  }
+  for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
+    const float* dyr = dy + (long long)row * C;
+    const float* xr = x + (long long)row * C;
+    const float mu = mean[row], r = rstd[row];
+    float g[CPL], xh[CPL];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      const int c = lane + 32 * k;
+      const float d = dyr[c];
+      xh[k] = (xr[c] - mu) * r;
+      g[k] = d * wv[k];
+      s1 += g[k];
+      s2 += g[k] * xh[k];
+      dwa[k] += d * xh[k];
+      dba[k] += d;
+    }
+    s1 = warp_sum(s1) * (1.0f / C);
+    s2 = warp_sum(s2) * (1.0f / C);
+    float* dr = dres + (long long)row * C;
+    ActT* da = dres_act + (long long)row * C;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      const int c = lane + 32 * k;
+      float o = r * (g[k] - s1 - xh[k] * s2);
+      if (accumulate) o += dr[c];
+      dr[c] = o;
+      st_f(da + c, o);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    red[warp * 2 * C + lane + 32 * k] = dwa[k];
+    red[warp * 2 * C + C + lane + 32 * k] = dba[k];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < 2 * C; c += blockDim.x) {
+    float s = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) s += red[wi * 2 * C + c];
+    part[(long long)blockIdx.x * 2 * C + c] = s;
+  }
+}
+
+__global__ void ln_param_reduce_kernel(const float* __restrict__ part, int nblocks, int C, float* __restrict__ dw,
+                                       float* __restrict__ db) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= 2 * C) return;
+  float s = 0.f;
+  for (int b = 0; b < nblocks; ++b) s += part[(long long)b * 2 * C + c];
+  if (c < C) dw[c] += s;
+  else db[c - C] += s;
+}
+
+// ================================================================ bias gradients
+// out[n] += sum_m x[m, n], rows in chunks of COLSUM_ROWS summed in order, then chunks
+// summed in order.
+constexpr int COLSUM_ROWS = 256;
+template <typename T>
+__global__ void colsum_partial_kernel(const T* __restrict__ x, long long ldx, int M, int N,
+                                      float* __restrict__ part) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const int m0 = blockIdx.y * COLSUM_ROWS, m1 = min(M, m0 + COLSUM_ROWS);
+  float s = 0.f;
+  for (int m = m0; m < m1; ++m) s += ld_f(x + (long long)m * ldx + n);
+  part[(long long)blockIdx.y * N + n] = s;
+}
+__global__ void colsum_reduce_kernel(const float* __restrict__ part, int nchunks, int N, float* __restrict__ out) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float s = 0.f;
+  for (int k = 0; k < nchunks; ++k) s += part[(long long)k * N + n];
+  out[n] += s;
+}
+
+// ================================================================ cross-entropy
+// Combines the per-(row, column-tile) partials of the fused lm_head epilogue:
+// lse = log sum_v exp(z_v) over all padded columns (L9 "2:06:39 – 2:14:58": pad rows are
+// live output logits); loss_row = lse - z[target] (F.cross_entropy, L9 "52:38 – 1:06:18");
+// argmax = lowest column reaching the row maximum.  Target -1 is ignored.
+__device__ __forceinline__ void lse_combine(float& m, float& s, float om, float os) {
+  const float nm = fmaxf(m, om);
+  if (nm == -INFINITY) return;
+  s = s * __expf(m - nm) + os * __expf(om - nm);
+  m = nm;
+}
+__device__ __forceinline__ void amax_combine(float& av, int& ai, float ov, int oi) {
+  if (ov > av || (ov == av && oi < ai)) {
+    av = ov;
+    ai = oi;
+  }
+}
+
+__global__ void ce_finalize_kernel(const CePartial* __restrict__ part, int n_tiles, const float* __restrict__ zt,
+                                   const int* __restrict__ targets, int N, int V, float* __restrict__ lse,
+                                   float* __restrict__ loss_row, int* __restrict__ argmax) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (row >= N) return;
+  float m = -INFINITY, s = 0.f, av = -INFINITY;
+  int ai = 0x7fffffff;
+  for (int t = lane; t < n_tiles; t += 32) {
+    const CePartial p = part[(long long)row * n_tiles + t];
+    lse_combine(m, s, p.max, p.sum);
+    amax_combine(av, ai, p.amax, p.aidx);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, o), os = __shfl_xor_sync(0xffffffffu, s, o);
+    const float oav = __shfl_xor_sync(0xffffffffu, av, o);
+    const int oai = __shfl_xor_sync(0xffffffffu, ai, o);
+    lse_combine(m, s, om, os);
+    amax_combine(av, ai, oav, oai);
+  }
+  if (lane == 0) {
+    const float l = m + logf(s);
+    const int y = targets[row];
+    const bool valid = (y >= 0 && y < V);
+    if (!valid && y != -1) raise_device_error(DEVERR_TARGET);
+    lse[row] = l;
+    loss_row[row] = valid ? (l - zt[row]) : 0.f;
+    argmax[row] = ai;
+  }
+}
+
+// fp32 parity mode: the same quantities straight from an fp32 logits row.
+__global__ void __launch_bounds__(256) ce_rowwise_kernel(const float* __restrict__ logits, long long ld,
+                                                         const int* __restrict__ targets, int N, int Vp, int V,
+                                                         float* __restrict__ lse, float* __restrict__ loss_row,
+                                                         int* __restrict__ argmax) {
+  __shared__ float sm[8], ss[8], sav[8];
+  __shared__ int sai[8];
+  const int row = blockIdx.x;
+  const float* z = logits + (long long)row * ld;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float m = -INFINITY, s = 0.f, av = -INFINITY;
+  int ai = 0x7fffffff;
+  for (int v = threadIdx.x; v < Vp; v += blockDim.x) {
+    const float x = z[v];
+    lse_combine(m, s, x, 1.0f);
+    amax_combine(av, ai, x, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, o), os = __shfl_xor_sync(0xffffffffu, s, o);
+    const float oav = __shfl_xor_sync(0xffffffffu, av, o);
+    const int oai = __shfl_xor_sync(0xffffffffu, ai, o);
+    lse_combine(m, s, om, os);
+    amax_combine(av, ai, oav, oai);
+  }
+  if (lane == 0) {
+    sm[warp] = m; ss[warp] = s; sav[warp] = av; sai[warp] = ai;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int wi = 1; wi < 8; ++wi) {
+      lse_combine(m, s, sm[wi], ss[wi]);
+      amax_combine(av, ai, sav[wi], sai[wi]);
+    }
+    const float l = m + logf(s);
+    const int y = targets[row];
+    const bool valid = (y >= 0 && y < V);
+    if (!valid && y != -1) raise_device_error(DEVERR_TARGET);
+    lse[row] = l;
+    loss_row[row] = valid ? (l - z[y < 0 ? 0 : y]) : 0.f;
+    argmax[row] = ai;
+  }
+}
+
+// loss = mean of loss_row over valid rows (fixed-order double sum); dz_scale =
+// grad_scale / count, grad_scale = 1 / grad_accum_steps (L9 "2:34:49 – 2:46:43").
+__global__ void __launch_bounds__(1024) loss_reduce_kernel(const float* __restrict__ loss_row,
+                                                           const int* __restrict__ targets, int N, float grad_scale,
+                                                           float* loss_out, float* dz_scale_out, int* count_out) {
+  __shared__ double sd[1024];
+  __shared__ int sc[1024];
+  double s = 0.0;
+  int c = 0;
+  for (int i = threadIdx.x; i < N; i += 1024) {
+    s += (double)loss_row[i];
+    c += (targets[i] != -1) ? 1 : 0;
+  }
+  sd[threadIdx.x] = s;
+  sc[threadIdx.x] = c;
+  __syncthreads();
+  for (int o = 512; o > 0; o >>= 1) {
+    if ((int)threadIdx.x < o) {
+      sd[threadIdx.x] += sd[threadIdx.x + o];
+      sc[threadIdx.x] += sc[threadIdx.x + o];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int cnt = sc[0];
+    *loss_out = cnt > 0 ? (float)(sd[0] / cnt) : 0.f;
+    *dz_scale_out = cnt > 0 ? grad_scale / (float)cnt : 0.f;
+    *count_out = cnt;
+  }
+}
+
+// In place: z[row, v] <- (exp(z - lse) - [v == y]) * scale on valid rows, 0 on ignored rows.
+template <typename T>
+__global__ void ce_dz_kernel(T* __restrict__ z, long long ld, const float* __restrict__ lse,
+                             const int* __restrict__ targets, const float* __restrict__ dz_scale, int Vp) {
+  const int row = blockIdx.y;
+  const int y = targets[row];
+  const float l = lse[row];
+  const float sc = (y >= 0) ? *dz_scale : 0.f;
+  T* zr = z + (long long)row * ld;
+  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < Vp; v += gridDim.x * blockDim.x) {
+    const float p = expf(ld_f(zr + v) - l);
+    st_f(zr + v, (p - (v == y ? 1.f : 0.f)) * sc);
+  }
+}
+__global__ void ce_dz_bf16x8_kernel(uint4* __restrict__ z, long long ld8, const float* __restrict__ lse,
+                                    const int* __restrict__ targets, const float* __restrict__ dz_scale, int Vp8) {
+  const int row = blockIdx.y;
+  const int y = targets[row];
+  const float l = lse[row];
+  const float sc = (y >= 0) ? *dz_scale : 0.f;
+  uint4* zr = z + (long long)row * ld8;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < Vp8; i += gridDim.x * blockDim.x) {
+    uint4 q = zr[i];
+    uint32_t* w = reinterpret_cast<uint32_t*>(&q);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = unpack_bf16x2(w[k]);
+      const int v0 = i * 8 + 2 * k;
+      const float a = (expf(f.x - l) - (v0 == y ? 1.f : 0.f)) * sc;
+      const float b = (expf(f.y - l) - (v0 + 1 == y ? 1.f : 0.f)) * sc;
+      w[k] = pack_bf16x2(a, b);
+    }
+    zr[i] = q;
+  }
+}
+
+// ================================================================ encoder backward
+// dwte[v] += sum of dx0 rows at positions holding token v; dwpe[t] += sum_b dx0[b, t].
+// Deterministic: (token, position) keys are sorted in one CTA (bitonic), runs of equal
+// tokens are summed in position order by fixed 32-entry chunks; a run that crosses chunk
+// boundaries is finished by the chunk where it starts, adding the later chunks' partial
+// sums in chunk order.
+constexpr int ENC_CHUNK = 32;
+constexpr int ENC_POS_BITS = 15;   // positions < 32768
+
+__global__ void __launch_bounds__(1024) enc_sort_kernel(const int* __restrict__ tok, int N, int V, int P,
+                                                        uint32_t* __restrict__ sorted) {
+  extern __shared__ uint32_t keys[];
+  for (int i = threadIdx.x; i < P; i += 1024) {
+    uint32_t k = 0xFFFFFFFFu;
+    if (i < N) {
+      int t = tok[i];
+      t = t < 0 ? 0 : (t >= V ? V - 1 : t);
+      k = (static_cast<uint32_t>(t) << ENC_POS_BITS) | static_cast<uint32_t>(i);
+    }
+    keys[i] = k;
+  }
+  for (int k = 2; k <= P; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      __syncthreads();
+      for (int i = threadIdx.x; i < P; i += 1024) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint32_t a = keys[i], b = keys[ixj];
+          const bool asc = (i & k) == 0;
+          if ((a > b) == asc) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < N; i += 1024) sorted[i] = keys[i];
+}
+
+__device__ __forceinline__ int key_tok(uint32_t k) { return static_cast<int>(k >> ENC_POS_BITS); }
+
+__global__ void enc_chunk_kernel(const uint32_t* __restrict__ sorted, const float* __restrict__ dx0,
+                                 float* __restrict__ dwte, float* __restrict__ part, int N, int C) {
+  const int c = blockIdx.x;
+  const int ch = blockIdx.y * 128 + threadIdx.x * 4;
+  if (ch >= C) return;
+  const int i0 = c * ENC_CHUNK, i1 = min(N, i0 + ENC_CHUNK);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  int seg_start = i0;
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t key = sorted[i];
+    const int t = key_tok(key);
+    const int pos = static_cast<int>(key & ((1u << ENC_POS_BITS) - 1));
+    const float4 d = *reinterpret_cast<const float4*>(dx0 + (long long)pos * C + ch);
+    acc.x += d.x; acc.y += d.y; acc.z += d.z; acc.w += d.w;
+    const bool run_end = (i + 1 == N) || key_tok(sorted[i + 1]) != t;
+    if (run_end || i + 1 == i1) {
+      const bool starts_here = (seg_start > i0) || (i0 == 0) || key_tok(sorted[i0 - 1]) != t;
+      if (starts_here && run_end) {
+        float4* o = reinterpret_cast<float4*>(dwte + (long long)t * C + ch);
+        float4 w = *o;
+        w.x += acc.x; w.y += acc.y; w.z += acc.z; w.w += acc.w;
+        *o = w;
+      } else {
+        const int slot = (seg_start == i0) ? 0 : 1;
+        *reinterpret_cast<float4*>(part + ((long long)c * 2 + slot) * C + ch) = acc;
+      }
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      seg_start = i + 1;
+    }
+  }
+}
+
+__global__ void enc_fixup_kernel(const uint32_t* __restrict__ sorted, float* __restrict__ dwte,
+                                 const float* __restrict__ part, int N, int C, int nchunks) {
+  const int c = blockIdx.x;
+  const int ch = blockIdx.y * 128 + threadIdx.x * 4;
+  if (ch >= C) return;
+  const int i0 = c * ENC_CHUNK, i1 = min(N, i0 + ENC_CHUNK);
+  const int t = key_tok(sorted[i1 - 1]);
+  const bool crosses_out = (i1 < N) && key_tok(sorted[i1]) == t;
+  const bool crosses_in = (i0 > 0) && key_tok(sorted[i0 - 1]) == t && key_tok(sorted[i0]) == t;
+  if (!crosses_out || crosses_in) return;
+  const int slot = (key_tok(sorted[i0]) == t) ? 0 : 1;
+  float4 tot = *reinterpret_cast<const float4*>(part + ((long long)c * 2 + slot) * C + ch);
+  for (int c2 = c + 1; c2 < nchunks && key_tok(sorted[c2 * ENC_CHUNK]) == t; ++c2) {
+    const float4 p = *reinterpret_cast<const float4*>(part + ((long long)c2 * 2) * C + ch);
+    tot.x += p.x; tot.y += p.y; tot.z += p.z; tot.w += p.w;
+  }
+  float4* o = reinterpret_cast<float4*>(dwte + (long long)t * C + ch);
+  float4 w = *o;
+  w.x += tot.x; w.y += tot.y; w.z += tot.z; w.w += tot.w;
+  *o = w;
+}
+
+__global__ void dwpe_kernel(const float* __restrict__ dx0, float* __restrict__ dwpe, int B, int T, int C) {
+  const long long total = (long long)T * C;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int b = 0; b < B; ++b) s += dx0[(long long)b * total + i];
+    dwpe[i] += s;
+  }
+}
+
+// ================================================================ norm, AdamW, init
+// Global gradient norm sqrt(sum g^2) (L9 "2:14:58 – 2:25:57": clip_grad_norm_ at 1.0),
+// fixed grid and fixed-order double partials; scale = min(1, clip / (norm + 1e-6)).
+__global__ void __launch_bounds__(512) sumsq_kernel(const float* __restrict__ g, long long n,
+                                                    double* __restrict__ part) {
+  __shared__ double sd[512];
+  double s = 0.0;
+  const long long n4 = n / 4;
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  for (long long i = blockIdx.x * 512LL + threadIdx.x; i < n4; i += (long long)gridDim.x * 512) {
+    const float4 v = g4[i];
+    s += (double)(v.x * v.x) + (double)(v.y * v.y) + (double)(v.z * v.z) + (double)(v.w * v.w);
+  }
+  if (blockIdx.x == 0)
+    for (long long i = n4 * 4 + threadIdx.x; i < n; i += 512) s += (double)g[i] * (double)g[i];
+  sd[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = 256; o > 0; o >>= 1) {
+    if ((int)threadIdx.x < o) sd[threadIdx.x] += sd[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) part[blockIdx.x] = sd[0];
+}
+__global__ void norm_finalize_kernel(const double* __restrict__ part, int nparts, float clip, float* out2) {
+  __shared__ double sd[256];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += 256) s += part[i];
+  sd[threadIdx.x] = s;
+  __syncthreads();
+  for (int o = 128; o > 0; o >>= 1) {
+    if ((int)threadIdx.x < o) sd[threadIdx.x] += sd[threadIdx.x + o];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const double norm = sqrt(sd[0]);
+    out2[0] = (float)norm;
+    out2[1] = (float)fmin(1.0, (double)clip / (norm + 1e-6));
+  }
+}
+
+// AdamW with decoupled weight decay and bias correction (torch.optim.AdamW semantics; L9
+// "2:14:58 – 2:25:57" betas/eps, "2:25:57 – 2:34:49" decay on >= 2-D tensors only).
+// One launch updates every tensor; each block reads its (offset, count, decay) entry.
+__global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
+                                                    float* __restrict__ m, float* __restrict__ v,
+                                                    bf16* __restrict__ shadow, const AdamBlock* __restrict__ blocks,
+                                                    const float* __restrict__ clip_scale, float lr, float b1,
+                                                    float b2, float eps, float wd, float bc1, float bc2) {
+  const AdamBlock blk = blocks[blockIdx.x];
+  const float s = *clip_scale;
+  const float decay = blk.decay ? (1.0f - lr * wd) : 1.0f;
+  for (int i = threadIdx.x; i < blk.n; i += blockDim.x) {
+    const long long idx = blk.off + i;
+    const float gi = g[idx] * s;
+    const float mi = b1 * m[idx] + (1.0f - b1) * gi;
+    const float vi = b2 * v[idx] + (1.0f - b2) * gi * gi;
+    const float mh = mi / bc1;
+    const float vh = vi / bc2;
+    const float pi = p[idx] * decay - lr * mh / (sqrtf(vh) + eps);
+    p[idx] = pi;
+    m[idx] = mi;
+    v[idx] = vi;
+    if (shadow != nullptr && blk.decay) shadow[idx] = __float2bfloat16_rn(pi);
+  }
+}
+
+// Initialisation draw: value e of a tensor = float(std * sqrt(-2 ln u1) cos(2 pi u2)) with
+// u1 = 1 - (r_{2e} >> 11) 2^-53, u2 = (r_{2e+1} >> 11) 2^-53, r_j the j-th SplitMix64
+// output (Steele, Lea & Flood 2014) of the tensor's state.  Double-precision log, cos and
+// sqrt are CUDA's, called.
+__device__ __forceinline__ uint64_t splitmix64_at(uint64_t state, uint64_t j) {
+  uint64_t z = state + (j + 1ull) * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+__global__ void init_normal_kernel(float* __restrict__ p, long long n, uint64_t state, double std) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x) {
+    const uint64_t r1 = splitmix64_at(state, 2ull * e), r2 = splitmix64_at(state, 2ull * e + 1ull);
+    const double u1 = 1.0 - (double)(r1 >> 11) * 0x1.0p-53;
+    const double u2 = (double)(r2 >> 11) * 0x1.0p-53;
+    const double z = sqrt(-2.0 * log(u1)) * cos(2.0 * 3.141592653589793 * u2);
+    p[e] = (float)(std * z);
+  }
+}
+__global__ void fill_kernel(float* __restrict__ p, long long n, float value) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x)
+    p[e] = value;
+}
+__global__ void cast_bf16_kernel(const float* __restrict__ s, bf16* __restrict__ d, long long n) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n;
+       e += (long long)gridDim.x * blockDim.x)
+    d[e] = __float2bfloat16_rn(s[e]);
+}
+
+inline int grid_for(long long n, int threads, int cap = 148 * 16) {
+  long long g = cdivll(n, threads);
+  if (g > cap) g = cap;
+  return (int)(g < 1 ? 1 : g);
+}
+inline int ok() { return cudaGetLastError() == cudaSuccess ? 0 : -3; }
+
+template <typename OutT>
+int ln_fwd_dispatch(cudaStream_t st, const float* x, const float* w, const float* b, OutT* y, float* mean,
+                    float* rstd, int N, int C) {
+  const int grid = cdiv(N, 8);
+  switch (C) {
+#define LNF(CPL) case CPL * 32: ln_fwd_kernel<OutT, CPL><<<grid, 256, 0, st>>>(x, w, b, y, mean, rstd, N); break;
+    LNF(1) LNF(2) LNF(4) LNF(8) LNF(12) LNF(16) LNF(24) LNF(32)
+#undef LNF
+    default: return -4;
+  }
+  note_kernel_launches(1);
+  return ok();
+}
+
+template <typename ActT>
+int ln_bwd_dispatch(cudaStream_t st, const float* dy, const float* x, const float* mean, const float* rstd,
+                    const float* w, float* dres, ActT* dres_act, int acc, float* part, int nblocks, int N, int C) {
+  const int smem = 8 * 2 * C * (int)sizeof(float);
+  switch (C) {
+#define LNB(CPL)                                                                                               \
+  case CPL * 32: {                                                                                             \
+    auto k = ln_bwd_kernel<ActT, CPL>;                                                                         \
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) return -3; \
+    k<<<nblocks, 256, smem, st>>>(dy, x, mean, rstd, w, dres, dres_act, acc, part, N);                         \
+    break;                                                                                                     \
+  }
+    LNB(1) LNB(2) LNB(4) LNB(8) LNB(12) LNB(16) LNB(24) LNB(32)
+#undef LNB
+    default: return -4;
+  }
+  note_kernel_launches(1);
+  return ok();
+}
+
+}  // namespace
+
+// ==================================================================== launchers
+int launch_encoder_fwd(cudaStream_t st, const int* tok, const float* wte, const float* wpe, float* x, int N, int T,
+                       int C, int V) {
+  if (C % 4) return -4;
+  const long long total = (long long)N * (C / 4);
+  encoder_fwd_kernel<<<grid_for(total, 256), 256, 0, st>>>(tok, reinterpret_cast<const float4*>(wte),
+                                                           reinterpret_cast<const float4*>(wpe),
+                                                           reinterpret_cast<float4*>(x), N, T, C / 4, V);
+  note_kernel_launches(1);
+  return ok();
+}
+
+int launch_layernorm_fwd(cudaStream_t st, bool is_bf16, const float* x, const float* w, const float* b, void* y,
+                         float* mean, float* rstd, int N, int C) {
+  if (is_bf16) return ln_fwd_dispatch<bf16>(st, x, w, b, reinterpret_cast<bf16*>(y), mean, rstd, N, C);
+  return ln_fwd_dispatch<float>(st, x, w, b, reinterpret_cast<float*>(y), mean, rstd, N, C);
+}
+
+int layernorm_bwd_blocks(int num_sms) { return 2 * num_sms; }
+
+int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const float* dy, const float* x, const float* mean,
+                         const float* rstd, const float* w, float* dres, void* dres_act, bool accumulate, float* part,
+                         int nblocks, float* dw, float* db, int N, int C) {
+  int rc = is_bf16 ? ln_bwd_dispatch<bf16>(st, dy, x, mean, rstd, w, dres, reinterpret_cast<bf16*>(dres_act),
+                                           accumulate, part, nblocks, N, C)
+                   : ln_bwd_dispatch<float>(st, dy, x, mean, rstd, w, dres, reinterpret_cast<float*>(dres_act),
+                                            accumulate, part, nblocks, N, C);
+  if (rc) return rc;
+  ln_param_reduce_kernel<<<cdiv(2 * C, 256), 256, 0, st>>>(part, nblocks, C, dw, db);
+  note_kernel_launches(1);
+  return ok();
+}
+
+int colsum_chunks(int M) { return cdiv(M, COLSUM_ROWS); }
+
+int launch_colsum(cudaStream_t st, bool is_bf16, const void* x, long long ldx, int M, int N, float* part,
+                  int nchunks, float* out) {
+  dim3 grid(cdiv(N, 256), nchunks);
+  if (is_bf16) colsum_partial_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, part);
+  else colsum_partial_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, part);
+  colsum_reduce_kernel<<<cdiv(N, 256), 256, 0, st>>>(part, nchunks, N, out);
+  note_kernel_launches(2);
+  return ok();
+}
+
+int launch_ce_finalize(cudaStream_t st, const CePartial* part, int n_tiles, const float* zt, const int* targets,
+                       int N, int V, float* lse, float* loss_row, int* argmax) {
+  ce_finalize_kernel<<<cdiv(N, 8), 256, 0, st>>>(part, n_tiles, zt, targets, N, V, lse, loss_row, argmax);
+  note_kernel_launches(1);
+  return ok();
+}
+
+int launch_ce_rowwise(cudaStream_t st, const float* logits, long long ld, const int* targets, int N, int Vp, int V,
+                      float* lse, float* loss_row, int* argmax) {
+  ce_rowwise_kernel<<<N, 256, 0, st>>>(logits, ld, targets, N, Vp, V, lse, loss_row, argmax);
+  note_kernel_launches(1);
+  return ok();
+}
+
+int launch_loss_reduce(cudaStream_t st, const float* loss_row, const int* targets, int N, float grad_scale,
+                       float* loss_out, float* dz_scale_out, int* count_out) {
+  loss_reduce_kernel<<<1, 1024, 0, st>>>(loss_row, targets, N, grad_scale, loss_out, dz_scale_out, count_out);
+  note_kernel_launches(1);
+  return ok();
+}
+
+int launch_ce_dz(cudaStream_t st, bool is_bf16, void* logits, long long ld, const float* lse, const int* targets,
+                 const float* dz_scale, int N, int Vp) {
+  if (is_bf16 && Vp % 8 == 0 && ld % 8 == 0) {
+    const int v8 = Vp / 8;
+    dim3 grid(cdiv(v8, 256), N);
+    ce_dz_bf16x8_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<uint4*>(logits), ld / 8, lse, targets, dz_scale, v8);
+  } else {
+    dim3 grid(cdiv(Vp, 256), N);
+    if (is_bf16) ce_dz_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<bf16*>(logits), ld, lse, targets, dz_scale, Vp);
+    else ce_dz_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<float*>(logits), ld, lse, targets, dz_scale, Vp);
+  }
+  note_kernel_launches(1);
+  return ok();
+}
+
+size_t encoder_bwd_part_floats(int N, int C) { return (size_t)cdiv(N, ENC_CHUNK) * 2 * (size_t)C; }
+
+int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float* dwte, float* dwpe, int B, int T,
+                       int C, uint32_t* sorted_keys, float* chunk_part, int V) {
+  const int N = B * T;
+  if (N > (1 << ENC_POS_BITS) || V > (1 << (32 - ENC_POS_BITS)) || C % 4) return -4;
+  int P = 1;
+  while (P < N) P <<= 1;
+  const int smem = P * (int)sizeof(uint32_t);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(enc_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return -3;
+  enc_sort_kernel<<<1, 1024, smem, st>>>(tok, N, V, P, sorted_keys);
+  const int nchunks = cdiv(N, ENC_CHUNK);
+  dim3 grid(nchunks, cdiv(C, 128));
+  enc_chunk_kernel<<<grid, 32, 0, st>>>(sorted_keys, dx0, dwte, chunk_part, N, C);
+  enc_fixup_kernel<<<grid, 32, 0, st>>>(sorted_keys, dwte, chunk_part, N, C, nchunks);
+  dwpe_kernel<<<grid_for((long long)T * C, 256), 256, 0, st>>>(dx0, dwpe, B, T, C);
+  note_kernel_launches(4);
+  return ok();
+}
+
+int launch_global_norm(cudaStream_t st, const float* g, long long n, double* part, int nparts, float clip,
+                       float* out2) {
+  sumsq_kernel<<<nparts, 512, 0, st>>>(g, n, part);
+  norm_finalize_kernel<<<1, 256, 0, st>>>(part, nparts, clip, out2);
+  note_kernel_launches(2);
+  return ok();
+}
+
+int launch_adamw(cudaStream_t st, float* p, const float* g, float* m, float* v, uint16_t* shadow,
+                 const AdamBlock* blocks, int nblocks, const float* clip_scale, float lr, float b1, float b2,
+                 float eps, float wd, float bc1, float bc2) {
+  adamw_kernel<<<nblocks, 256, 0, st>>>(p, g, m, v, reinterpret_cast<bf16*>(shadow), blocks, clip_scale, lr, b1, b2,
+                                        eps, wd, bc1, bc2);
+  note_kernel_launches(1);
+  return ok();
+}
+
+int launch_init_normal(cudaStream_t st, float* p, long long n, uint64_t state, double std) {
+  init_normal_kernel<<<grid_for(n, 256), 256, 0, st>>>(p, n, state, std);
+  note_kernel_launches(1);
+  return ok();
+}
+int launch_fill(cudaStream_t st, float* p, long long n, float value) {
+  fill_kernel<<<grid_for(n, 256), 256, 0, st>>>(p, n, value);
+  note_kernel_launches(1);
+  return ok();
+}
+int launch_cast_bf16(cudaStream_t st, const float* src, uint16_t* dst, long long n) {
+  cast_bf16_kernel<<<grid_for(n, 256), 256, 0, st>>>(src, reinterpret_cast<bf16*>(dst), n);
+  note_kernel_launches(1);
+  return ok();
+}

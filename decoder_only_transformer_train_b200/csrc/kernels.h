@@ -1,0 +1,51 @@
+// Host launchers of the memory-bound kernels of the training step.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include "gemm.h"
+
+struct AdamBlock {      // one block of the multi-tensor AdamW launch
+  long long off;        // first element (flat parameter index)
+  int n;                // elements in this block
+  int decay;            // 1 if weight decay applies to this tensor
+};
+
+// act = float (fp32 mode) or bf16 (bf16 mode), chosen by `bf16`.
+int launch_encoder_fwd(cudaStream_t st, const int* tok, const float* wte, const float* wpe, float* x, int N, int T,
+                       int C, int V);
+int launch_layernorm_fwd(cudaStream_t st, bool bf16, const float* x, const float* w, const float* b, void* y,
+                         float* mean, float* rstd, int N, int C);
+int launch_layernorm_bwd(cudaStream_t st, bool bf16, const float* dy, const float* x, const float* mean,
+                         const float* rstd, const float* w, float* dres, void* dres_act, bool accumulate,
+                         float* part, int nblocks, float* dw, float* db, int N, int C);
+int layernorm_bwd_blocks(int num_sms);
+int launch_colsum(cudaStream_t st, bool bf16, const void* x, long long ldx, int M, int N, float* part, int nchunks,
+                  float* out);
+int colsum_chunks(int M);
+int launch_ce_finalize(cudaStream_t st, const CePartial* part, int n_tiles, const float* zt, const int* targets,
+                       int N, int V, float* lse, float* loss_row, int* argmax);
+int launch_ce_rowwise(cudaStream_t st, const float* logits, long long ld, const int* targets, int N, int Vp, int V,
+                      float* lse, float* loss_row, int* argmax);
+int launch_loss_reduce(cudaStream_t st, const float* loss_row, const int* targets, int N, float grad_scale,
+                       float* loss_out, float* dz_scale_out, int* count_out);
+int launch_ce_dz(cudaStream_t st, bool bf16, void* logits, long long ld, const float* lse, const int* targets,
+                 const float* dz_scale, int N, int Vp);
+int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float* dwte, float* dwpe, int B, int T,
+                       int C, uint32_t* sorted_keys, float* chunk_part, int V);
+size_t encoder_bwd_part_floats(int N, int C);
+int launch_global_norm(cudaStream_t st, const float* g, long long n, double* part, int nparts, float clip,
+                       float* out2);
+int launch_adamw(cudaStream_t st, float* p, const float* g, float* m, float* v, uint16_t* shadow,
+                 const AdamBlock* blocks, int nblocks, const float* clip_scale, float lr, float b1, float b2,
+                 float eps, float wd, float bc1, float bc2);
+int launch_init_normal(cudaStream_t st, float* p, long long n, uint64_t state, double std);
+int launch_fill(cudaStream_t st, float* p, long long n, float value);
+int launch_cast_bf16(cudaStream_t st, const float* src, uint16_t* dst, long long n);
+int launch_attn_fwd(cudaStream_t st, bool bf16, const void* qkv, void* out, float* lse, int B, int T, int H,
+                    int hd);
+int launch_attn_bwd(cudaStream_t st, bool bf16, const void* qkv, const void* out, const void* dout,
+                    const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd);
+int read_and_clear_device_error(int* code);
+// Host-side count of the kernels launched by this library (for benchmark reporting).
+void note_kernel_launches(int n);
+long long kernel_launch_count();

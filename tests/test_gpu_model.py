@@ -1,0 +1,211 @@
+"""Model-level parity on a B200: the whole training step through the C ABI against the
+CPU oracle on the same seeded inputs and weights.
+
+Tolerances: fp32 mode - loss 1e-4 relative, per-tensor gradients and updated weights
+1e-4 relative L2; bf16 mode - loss 2e-2 absolute, per-tensor gradient relative L2 2e-2;
+token gathers, masks and the argmax bit-exact (argmax on rows whose reference top-2 gap
+exceeds the bf16 logit error)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from decoder_only_transformer_train_b200 import binding as BD
+from decoder_only_transformer_train_b200 import synthetic as S
+from gpu_common import cuda_i32, rel_l2, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+TINY = O.TINY   # L=2, C=64, H=4, T=64, V=512
+
+
+def _bd_config(cfg: O.Config, B: int, k: int, prec: int) -> BD.Config:
+    return BD.Config(n_layer=cfg.n_layer, n_embd=cfg.n_embd, n_head=cfg.n_head, block_size=cfg.block_size,
+                     vocab_size=cfg.vocab_size, padded_vocab_size=cfg.padded_vocab_size, max_batch=B,
+                     grad_accum_steps=k, precision=prec)
+
+
+def _per_tensor(flat_gpu: np.ndarray, ref: dict, cfg: O.Config):
+    got = O.unflatten(torch.from_numpy(flat_gpu).double(), cfg)
+    return {n: rel_l2(got[n], ref[n]) for n, _ in O.param_specs(cfg)}
+
+
+def _run_step(cfg, prec, B, T, k=1, seed_w=1, seed_d=2, lr=6e-4):
+    """One optimizer step over k micro-batches on the GPU and in the oracle (fp64)."""
+    params = O.init_params(cfg, seed_w, dtype=torch.float64)
+    flat = O.flatten(params, cfg).numpy().astype(np.float32)
+    params = O.unflatten(torch.from_numpy(flat).double(), cfg)     # oracle starts from the same fp32 values
+    batches = [S.token_batch(seed_d, B, T, cfg.vocab_size, micro_step=i) for i in range(k)]
+    model = BD.GPT2(_bd_config(cfg, B, k, prec), seed=seed_w)
+    model.set_params(flat)
+    model.zero_grad()
+    losses = []
+    for x, y in batches:
+        losses.append(model.forward(cuda_i32(x), cuda_i32(y)))
+        model.backward()
+    grads_gpu = model.get_grads()
+    norm_gpu = model.adamw_step(lr)
+    params_gpu = model.get_params()
+    argmax_gpu = model.get_argmax(B * T)
+    model.close()
+    m = {n: torch.zeros_like(t) for n, t in params.items()}
+    v = {n: torch.zeros_like(t) for n, t in params.items()}
+    p_ref = {n: t.clone() for n, t in params.items()}
+    tb = [(torch.from_numpy(x), torch.from_numpy(y)) for x, y in batches]
+    loss_ref, norm_ref, grads_ref = O.train_step(p_ref, m, v, 1, cfg, tb, lr)
+    _, cache = O.forward(params, cfg, *tb[-1])
+    return dict(losses=losses, loss_ref=loss_ref, grads_gpu=grads_gpu, grads_ref=grads_ref, norm_gpu=norm_gpu,
+                norm_ref=norm_ref, params_gpu=params_gpu, params_ref=p_ref, params0=params,
+                argmax_gpu=argmax_gpu, logits_ref=cache["logits"])
+
+
+def test_init_matches_oracle_generator():
+    cfg = TINY
+    model = BD.GPT2(_bd_config(cfg, 2, 1, BD.GPT2_FP32), seed=1234)
+    got = model.get_params()
+    model.close()
+    ref = O.flatten(O.init_params(cfg, 1234, dtype=torch.float32), cfg).numpy()
+    assert got.shape == ref.shape
+    close = np.isclose(got, ref, rtol=2e-7, atol=0)
+    assert close.mean() > 0.9999 and np.array_equal(got[ref == 1.0], ref[ref == 1.0])
+    assert np.max(np.abs(got - ref)) < 1e-6
+
+
+def test_tiny_fp32_step_matches_oracle():
+    r = _run_step(TINY, BD.GPT2_FP32, B=2, T=64)
+    assert abs(r["losses"][0] - r["loss_ref"]) <= 1e-4 * abs(r["loss_ref"])
+    errs = _per_tensor(r["grads_gpu"], r["grads_ref"], TINY)
+    assert max(errs.values()) < 1e-4, {k: v for k, v in errs.items() if v >= 1e-4}
+    assert abs(r["norm_gpu"] - r["norm_ref"]) <= 1e-4 * r["norm_ref"]
+    werr = _per_tensor(r["params_gpu"], r["params_ref"], TINY)
+    assert max(werr.values()) < 1e-4
+    # the update itself (p1 - p0), a stricter view of the same check
+    p0 = O.flatten(r["params0"], TINY).numpy()
+    d_gpu = O.unflatten(torch.from_numpy(r["params_gpu"] - p0).double(), TINY)
+    d_ref = {n: r["params_ref"][n] - r["params0"][n] for n in d_gpu}
+    derr = {n: rel_l2(d_gpu[n], d_ref[n]) for n in d_gpu}
+    assert max(derr.values()) < 1e-2, derr
+
+
+def test_tiny_bf16_step_matches_oracle():
+    r = _run_step(TINY, BD.GPT2_BF16, B=2, T=64)
+    assert abs(r["losses"][0] - r["loss_ref"]) < 2e-2
+    errs = _per_tensor(r["grads_gpu"], r["grads_ref"], TINY)
+    assert max(errs.values()) < 2e-2, {k: v for k, v in errs.items() if v >= 2e-2}
+    z = r["logits_ref"]
+    top2 = torch.topk(z, 2, dim=1).values
+    clear = (top2[:, 0] - top2[:, 1]) > 0.05
+    assert torch.equal(torch.from_numpy(r["argmax_gpu"]).long()[clear], O.argmax_lowest(z).long()[clear])
+
+
+def test_grad_accumulation_fp32_equals_one_batch():
+    cfg = TINY
+    flat = O.flatten(O.init_params(cfg, 5, dtype=torch.float32), cfg).numpy()
+    x, y = S.token_batch(6, 4, 32, cfg.vocab_size)
+    big = BD.GPT2(_bd_config(cfg, 4, 1, BD.GPT2_FP32), seed=5)
+    big.set_params(flat)
+    big.zero_grad()
+    big.forward(cuda_i32(x), cuda_i32(y))
+    big.backward()
+    g_big = big.get_grads()
+    big.close()
+    acc = BD.GPT2(_bd_config(cfg, 2, 2, BD.GPT2_FP32), seed=5)
+    acc.set_params(flat)
+    acc.zero_grad()
+    for i in range(2):
+        acc.forward(cuda_i32(x[2 * i:2 * i + 2]), cuda_i32(y[2 * i:2 * i + 2]))
+        acc.backward()
+    g_acc = acc.get_grads()
+    acc.close()
+    assert rel_l2(g_acc, g_big) < 1e-5
+
+
+def test_bf16_step_is_deterministic():
+    cfg = TINY
+    outs = []
+    for _ in range(2):
+        model = BD.GPT2(_bd_config(cfg, 2, 1, BD.GPT2_BF16), seed=9)
+        x, y = S.token_batch(10, 2, 64, cfg.vocab_size)
+        model.zero_grad()
+        model.forward(cuda_i32(x), cuda_i32(y))
+        model.backward()
+        outs.append(model.get_grads())
+        model.close()
+    assert np.array_equal(outs[0], outs[1])
+
+
+def test_error_paths_return_codes_without_trapping():
+    cfg = TINY
+    model = BD.GPT2(_bd_config(cfg, 2, 1, BD.GPT2_BF16), seed=1)
+    x, y = S.token_batch(2, 2, 64, cfg.vocab_size)
+    with pytest.raises(BD.Gpt2Error) as e:
+        model.backward()                                   # no forward yet
+    assert e.value.code == -8
+    with pytest.raises(BD.Gpt2Error) as e:
+        model.forward(cuda_i32(np.zeros((3, 64))), None)   # B > max_batch
+    assert e.value.code == -4
+    with pytest.raises(BD.Gpt2Error) as e:
+        model.forward(cuda_i32(np.zeros((2, 65))), None)   # T > block_size
+    assert e.value.code == -4
+    bad = x.copy()
+    bad[1, 5] = cfg.vocab_size + 3
+    with pytest.raises(BD.Gpt2Error) as e:
+        model.forward(cuda_i32(bad), cuda_i32(y))
+    assert e.value.code == -5
+    badt = y.copy()
+    badt[0, 0] = -7
+    with pytest.raises(BD.Gpt2Error) as e:
+        model.forward(cuda_i32(x), cuda_i32(badt))
+    assert e.value.code == -6
+    # the context stays usable after reported errors
+    loss = model.forward(cuda_i32(x), cuda_i32(y))
+    assert abs(loss - math.log(cfg.padded_vocab_size)) < 0.2
+    model.close()
+
+
+def test_ignore_index_rows_are_left_out():
+    cfg = TINY
+    x, y = S.token_batch(2, 2, 64, cfg.vocab_size)
+    y = y.copy()
+    y[0, ::3] = -1
+    params = O.init_params(cfg, 1, dtype=torch.float64)
+    loss_ref, _ = O.forward(params, cfg, torch.from_numpy(x), torch.from_numpy(y))
+    model = BD.GPT2(_bd_config(cfg, 2, 1, BD.GPT2_FP32), seed=1)
+    model.set_params(O.flatten(params, cfg).numpy().astype(np.float32))
+    loss = model.forward(cuda_i32(x), cuda_i32(y))
+    model.close()
+    assert abs(loss - float(loss_ref)) <= 1e-4 * float(loss_ref)
+
+
+@pytest.mark.slow
+def test_gpt2_124m_bf16_step_matches_fp32_oracle():
+    """GPT-2 124M, B=4, T=1024: one bf16 forward + backward against the fp32 oracle."""
+    cfg = O.GPT2_124M
+    B, T = 4, 1024
+    params = O.init_params(cfg, 1, dtype=torch.float32)
+    x, y = S.token_batch(2, B, T, cfg.vocab_size)
+    model = BD.GPT2(_bd_config(cfg, B, 1, BD.GPT2_BF16), seed=1)
+    model.set_params(O.flatten(params, cfg).numpy())
+    model.zero_grad()
+    loss = model.forward(cuda_i32(x), cuda_i32(y))
+    model.backward()
+    grads = model.get_grads()
+    am = model.get_argmax(B * T)
+    model.close()
+    loss_ref, cache = O.forward(params, cfg, torch.from_numpy(x), torch.from_numpy(y))
+    grads_ref = O.backward(params, cfg, cache)
+    assert abs(loss - float(loss_ref)) < 2e-2
+    errs = _per_tensor(grads, grads_ref, cfg)
+    assert max(errs.values()) < 2e-2, sorted(errs.items(), key=lambda kv: -kv[1])[:5]
+    z = cache["logits"]
+    top2 = torch.topk(z, 2, dim=1).values
+    clear = (top2[:, 0] - top2[:, 1]) > 0.05
+    assert torch.equal(torch.from_numpy(am).long()[clear], O.argmax_lowest(z).long()[clear])
