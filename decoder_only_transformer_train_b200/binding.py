@@ -63,6 +63,8 @@ _PROTOS = {
     "gpt2op_classifier_aux_floats": (_i64, [_i, _i]),
     "gpt2op_classifier_fwd_bwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "gpt2op_device_error": (_i, []),
+    "gpt2_lr_cosine": (ctypes.c_double, [_i64, ctypes.c_double, _i64, _i64, ctypes.c_double]),
+    "gpt2_kernel_launches": (_i64, []),
     "gpt2_profile_start": (_i, [_vp]),
     "gpt2_profile_stop": (_i, [_vp, _vp, _vp, _vp, _vp]),
 }

@@ -72,3 +72,12 @@ def test_no_host_api_rejects_bad_config_without_gpu(libpath):
     assert lib.gpt2_create(ctypes.byref(bad), 1, ctypes.byref(h)) == -4
     assert not h.value
     assert lib.gpt2_create(None, 1, ctypes.byref(h)) == -1
+
+
+def test_lr_schedule_host_function_matches_oracle(libpath):
+    import oracle as O
+    from decoder_only_transformer_train_b200 import binding
+    lib = binding.load(libpath)
+    for it in (0, 1, 100, 714, 715, 716, 1000, 5000, 19072, 19073, 19074, 25000):
+        got = lib.gpt2_lr_cosine(it, 6e-4, 715, 19073, 0.1)
+        assert abs(got - O.get_lr(it)) <= 1e-15, it
