@@ -276,6 +276,21 @@ def test_forward_backward_against_autograd_formulation():
         assert err < 1e-10, (n, err)
 
 
+def test_key_bias_gradient_is_zero_by_softmax_shift_invariance():
+    """Adding a vector b to every key adds q.b to all scores of a query; the softmax
+    ignores a constant shift, so d loss / d (key bias) = 0 exactly."""
+    cfg = SMALL
+    p = _perturbed_params(cfg)
+    x, y = _batch(cfg)
+    _, cache = O.forward(p, cfg, x, y)
+    g = O.backward(p, cfg, cache)
+    C = cfg.n_embd
+    for l in range(cfg.n_layer):
+        b = g[f"h.{l}.attn.c_attn.bias"]
+        assert float(b[C:2 * C].abs().max()) < 1e-12 * float(b.abs().max())
+        assert float(b[:C].abs().max()) > 0 and float(b[2 * C:].abs().max()) > 0
+
+
 def test_finite_differences_every_tensor():
     cfg = SMALL
     p = _perturbed_params(cfg, seed=3)
