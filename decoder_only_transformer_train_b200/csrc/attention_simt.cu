@@ -270,9 +270,18 @@ int launch_attn_bwd_simt(cudaStream_t st, bool is_bf16, const void* qkv, const v
 
 int launch_attn_fwd(cudaStream_t st, bool is_bf16, const void* qkv, void* out, float* lse, int B, int T, int H,
                     int hd) {
+  if (is_bf16 && hd == 64) return launch_attn_fwd_tc(st, qkv, out, lse, B, T, H, hd);
   return launch_attn_fwd_simt(st, is_bf16, qkv, out, lse, B, T, H, hd);
 }
 int launch_attn_bwd(cudaStream_t st, bool is_bf16, const void* qkv, const void* out, const void* dout,
                     const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd) {
+  if (is_bf16 && hd == 64) {
+    dim3 gD(cdiv(T * H, 8), B);
+    attn_bwd_D<bf16><<<gD, 256, 0, st>>>(reinterpret_cast<const bf16*>(out), reinterpret_cast<const bf16*>(dout),
+                                         Dbuf, T, H, hd);
+    note_kernel_launches(1);
+    if (cudaGetLastError() != cudaSuccess) return -3;
+    return launch_attn_bwd_tc(st, qkv, dout, lse, Dbuf, dqkv, B, T, H, hd);
+  }
   return launch_attn_bwd_simt(st, is_bf16, qkv, out, dout, lse, Dbuf, dqkv, B, T, H, hd);
 }

@@ -1,0 +1,650 @@
+// Causal flash-attention forward on the sm_100a tensor cores (head size 64, bf16).
+//
+// "Karpathy's Zero to Hero, Lecture 9" notes, "2:00:19 – 2:06:39 FlashAttention": the
+// scores, mask, softmax and weighted sum fused in one kernel that never writes the T x T
+// matrix, using the online softmax (running max and sum).
+//
+// One CTA per (batch, head, 128-query tile), heaviest (latest) query tiles first.
+//   warp 0      : TMA producer - Q once, then K_j / V_j tiles of 128 keys (3 stages),
+//                 all straight out of the qkv activation [B*T, 3C]
+//   warp 1      : TMEM allocator + MMA issuer:  S_j = Q K_j^T  (128 x 128, TMEM)
+//                                                O_j = P_j V_j  (128 x 64,  TMEM)
+//   warps 2..5  : softmax - thread r owns query row r (= TMEM lane r): reads S_j, applies
+//                 the causal mask, updates the running max / sum, writes P_j (bf16) to
+//                 shared memory in the 128-byte-swizzled K-major layout the MMA reads,
+//                 and folds O_j into its register accumulator with the rescale factor.
+// S and O are double-buffered in TMEM (2 x 128 + 2 x 64 columns), P in shared memory, so
+// the MMA of S_{j+1} overlaps the softmax of S_j.
+#include <math.h>
+#include "sm100.cuh"
+#include "kernels.h"
+
+namespace {
+
+constexpr int QT = 128;          // queries per CTA
+constexpr int KT = 128;          // keys per tile
+constexpr int HD = 64;
+constexpr int KV_STAGES = 3;
+constexpr int NUM_THREADS = 192;
+constexpr int TILE_BYTES = KT * HD * 2;        // 16 KB: one Q, K or V tile
+constexpr int P_BYTES = QT * KT * 2;           // 32 KB
+constexpr int SMEM_BYTES = TILE_BYTES + 2 * KV_STAGES * TILE_BYTES + 2 * P_BYTES + 512 + 1024;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t S_COL = 0;                  // S buffers: columns [0, 256)
+constexpr uint32_t O_COL = 256;                // O buffers: columns [256, 384)
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
+                   int B, int T, int H, float scale_log2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + TILE_BYTES;
+  uint8_t* sV = sK + KV_STAGES * TILE_BYTES;
+  uint8_t* sP = sV + KV_STAGES * TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * P_BYTES);
+  uint64_t* q_full = bars;                       // 1
+  uint64_t* kv_full = bars + 1;                  // KV_STAGES
+  uint64_t* kv_empty = kv_full + KV_STAGES;      // KV_STAGES
+  uint64_t* s_full = kv_empty + KV_STAGES;       // 2
+  uint64_t* s_empty = s_full + 2;                // 2
+  uint64_t* p_full = s_empty + 2;                // 2
+  uint64_t* p_empty = p_full + 2;                // 2
+  uint64_t* o_full = p_empty + 2;                // 2
+  uint64_t* o_empty = o_full + 2;                // 2
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_qt = cdiv(T, QT);
+  const int BH = B * H;
+  const int qt = n_qt - 1 - (int)(blockIdx.x / BH);     // heaviest tiles first
+  const int bh = (int)(blockIdx.x % BH);
+  const int b = bh / H, h = bh % H;
+  const int C = H * HD;
+  const int q0 = qt * QT;
+  const int row0 = b * T;                               // first token row of this sequence
+  const int n_kv = qt + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], 128);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&p_empty[i], 1);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&o_empty[i], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      mbar_arrive_expect_tx(q_full, TILE_BYTES);
+      tma_load_2d(sQ, &tm_qkv, h * HD, row0 + q0, q_full);
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % KV_STAGES;
+        if (!mbar_wait(&kv_empty[s], ((j / KV_STAGES) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * TILE_BYTES);
+        tma_load_2d(sK + s * TILE_BYTES, &tm_qkv, C + h * HD, row0 + j * KT, &kv_full[s]);
+        tma_load_2d(sV + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + j * KT, &kv_full[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_s = make_idesc_bf16(QT, KT, false, false);   // Q, K both K-major
+      constexpr uint32_t idesc_o = make_idesc_bf16(QT, HD, false, true);    // P K-major, V MN-major
+      const uint32_t aQ = smem_u32(sQ);
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % KV_STAGES;
+        if (!mbar_wait(&kv_full[s], (j / KV_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait(&s_empty[j & 1], ((j >> 1) & 1) ^ 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t bK = smem_u32(sK + s * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k)
+          tc_mma_bf16(tmem + S_COL + (j & 1) * KT, make_sdesc_sw128(aQ + k * 32, 16, 1024),
+                      make_sdesc_sw128(bK + k * 32, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
+        tc_commit(&s_full[j & 1]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        if (j + 1 < n_kv && !issue_s(j + 1)) break;
+        const int s = j % KV_STAGES;
+        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag)) break;
+        if (!mbar_wait(&o_empty[j & 1], ((j >> 1) & 1) ^ 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t aP = smem_u32(sP + (j & 1) * P_BYTES);
+        const uint32_t bV = smem_u32(sV + s * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < KT / 16; ++k)
+          tc_mma_bf16(tmem + O_COL + (j & 1) * HD, make_sdesc_sw128(aP + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                      make_sdesc_sw128(bV + k * 2048, 8192, 1024), idesc_o, k > 0 ? 1u : 0u);
+        tc_commit(&o_full[j & 1]);
+        tc_commit(&kv_empty[s]);
+        tc_commit(&p_empty[j & 1]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                 // query row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    float m = -INFINITY, l = 0.f, alpha_pending = 1.f;
+    float o[HD];
+#pragma unroll
+    for (int d = 0; d < HD; ++d) o[d] = 0.f;
+    bool ok = true;
+
+    auto fold_o = [&](int i) -> bool {          // o = o * alpha_i + O_i
+      if (!mbar_wait(&o_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < HD; c += 32) {
+        tmem_ld32(tmem + lane_off + O_COL + (i & 1) * HD + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int d = 0; d < 32; ++d) o[c + d] = o[c + d] * alpha_pending + __uint_as_float(v[d]);
+      }
+      tc_fence_before();
+      mbar_arrive(&o_empty[i & 1]);
+      return true;
+    };
+
+    for (int j = 0; j < n_kv && ok; ++j) {
+      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float s[KT];
+#pragma unroll
+      for (int c = 0; c < KT; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + S_COL + (j & 1) * KT + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int d = 0; d < 32; ++d) s[c + d] = __uint_as_float(v[d]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_empty[j & 1]);              // S_j is in registers: the MMA may reuse it
+      const bool diag = (j == qt);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < KT; ++c) {
+        if (diag && c > r) s[c] = -INFINITY;     // key j*KT+c after query q0+r
+        mx = fmaxf(mx, s[c]);
+      }
+      const float m_new = fmaxf(m, mx * scale_log2);
+      const float alpha = ex2(m - m_new);
+      float sum = 0.f;
+      // P_j must not overwrite the buffer the MMA of O_{j-2} is still reading
+      if (!mbar_wait(&p_empty[j & 1], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      uint8_t* prow = sP + (j & 1) * P_BYTES + r * 128;
+#pragma unroll
+      for (int g = 0; g < KT / 8; ++g) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[e] = ex2(s[g * 8 + e] * scale_log2 - m_new);
+          sum += p[e];
+        }
+        uint4 w;
+        w.x = pack_bf16x2(p[0], p[1]);
+        w.y = pack_bf16x2(p[2], p[3]);
+        w.z = pack_bf16x2(p[4], p[5]);
+        w.w = pack_bf16x2(p[6], p[7]);
+        const int chunk = g >> 3, gi = g & 7;
+        *reinterpret_cast<uint4*>(prow + chunk * 16384 + ((gi ^ (r & 7)) << 4)) = w;
+      }
+      fence_async_smem();
+      mbar_arrive(&p_full[j & 1]);
+      l = l * alpha + sum;
+      m = m_new;
+      if (j > 0 && !fold_o(j - 1)) { ok = false; break; }
+      alpha_pending = alpha;
+    }
+    if (ok) ok = fold_o(n_kv - 1);
+    const int qi = q0 + r;
+    if (ok && qi < T) {
+      const float inv = 1.0f / l;
+      bf16* orow = out + (long long)(row0 + qi) * C + h * HD;
+#pragma unroll
+      for (int g = 0; g < HD / 8; ++g) {
+        uint4 w;
+        w.x = pack_bf16x2(o[g * 8 + 0] * inv, o[g * 8 + 1] * inv);
+        w.y = pack_bf16x2(o[g * 8 + 2] * inv, o[g * 8 + 3] * inv);
+        w.z = pack_bf16x2(o[g * 8 + 4] * inv, o[g * 8 + 5] * inv);
+        w.w = pack_bf16x2(o[g * 8 + 6] * inv, o[g * 8 + 7] * inv);
+        reinterpret_cast<uint4*>(orow)[g] = w;
+      }
+      lse[(long long)bh * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+typedef CUresult (*PFN_encode)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+PFN_encode encode_fn() {
+  static PFN_encode fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encode>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+// Tensor-core forward for head size 64 in bf16; returns -4 when the shape is not covered.
+int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, int B, int T, int H, int hd) {
+  if (hd != HD) return -4;
+  const int C = H * HD;
+  PFN_encode fn = encode_fn();
+  if (fn == nullptr) return -3;
+  if ((reinterpret_cast<uintptr_t>(qkv) & 15) != 0) return -1;
+  CUtensorMap tm;
+  cuuint64_t dims[2] = {(cuuint64_t)(3 * C), (cuuint64_t)B * T};
+  cuuint64_t strides[1] = {(cuuint64_t)(3 * C) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(qkv), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return -3;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
+        cudaSuccess)
+      return -3;
+    attr = true;
+  }
+  const int grid = cdiv(T, QT) * B * H;
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, reinterpret_cast<bf16*>(out), lse, B, T, H,
+                                                            scale_log2);
+  note_kernel_launches(1);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+// ============================================================================ backward
+// Gradients of the causal attention with the probabilities recomputed from the saved
+// log-sum-exp (scaled scores z = q.k / sqrt(hd), P = softmax(z), D = rowsum(dO * O)):
+//   dV = P^T dO,   dZ = P * (dO V^T - D),   dQ = dZ K / sqrt(hd),   dK = dZ^T Q / sqrt(hd).
+// Two kernels keep every sum in a fixed order (no atomics): one CTA per 128-key tile
+// accumulates dK and dV over the query tiles at or after it, one CTA per 128-query tile
+// accumulates dQ over the key tiles at or before it.
+namespace {
+
+constexpr int BWD_THREADS = 192;
+constexpr int BWD_STAGES = 2;
+// smem: 2 resident tiles (K_j,V_j or Q_i,dO_i) + BWD_STAGES x 2 streamed tiles + 2 P-like
+// 128x128 bf16 operands + per-row scalars + barriers
+constexpr int BWD_SMEM = 2 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + 2 * BWD_STAGES * 512 + 512 + 1024;
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Writes 32 bf16 values (columns col0 .. col0+31, col0 a multiple of 32) into row r of a
+// 128 x 128 K-major operand stored as two 64-column chunks of 128-byte swizzled rows.
+__device__ __forceinline__ void store_32_sw128(uint8_t* base, int r, int col0, const float* v) {
+  uint8_t* row = base + (col0 >> 6) * 16384 + r * 128;
+  const int g0 = (col0 & 63) >> 3;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint4 w;
+    w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+    w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+    w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+    w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+    *reinterpret_cast<uint4*>(row + (((g0 + g) ^ (r & 7)) << 4)) = w;
+  }
+}
+
+// MODE 0: dK/dV kernel (CTA = key tile j; streams Q_i, dO_i for i >= j)
+// MODE 1: dQ kernel    (CTA = query tile i; streams K_j, V_j for j <= i)
+template <int MODE>
+__global__ void __launch_bounds__(BWD_THREADS, 1)
+attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+                   const float* __restrict__ lse, const float* __restrict__ Dbuf, bf16* __restrict__ dqkv, int B,
+                   int T, int H, float scale, float scale_log2) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sR0 = smem;                                   // resident: K_j (MODE 0) / Q_i (MODE 1)
+  uint8_t* sR1 = sR0 + TILE_BYTES;                       // resident: V_j (MODE 0) / dO_i (MODE 1)
+  uint8_t* sA = sR1 + TILE_BYTES;                        // streamed: Q_i (MODE 0) / K_j (MODE 1)
+  uint8_t* sB = sA + BWD_STAGES * TILE_BYTES;            // streamed: dO_i (MODE 0) / V_j (MODE 1)
+  uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P^T (MODE 0) ; unused (MODE 1)
+  uint8_t* sDS = sP + P_BYTES;                           // dZ^T (MODE 0) / dZ (MODE 1)
+  float* sRow = reinterpret_cast<float*>(sDS + P_BYTES); // [BWD_STAGES][2][128]: lse2 and D per streamed tile
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sRow + BWD_STAGES * 256);
+  uint64_t* r_full = bars;                               // resident tiles loaded
+  uint64_t* t_full = bars + 1;                           // [BWD_STAGES]
+  uint64_t* t_empty = t_full + BWD_STAGES;               // [BWD_STAGES]
+  uint64_t* sd_full = t_empty + BWD_STAGES;              // S and dP in TMEM
+  uint64_t* sd_empty = sd_full + 1;                      // S and dP read out
+  uint64_t* ps_full = sd_empty + 1;                      // operands in smem
+  uint64_t* ps_empty = ps_full + 1;                      // operands consumed
+  uint64_t* acc_full = ps_empty + 1;                     // accumulation done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_t = cdiv(T, 128);
+  const int BH = B * H;
+  // heaviest CTAs first: key tile 0 (MODE 0) / the last query tile (MODE 1) loop longest
+  const int tile = (MODE == 0) ? (int)(blockIdx.x / BH) : n_t - 1 - (int)(blockIdx.x / BH);
+  const int bh = (int)(blockIdx.x % BH);
+  const int b = bh / H, h = bh % H;
+  const int C = H * HD;
+  const int row0 = b * T;
+  const int it0 = (MODE == 0) ? tile : 0;                // streamed tiles [it0, it1)
+  const int it1 = (MODE == 0) ? n_t : tile + 1;
+  const int n_it = it1 - it0;
+  // TMEM columns: S [0,128), dP [128,256), acc0 [256,320) (dV or dQ), acc1 [320,384) (dK)
+  const uint32_t S_C = 0, DP_C = 128, A0_C = 256, A1_C = 320;
+
+  if (threadIdx.x == 0) {
+    mbar_init(r_full, 1);
+    for (int s = 0; s < BWD_STAGES; ++s) {
+      mbar_init(&t_full[s], 1);
+      mbar_init(&t_empty[s], 1);
+    }
+    mbar_init(sd_full, 1);
+    mbar_init(sd_empty, 128);
+    mbar_init(ps_full, 128);
+    mbar_init(ps_empty, 1);
+    mbar_init(acc_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- TMA producer
+      mbar_arrive_expect_tx(r_full, 2 * TILE_BYTES);
+      if (MODE == 0) {
+        tma_load_2d(sR0, &tm_qkv, C + h * HD, row0 + tile * 128, r_full);       // K_j
+        tma_load_2d(sR1, &tm_qkv, 2 * C + h * HD, row0 + tile * 128, r_full);   // V_j
+      } else {
+        tma_load_2d(sR0, &tm_qkv, h * HD, row0 + tile * 128, r_full);           // Q_i
+        tma_load_2d(sR1, &tm_do, h * HD, row0 + tile * 128, r_full);            // dO_i
+      }
+      for (int n = 0; n < n_it; ++n) {
+        const int s = n % BWD_STAGES;
+        const int t = it0 + n;
+        if (!mbar_wait(&t_empty[s], ((n / BWD_STAGES) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&t_full[s], 2 * TILE_BYTES);
+        if (MODE == 0) {
+          tma_load_2d(sA + s * TILE_BYTES, &tm_qkv, h * HD, row0 + t * 128, &t_full[s]);      // Q_i
+          tma_load_2d(sB + s * TILE_BYTES, &tm_do, h * HD, row0 + t * 128, &t_full[s]);       // dO_i
+        } else {
+          tma_load_2d(sA + s * TILE_BYTES, &tm_qkv, C + h * HD, row0 + t * 128, &t_full[s]);  // K_j
+          tma_load_2d(sB + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + t * 128, &t_full[s]);  // V_j
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------------------------------------------------------- MMA issuer
+      constexpr uint32_t idesc_sq = make_idesc_bf16(128, 128, false, false);   // 128x128, K=64, both K-major
+      constexpr uint32_t idesc_acc = make_idesc_bf16(128, HD, false, true);    // 128x64, K=128, B MN-major
+      bool ok = mbar_wait(r_full, 0, abort_flag);
+      const uint32_t r0 = smem_u32(sR0), r1 = smem_u32(sR1);
+      auto issue_sd = [&](int n) -> bool {
+        const int s = n % BWD_STAGES;
+        if (!mbar_wait(&t_full[s], (n / BWD_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait(sd_empty, (n & 1) ^ 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t a = smem_u32(sA + s * TILE_BYTES), bq = smem_u32(sB + s * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < HD / 16; ++k) {
+          if (MODE == 0) {
+            // S^T = K_j Q_i^T ; dP^T = V_j dO_i^T
+            tc_mma_bf16(tmem + S_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
+                        idesc_sq, k > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024), make_sdesc_sw128(bq + k * 32, 16, 1024),
+                        idesc_sq, k > 0 ? 1u : 0u);
+          } else {
+            // S = Q_i K_j^T ; dP = dO_i V_j^T
+            tc_mma_bf16(tmem + S_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
+                        idesc_sq, k > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024), make_sdesc_sw128(bq + k * 32, 16, 1024),
+                        idesc_sq, k > 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(sd_full);
+        return true;
+      };
+      if (ok) ok = issue_sd(0);
+      for (int n = 0; n < n_it && ok; ++n) {
+        if (n + 1 < n_it && !issue_sd(n + 1)) break;
+        const int s = n % BWD_STAGES;
+        if (!mbar_wait(ps_full, n & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(sA + s * TILE_BYTES), bq = smem_u32(sB + s * TILE_BYTES);
+        const uint32_t dsA = smem_u32(sDS);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t koff = (k >> 2) * 16384 + (k & 3) * 32;
+          if (MODE == 0) {
+            // dV += P^T dO_i ; dK += dZ^T Q_i   (B operands MN-major: [128 queries x 64])
+            tc_mma_bf16(tmem + A0_C, make_sdesc_sw128(smem_u32(sP) + koff, 16, 1024),
+                        make_sdesc_sw128(bq + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
+            tc_mma_bf16(tmem + A1_C, make_sdesc_sw128(dsA + koff, 16, 1024),
+                        make_sdesc_sw128(a + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
+          } else {
+            // dQ += dZ K_j
+            tc_mma_bf16(tmem + A0_C, make_sdesc_sw128(dsA + koff, 16, 1024),
+                        make_sdesc_sw128(a + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(&t_empty[s]);
+        tc_commit(ps_empty);
+      }
+      if (ok) tc_commit(acc_full);
+    }
+  } else {
+    // ------------------------------------------------------------------ elementwise
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const int tid = threadIdx.x - 64;                    // 0..127 within the elementwise warps
+    const float LOG2E = 1.4426950408889634f;
+    float row_lse2 = 0.f, row_D = 0.f;
+    if (MODE == 1) {
+      const int qi = tile * 128 + r;
+      row_lse2 = (qi < T) ? lse[(long long)bh * T + qi] * LOG2E : 0.f;
+      row_D = (qi < T) ? Dbuf[(long long)bh * T + qi] : 0.f;
+    }
+    bool ok = true;
+    for (int n = 0; n < n_it && ok; ++n) {
+      const int t = it0 + n;
+      const int s = n % BWD_STAGES;
+      float* lse2_s = sRow + s * 256;
+      float* D_s = lse2_s + 128;
+      if (MODE == 0) {
+        // per-query scalars of the streamed query tile
+        const int qi = t * 128 + tid;
+        lse2_s[tid] = (qi < T) ? lse[(long long)bh * T + qi] * LOG2E : 0.f;
+        D_s[tid] = (qi < T) ? Dbuf[(long long)bh * T + qi] : 0.f;
+        named_bar_sync(1, 128);
+      }
+      if (!mbar_wait(sd_full, n & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      // the previous tile's MMAs must be done reading the P / dZ operands
+      if (!mbar_wait(ps_empty, (n & 1) ^ 1, abort_flag)) { ok = false; break; }
+      const bool diag = (t == tile);
+#pragma unroll 1
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t us[32], ud[32];
+        tmem_ld32(tmem + lane_off + S_C + c0, us);
+        tmem_ld32(tmem + lane_off + DP_C + c0, ud);
+        tmem_wait_ld();
+        float pv[32], dz[32];
+#pragma unroll
+        for (int d = 0; d < 32; ++d) {
+          const int c = c0 + d;
+          float p, Dv;
+          bool masked;
+          if (MODE == 0) {           // row r = key, column c = query
+            masked = diag && (c < r);
+            p = ex2(__uint_as_float(us[d]) * scale_log2 - lse2_s[c]);
+            Dv = D_s[c];
+          } else {                   // row r = query, column c = key
+            masked = diag && (c > r);
+            p = ex2(__uint_as_float(us[d]) * scale_log2 - row_lse2);
+            Dv = row_D;
+          }
+          p = masked ? 0.f : p;
+          pv[d] = p;
+          dz[d] = p * (__uint_as_float(ud[d]) - Dv);
+        }
+        if (MODE == 0) store_32_sw128(sP, r, c0, pv);
+        store_32_sw128(sDS, r, c0, dz);
+      }
+      tc_fence_before();
+      mbar_arrive(sd_empty);
+      fence_async_smem();
+      mbar_arrive(ps_full);
+      if (MODE == 0) named_bar_sync(1, 128);   // the scalar buffer of stage s is rewritten two tiles later
+    }
+    // ---- epilogue: accumulators -> dqkv (bf16)
+    if (ok && mbar_wait(acc_full, 0, abort_flag)) {
+      tc_fence_after();
+      const int gi = tile * 128 + r;
+      bf16* row = dqkv + (long long)(row0 + gi) * (3 * C) + h * HD;
+      const int nacc = (MODE == 0) ? 2 : 1;
+      for (int a = 0; a < nacc; ++a) {
+        // MODE 0: a=0 dV (column block 2C), a=1 dK (column block C, times scale); MODE 1: dQ (times scale)
+        const uint32_t col = (a == 0) ? A0_C : A1_C;
+        const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
+        bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C));
+        float v[HD];
+#pragma unroll
+        for (int c = 0; c < HD; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(tmem + lane_off + col + c, u);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < 32; ++d) v[c + d] = __uint_as_float(u[d]) * mul;
+        }
+        if (gi < T) {
+#pragma unroll
+          for (int g = 0; g < HD / 8; ++g) {
+            uint4 w;
+            w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
+            w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
+            w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
+            w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+            reinterpret_cast<uint4*>(dst)[g] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+int encode_rows64(CUtensorMap* tm, const void* base, int cols, long long rows) {
+  PFN_encode fn = encode_fn();
+  if (fn == nullptr) return -3;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return -1;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS ? 0 : -3;
+}
+
+}  // namespace
+
+// Tensor-core backward for head size 64 in bf16 (D = rowsum(dO * O) precomputed).
+int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const float* lse, const float* Dbuf,
+                       void* dqkv, int B, int T, int H, int hd) {
+  if (hd != HD) return -4;
+  const int C = H * HD;
+  CUtensorMap tq, td;
+  int rc = encode_rows64(&tq, qkv, 3 * C, (long long)B * T);
+  if (rc) return rc;
+  rc = encode_rows64(&td, dout, C, (long long)B * T);
+  if (rc) return rc;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(attn_bwd_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, BWD_SMEM) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(attn_bwd_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, BWD_SMEM) !=
+            cudaSuccess)
+      return -3;
+    attr = true;
+  }
+  const int grid = cdiv(T, 128) * B * H;
+  const float scale = 1.0f / sqrtf((float)HD);
+  const float scale_log2 = 1.4426950408889634f * scale;
+  attn_bwd_tc_kernel<0><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv), B, T,
+                                                             H, scale, scale_log2);
+  attn_bwd_tc_kernel<1><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv), B, T,
+                                                             H, scale, scale_log2);
+  note_kernel_launches(2);
+  return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}

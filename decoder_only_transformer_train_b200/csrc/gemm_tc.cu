@@ -112,8 +112,11 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
       for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] + b[j];
       bf16* c = reinterpret_cast<bf16*>(ep.C) + (long long)m * ep.ldc + n0;
       if (full) store_bf16x32(c, v);
-      else
-        for (int j = 0; j < nvalid; ++j) c[j] = __float2bfloat16_rn(v[j]);
+      else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) c[j] = __float2bfloat16_rn(v[j]);
+      }
       break;
     }
     case EPI_STORE_F32: {
@@ -121,8 +124,11 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
       for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] + b[j];
       float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
       if (full) store_f32x32(c, v);
-      else
-        for (int j = 0; j < nvalid; ++j) c[j] = v[j];
+      else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) c[j] = v[j];
+      }
       break;
     }
     case EPI_ACCUM_F32: {
@@ -134,7 +140,9 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
         for (int j = 0; j < 32; ++j) o[j] += alpha * v[j];
         store_f32x32(c, o);
       } else {
-        for (int j = 0; j < nvalid; ++j) c[j] += alpha * v[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) c[j] += alpha * v[j];
       }
       break;
     }
@@ -148,7 +156,9 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
         for (int j = 0; j < 32; ++j) o[j] += alpha * v[j] + b[j];
         store_f32x32(c, o);
       } else {
-        for (int j = 0; j < nvalid; ++j) c[j] = r[j] + alpha * v[j] + b[j];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) c[j] = r[j] + alpha * v[j] + b[j];
       }
       break;
     }
@@ -165,10 +175,12 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
         store_bf16x32(u, v);
         store_bf16x32(c, g);
       } else {
-        for (int j = 0; j < nvalid; ++j) {
-          u[j] = __float2bfloat16_rn(v[j]);
-          c[j] = __float2bfloat16_rn(g[j]);
-        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) {
+            u[j] = __float2bfloat16_rn(v[j]);
+            c[j] = __float2bfloat16_rn(g[j]);
+          }
       }
       break;
     }
@@ -182,8 +194,9 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
         for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_f(uu[j]);
         store_bf16x32(c, v);
       } else {
-        for (int j = 0; j < nvalid; ++j)
-          c[j] = __float2bfloat16_rn(alpha * v[j] * gelu_tanh_grad_f(__bfloat162float(u[j])));
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) c[j] = __float2bfloat16_rn(alpha * v[j] * gelu_tanh_grad_f(__bfloat162float(u[j])));
       }
       break;
     }
@@ -214,15 +227,21 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
         }
       }
       if (full) store_bf16x32(c, v);
-      else
-        for (int j = 0; j < nvalid; ++j) c[j] = __float2bfloat16_rn(v[j]);
+      else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) c[j] = __float2bfloat16_rn(v[j]);
+      }
       break;
     }
     case EPI_SPLITK: {
       float* w = ep.ws + ((long long)split * ep.M + m) * (long long)N + n0;
       if (full && (N % 4 == 0)) store_f32x32(w, v);
-      else
-        for (int j = 0; j < nvalid; ++j) w[j] = v[j];
+      else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) w[j] = v[j];
+      }
       break;
     }
     default:

@@ -45,6 +45,9 @@ int launch_attn_fwd(cudaStream_t st, bool bf16, const void* qkv, void* out, floa
                     int hd);
 int launch_attn_bwd(cudaStream_t st, bool bf16, const void* qkv, const void* out, const void* dout,
                     const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd);
+int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, int B, int T, int H, int hd);
+int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const float* lse, const float* Dbuf,
+                       void* dqkv, int B, int T, int H, int hd);
 int read_and_clear_device_error(int* code);
 // Host-side count of the kernels launched by this library (for benchmark reporting).
 void note_kernel_launches(int n);
