@@ -319,12 +319,8 @@ namespace {
 constexpr int BWD_THREADS = 192;
 constexpr int BWD_STAGES = 2;
 // smem: 2 resident tiles (K_j,V_j or Q_i,dO_i) + BWD_STAGES x 2 streamed tiles + 2 P-like
-// 128x128 bf16 operands + per-row scalars + barriers
-constexpr int BWD_SMEM = 2 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + 2 * BWD_STAGES * 512 + 512 + 1024;
-
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
+// 128x128 bf16 operands + barriers
+constexpr int BWD_SMEM = 2 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + 512 + 1024;
 
 // Writes 32 bf16 values (columns col0 .. col0+31, col0 a multiple of 32) into row r of a
 // 128 x 128 K-major operand stored as two 64-column chunks of 128-byte swizzled rows.
@@ -357,8 +353,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   uint8_t* sB = sA + BWD_STAGES * TILE_BYTES;            // streamed: dO_i (MODE 0) / V_j (MODE 1)
   uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P^T (MODE 0) ; unused (MODE 1)
   uint8_t* sDS = sP + P_BYTES;                           // dZ^T (MODE 0) / dZ (MODE 1)
-  float* sRow = reinterpret_cast<float*>(sDS + P_BYTES); // [BWD_STAGES][2][128]: lse2 and D per streamed tile
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sRow + BWD_STAGES * 256);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + P_BYTES);
   uint64_t* r_full = bars;                               // resident tiles loaded
   uint64_t* t_full = bars + 1;                           // [BWD_STAGES]
   uint64_t* t_empty = t_full + BWD_STAGES;               // [BWD_STAGES]
@@ -500,7 +495,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int tid = threadIdx.x - 64;                    // 0..127 within the elementwise warps
     const float LOG2E = 1.4426950408889634f;
     float row_lse2 = 0.f, row_D = 0.f;
     if (MODE == 1) {
@@ -509,18 +503,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       row_D = (qi < T) ? Dbuf[(long long)bh * T + qi] : 0.f;
     }
     bool ok = true;
+    const float* lse_bh = lse + (long long)bh * T;
+    const float* D_bh = Dbuf + (long long)bh * T;
     for (int n = 0; n < n_it && ok; ++n) {
       const int t = it0 + n;
-      const int s = n % BWD_STAGES;
-      float* lse2_s = sRow + s * 256;
-      float* D_s = lse2_s + 128;
-      if (MODE == 0) {
-        // per-query scalars of the streamed query tile
-        const int qi = t * 128 + tid;
-        lse2_s[tid] = (qi < T) ? lse[(long long)bh * T + qi] * LOG2E : 0.f;
-        D_s[tid] = (qi < T) ? Dbuf[(long long)bh * T + qi] : 0.f;
-        named_bar_sync(1, 128);
-      }
       if (!mbar_wait(sd_full, n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
       // the previous tile's MMAs must be done reading the P / dZ operands
@@ -538,18 +524,19 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
           const int c = c0 + d;
           float p, Dv;
           bool masked;
-          if (MODE == 0) {           // row r = key, column c = query
-            masked = diag && (c < r);
-            p = ex2(__uint_as_float(us[d]) * scale_log2 - lse2_s[c]);
-            Dv = D_s[c];
+          if (MODE == 0) {           // row r = key, column c = query (queries past T are masked)
+            const int qi = t * 128 + c;
+            masked = (diag && (c < r)) || qi >= T;
+            const int qc = masked ? 0 : qi;
+            p = ex2(__uint_as_float(us[d]) * scale_log2 - __ldg(lse_bh + qc) * LOG2E);
+            Dv = __ldg(D_bh + qc);
           } else {                   // row r = query, column c = key
             masked = diag && (c > r);
             p = ex2(__uint_as_float(us[d]) * scale_log2 - row_lse2);
             Dv = row_D;
           }
-          p = masked ? 0.f : p;
-          pv[d] = p;
-          dz[d] = p * (__uint_as_float(ud[d]) - Dv);
+          pv[d] = masked ? 0.f : p;
+          dz[d] = masked ? 0.f : p * (__uint_as_float(ud[d]) - Dv);
         }
         if (MODE == 0) store_32_sw128(sP, r, c0, pv);
         store_32_sw128(sDS, r, c0, dz);
@@ -558,7 +545,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       mbar_arrive(sd_empty);
       fence_async_smem();
       mbar_arrive(ps_full);
-      if (MODE == 0) named_bar_sync(1, 128);   // the scalar buffer of stage s is rewritten two tiles later
     }
     // ---- epilogue: accumulators -> dqkv (bf16)
     if (ok && mbar_wait(acc_full, 0, abort_flag)) {
