@@ -95,23 +95,23 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const float* __restrict__ x
 
 // dx = rstd * (dxhat - mean(dxhat) - xhat * mean(dxhat * xhat)),  dxhat = dy * w;
 // dres = (accumulate ? dres : 0) + dx, also written in the activation type for the next
-// GEMM.  dw = sum_rows dy * xhat and db = sum_rows dy go to per-block partials in a fixed
-// row order (block b owns rows b*8+warp + k*gridDim*8).
+// GEMM.  dw = sum_rows dy * xhat and db = sum_rows dy are accumulated in each warp's own
+// shared-memory slice (fixed row order: block b, warp w owns rows b*8+w + k*gridDim*8),
+// then summed over the 8 warps in order into one partial per block.
 template <typename ActT, int CPL>
-__global__ void __launch_bounds__(256) ln_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
-                                                     const float* __restrict__ mean, const float* __restrict__ rstd,
-                                                     const float* __restrict__ w, float* __restrict__ dres,
-                                                     ActT* __restrict__ dres_act, int accumulate,
-                                                     float* __restrict__ part, int N) {
+__global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
+                                                        const float* __restrict__ mean, const float* __restrict__ rstd,
+                                                        const float* __restrict__ w, float* __restrict__ dres,
+                                                        ActT* __restrict__ dres_act, int accumulate,
+                                                        float* __restrict__ part, int N) {
   constexpr int C = CPL * 32;
   extern __shared__ float red[];   // [8][2C]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float wv[CPL], dwa[CPL], dba[CPL];
+  float* mine = red + warp * 2 * C;
 #pragma unroll
   for (int k = 0; k < CPL; ++k) {
-    wv[k] = w[lane + 32 * k];
-    dwa[k] = 0.f;
-    dba[k] = 0.f;
+    mine[lane + 32 * k] = 0.f;
+    mine[C + lane + 32 * k] = 0.f;
   }
   for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
     const float* dyr = dy + (long long)row * C;
@@ -124,11 +124,11 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const float* __restrict__ d
       const int c = lane + 32 * k;
       const float d = dyr[c];
       xh[k] = (xr[c] - mu) * r;
-      g[k] = d * wv[k];
+      g[k] = d * __ldg(w + c);
       s1 += g[k];
       s2 += g[k] * xh[k];
-      dwa[k] += d * xh[k];
-      dba[k] += d;
+      mine[c] += d * xh[k];
+      mine[C + c] += d;
     }
     s1 = warp_sum(s1) * (1.0f / C);
     s2 = warp_sum(s2) * (1.0f / C);
@@ -142,11 +142,6 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const float* __restrict__ d
       dr[c] = o;
       st_f(da + c, o);
     }
-  }
-#pragma unroll
-  for (int k = 0; k < CPL; ++k) {
-    red[warp * 2 * C + lane + 32 * k] = dwa[k];
-    red[warp * 2 * C + C + lane + 32 * k] = dba[k];
   }
   __syncthreads();
   for (int c = threadIdx.x; c < 2 * C; c += blockDim.x) {
@@ -162,7 +157,15 @@ __global__ void ln_param_reduce_kernel(const float* __restrict__ part, int nbloc
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= 2 * C) return;
   float s = 0.f;
-  for (int b = 0; b < nblocks; ++b) s += part[(long long)b * 2 * C + c];
+  int b = 0;
+  for (; b + 8 <= nblocks; b += 8) {   // loads first, then the sum in block order
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = part[(long long)(b + i) * 2 * C + c];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += v[i];
+  }
+  for (; b < nblocks; ++b) s += part[(long long)b * 2 * C + c];
   if (c < C) dw[c] += s;
   else db[c - C] += s;
 }
@@ -178,14 +181,30 @@ __global__ void colsum_partial_kernel(const T* __restrict__ x, long long ldx, in
   if (n >= N) return;
   const int m0 = blockIdx.y * COLSUM_ROWS, m1 = min(M, m0 + COLSUM_ROWS);
   float s = 0.f;
-  for (int m = m0; m < m1; ++m) s += ld_f(x + (long long)m * ldx + n);
+  int m = m0;
+  for (; m + 8 <= m1; m += 8) {   // loads first, then the sum in row order
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = ld_f(x + (long long)(m + i) * ldx + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += v[i];
+  }
+  for (; m < m1; ++m) s += ld_f(x + (long long)m * ldx + n);
   part[(long long)blockIdx.y * N + n] = s;
 }
 __global__ void colsum_reduce_kernel(const float* __restrict__ part, int nchunks, int N, float* __restrict__ out) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
   float s = 0.f;
-  for (int k = 0; k < nchunks; ++k) s += part[(long long)k * N + n];
+  int k = 0;
+  for (; k + 8 <= nchunks; k += 8) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = part[(long long)(k + i) * N + n];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s += v[i];
+  }
+  for (; k < nchunks; ++k) s += part[(long long)k * N + n];
   out[n] += s;
 }
 
