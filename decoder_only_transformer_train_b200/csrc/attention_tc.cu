@@ -9,12 +9,14 @@
 //                 all straight out of the qkv activation [B*T, 3C]
 //   warp 1      : TMEM allocator + MMA issuer:  S_j = Q K_j^T  (128 x 128, TMEM)
 //                                                O_j = P_j V_j  (128 x 64,  TMEM)
-//   warps 2..5  : softmax - thread r owns query row r (= TMEM lane r): reads S_j, applies
-//                 the causal mask, updates the running max / sum, writes P_j (bf16) to
-//                 shared memory in the 128-byte-swizzled K-major layout the MMA reads,
-//                 and folds O_j into its register accumulator with the rescale factor.
-// S and O are double-buffered in TMEM (2 x 128 + 2 x 64 columns), P in shared memory, so
-// the MMA of S_{j+1} overlaps the softmax of S_j.
+//   warps 2..9  : two softmax groups of four warps; group g takes the key tiles j with
+//                 j % 2 == g.  Thread r of a group owns query row r (= TMEM lane r): it
+//                 reads S_j, applies the causal mask, updates its running max / sum,
+//                 writes P_j (bf16) to shared memory in the 128-byte-swizzled K-major
+//                 layout the MMA reads, and folds O_j into its register accumulator.
+//                 At the end the two partial softmax states of each row are merged.
+// S, O and P are double-buffered by tile parity, so each group owns one buffer of each
+// and the MMAs of one group's tile overlap the other group's softmax.
 #include <math.h>
 #include "sm100.cuh"
 #include "kernels.h"
@@ -25,10 +27,12 @@ constexpr int QT = 128;          // queries per CTA
 constexpr int KT = 128;          // keys per tile
 constexpr int HD = 64;
 constexpr int KV_STAGES = 3;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
 constexpr int TILE_BYTES = KT * HD * 2;        // 16 KB: one Q, K or V tile
 constexpr int P_BYTES = QT * KT * 2;           // 32 KB
-constexpr int SMEM_BYTES = TILE_BYTES + 2 * KV_STAGES * TILE_BYTES + 2 * P_BYTES + 512 + 1024;
+constexpr int MERGE_STRIDE = HD + 3;           // floats per row of the merge buffer (m, l, o[64])
+constexpr int MERGE_BYTES = QT * MERGE_STRIDE * 4;
+constexpr int SMEM_BYTES = TILE_BYTES + 2 * KV_STAGES * TILE_BYTES + 2 * P_BYTES + MERGE_BYTES + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0;                  // S buffers: columns [0, 256)
 constexpr uint32_t O_COL = 256;                // O buffers: columns [256, 384)
@@ -52,7 +56,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
   uint8_t* sK = sQ + TILE_BYTES;
   uint8_t* sV = sK + KV_STAGES * TILE_BYTES;
   uint8_t* sP = sV + KV_STAGES * TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * P_BYTES);
+  float* sMerge = reinterpret_cast<float*>(sP + 2 * P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * P_BYTES + MERGE_BYTES);
   uint64_t* q_full = bars;                       // 1
   uint64_t* kv_full = bars + 1;                  // KV_STAGES
   uint64_t* kv_empty = kv_full + KV_STAGES;      // KV_STAGES
@@ -62,7 +67,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
   uint64_t* p_empty = p_full + 2;                // 2
   uint64_t* o_full = p_empty + 2;                // 2
   uint64_t* o_empty = o_full + 2;                // 2
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_empty + 2);
+  uint64_t* merge_bar = o_empty + 2;             // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -90,6 +96,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       mbar_init(&o_full[i], 1);
       mbar_init(&o_empty[i], 128);
     }
+    mbar_init(merge_bar, 128);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
@@ -156,96 +163,125 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
     }
   } else {
     // ------------------------------------------------------------------ softmax
+    const int grp = (warp - 2) >> 2;             // key tiles j with j % 2 == grp
     const int q = warp & 3;
     const int r = q * 32 + lane;                 // query row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t s_col = S_COL + grp * KT, o_col = O_COL + grp * HD;
+    uint8_t* prow = sP + grp * P_BYTES + r * 128;
     float m = -INFINITY, l = 0.f, alpha_pending = 1.f;
     float o[HD];
 #pragma unroll
     for (int d = 0; d < HD; ++d) o[d] = 0.f;
     bool ok = true;
 
-    auto fold_o = [&](int i) -> bool {          // o = o * alpha_i + O_i
-      if (!mbar_wait(&o_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
+    auto fold_o = [&](int k) -> bool {          // o = o * alpha + O (this group's k-th tile)
+      if (!mbar_wait(&o_full[grp], k & 1, abort_flag)) return false;
       tc_fence_after();
-      uint32_t v[32];
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
-        tmem_ld32(tmem + lane_off + O_COL + (i & 1) * HD + c, v);
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + o_col + c, v);
         tmem_wait_ld();
 #pragma unroll
         for (int d = 0; d < 32; ++d) o[c + d] = o[c + d] * alpha_pending + __uint_as_float(v[d]);
       }
       tc_fence_before();
-      mbar_arrive(&o_empty[i & 1]);
+      mbar_arrive(&o_empty[grp]);
       return true;
     };
 
-    for (int j = 0; j < n_kv && ok; ++j) {
-      if (!mbar_wait(&s_full[j & 1], (j >> 1) & 1, abort_flag)) { ok = false; break; }
+    int k = 0;
+    for (int j = grp; j < n_kv && ok; j += 2, ++k) {
+      if (!mbar_wait(&s_full[grp], k & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float s[KT];
-#pragma unroll
-      for (int c = 0; c < KT; c += 32) {
+      const bool diag = (j == qt);
+      // pass 1: row max (key j*KT+c after query q0+r is masked on the diagonal tile)
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c0 = 0; c0 < KT; c0 += 32) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + S_COL + (j & 1) * KT + c, v);
+        tmem_ld32(tmem + lane_off + s_col + c0, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int d = 0; d < 32; ++d) s[c + d] = __uint_as_float(v[d]);
-      }
-      tc_fence_before();
-      mbar_arrive(&s_empty[j & 1]);              // S_j is in registers: the MMA may reuse it
-      const bool diag = (j == qt);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < KT; ++c) {
-        if (diag && c > r) s[c] = -INFINITY;     // key j*KT+c after query q0+r
-        mx = fmaxf(mx, s[c]);
+        for (int d = 0; d < 32; ++d) {
+          const float x = (diag && c0 + d > r) ? -INFINITY : __uint_as_float(v[d]);
+          mx = fmaxf(mx, x);
+        }
       }
       const float m_new = fmaxf(m, mx * scale_log2);
       const float alpha = ex2(m - m_new);
+      // pass 2: P = 2^(s*scale*log2e - m_new), row sum, P_j to shared memory once the
+      // MMA of this group's previous tile is done reading the buffer
+      if (!mbar_wait(&p_empty[grp], (k & 1) ^ 1, abort_flag)) { ok = false; break; }
       float sum = 0.f;
-      // P_j must not overwrite the buffer the MMA of O_{j-2} is still reading
-      if (!mbar_wait(&p_empty[j & 1], ((j >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-      uint8_t* prow = sP + (j & 1) * P_BYTES + r * 128;
+#pragma unroll 1
+      for (int c0 = 0; c0 < KT; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + s_col + c0, v);
+        tmem_wait_ld();
+        float p[32];
 #pragma unroll
-      for (int g = 0; g < KT / 8; ++g) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = ex2(s[g * 8 + e] * scale_log2 - m_new);
-          sum += p[e];
+        for (int d = 0; d < 32; ++d) {
+          const float x = (diag && c0 + d > r) ? -INFINITY : __uint_as_float(v[d]);
+          p[d] = ex2(x * scale_log2 - m_new);
+          sum += p[d];
         }
-        uint4 w;
-        w.x = pack_bf16x2(p[0], p[1]);
-        w.y = pack_bf16x2(p[2], p[3]);
-        w.z = pack_bf16x2(p[4], p[5]);
-        w.w = pack_bf16x2(p[6], p[7]);
-        const int chunk = g >> 3, gi = g & 7;
-        *reinterpret_cast<uint4*>(prow + chunk * 16384 + ((gi ^ (r & 7)) << 4)) = w;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          uint4 w;
+          w.x = pack_bf16x2(p[g * 8 + 0], p[g * 8 + 1]);
+          w.y = pack_bf16x2(p[g * 8 + 2], p[g * 8 + 3]);
+          w.z = pack_bf16x2(p[g * 8 + 4], p[g * 8 + 5]);
+          w.w = pack_bf16x2(p[g * 8 + 6], p[g * 8 + 7]);
+          const int gi = ((c0 & 63) >> 3) + g;
+          *reinterpret_cast<uint4*>(prow + (c0 >> 6) * 16384 + ((gi ^ (r & 7)) << 4)) = w;
+        }
       }
+      tc_fence_before();
+      mbar_arrive(&s_empty[grp]);
       fence_async_smem();
-      mbar_arrive(&p_full[j & 1]);
+      mbar_arrive(&p_full[grp]);
       l = l * alpha + sum;
       m = m_new;
-      if (j > 0 && !fold_o(j - 1)) { ok = false; break; }
+      if (k > 0 && !fold_o(k - 1)) { ok = false; break; }
       alpha_pending = alpha;
     }
-    if (ok) ok = fold_o(n_kv - 1);
-    const int qi = q0 + r;
-    if (ok && qi < T) {
-      const float inv = 1.0f / l;
-      bf16* orow = out + (long long)(row0 + qi) * C + h * HD;
+    if (ok && k > 0) ok = fold_o(k - 1);
+    // merge the two groups' partial states of row r: group 1 hands its (m, l, o) over
+    float* mrow = sMerge + r * MERGE_STRIDE;
+    if (grp == 1) {
+      if (ok) {
+        mrow[0] = m;
+        mrow[1] = l;
 #pragma unroll
-      for (int g = 0; g < HD / 8; ++g) {
-        uint4 w;
-        w.x = pack_bf16x2(o[g * 8 + 0] * inv, o[g * 8 + 1] * inv);
-        w.y = pack_bf16x2(o[g * 8 + 2] * inv, o[g * 8 + 3] * inv);
-        w.z = pack_bf16x2(o[g * 8 + 4] * inv, o[g * 8 + 5] * inv);
-        w.w = pack_bf16x2(o[g * 8 + 6] * inv, o[g * 8 + 7] * inv);
-        reinterpret_cast<uint4*>(orow)[g] = w;
+        for (int d = 0; d < HD; ++d) mrow[2 + d] = o[d];
       }
-      lse[(long long)bh * T + qi] = (m + log2f(l)) * 0.6931471805599453f;
+      mbar_arrive(merge_bar);
+    } else {
+      ok = ok && mbar_wait(merge_bar, 0, abort_flag);
+      const int qi = q0 + r;
+      if (ok && qi < T) {
+        const float m1 = mrow[0], l1 = mrow[1];
+        const float M = fmaxf(m, m1);
+        const float a0 = ex2(m - M), a1 = ex2(m1 - M);
+        const float L = l * a0 + l1 * a1;
+        const float inv = 1.0f / L;
+        bf16* orow = out + (long long)(row0 + qi) * C + h * HD;
+#pragma unroll
+        for (int g = 0; g < HD / 8; ++g) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = (o[g * 8 + e] * a0 + mrow[2 + g * 8 + e] * a1) * inv;
+          uint4 w;
+          w.x = pack_bf16x2(v[0], v[1]);
+          w.y = pack_bf16x2(v[2], v[3]);
+          w.z = pack_bf16x2(v[4], v[5]);
+          w.w = pack_bf16x2(v[6], v[7]);
+          reinterpret_cast<uint4*>(orow)[g] = w;
+        }
+        lse[(long long)bh * T + qi] = (M + log2f(L)) * 0.6931471805599453f;
+      }
     }
   }
 
@@ -316,7 +352,7 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
 // accumulates dQ over the key tiles at or before it.
 namespace {
 
-constexpr int BWD_THREADS = 192;
+constexpr int BWD_THREADS = 320;   // producer, MMA, 8 elementwise warps
 constexpr int BWD_STAGES = 2;
 // smem: 2 resident tiles (K_j,V_j or Q_i,dO_i) + BWD_STAGES x 2 streamed tiles + 2 P-like
 // 128x128 bf16 operands + barriers
@@ -387,8 +423,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       mbar_init(&t_empty[s], 1);
     }
     mbar_init(sd_full, 1);
-    mbar_init(sd_empty, 128);
-    mbar_init(ps_full, 128);
+    mbar_init(sd_empty, 256);
+    mbar_init(ps_full, 256);
     mbar_init(ps_empty, 1);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -493,6 +529,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   } else {
     // ------------------------------------------------------------------ elementwise
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;            // columns [64*half, 64*half + 64) of each tile
     const int r = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float LOG2E = 1.4426950408889634f;
@@ -513,7 +550,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       if (!mbar_wait(ps_empty, (n & 1) ^ 1, abort_flag)) { ok = false; break; }
       const bool diag = (t == tile);
 #pragma unroll 1
-      for (int c0 = 0; c0 < 128; c0 += 32) {
+      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
         uint32_t us[32], ud[32];
         tmem_ld32(tmem + lane_off + S_C + c0, us);
         tmem_ld32(tmem + lane_off + DP_C + c0, ud);
@@ -553,27 +590,22 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       bf16* row = dqkv + (long long)(row0 + gi) * (3 * C) + h * HD;
       const int nacc = (MODE == 0) ? 2 : 1;
       for (int a = 0; a < nacc; ++a) {
-        // MODE 0: a=0 dV (column block 2C), a=1 dK (column block C, times scale); MODE 1: dQ (times scale)
-        const uint32_t col = (a == 0) ? A0_C : A1_C;
+        // MODE 0: a=0 dV (column block 2C), a=1 dK (column block C, times scale); MODE 1: dQ (times scale).
+        // Each warp of a lane quarter writes 32 of the 64 head columns.
+        const uint32_t col = ((a == 0) ? A0_C : A1_C) + half * 32;
         const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
-        bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C));
-        float v[HD];
-#pragma unroll
-        for (int c = 0; c < HD; c += 32) {
-          uint32_t u[32];
-          tmem_ld32(tmem + lane_off + col + c, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int d = 0; d < 32; ++d) v[c + d] = __uint_as_float(u[d]) * mul;
-        }
+        bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C)) + half * 32;
+        uint32_t u[32];
+        tmem_ld32(tmem + lane_off + col, u);
+        tmem_wait_ld();
         if (gi < T) {
 #pragma unroll
-          for (int g = 0; g < HD / 8; ++g) {
+          for (int g = 0; g < 4; ++g) {
             uint4 w;
-            w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-            w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-            w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-            w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
+            w.x = pack_bf16x2(__uint_as_float(u[g * 8 + 0]) * mul, __uint_as_float(u[g * 8 + 1]) * mul);
+            w.y = pack_bf16x2(__uint_as_float(u[g * 8 + 2]) * mul, __uint_as_float(u[g * 8 + 3]) * mul);
+            w.z = pack_bf16x2(__uint_as_float(u[g * 8 + 4]) * mul, __uint_as_float(u[g * 8 + 5]) * mul);
+            w.w = pack_bf16x2(__uint_as_float(u[g * 8 + 6]) * mul, __uint_as_float(u[g * 8 + 7]) * mul);
             reinterpret_cast<uint4*>(dst)[g] = w;
           }
         }

@@ -77,5 +77,21 @@ __device__ __forceinline__ float gelu_tanh_grad_f(float x) {
   return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * GELU_A * (1.0f + 3.0f * GELU_C * x * x);
 }
 
+// Same formulas with the hardware tanh approximation (tanh.approx.f32, relative error
+// about 2^-11), used where the result is rounded to bf16 anyway.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float gelu_tanh_fast(float x) {
+  const float t = tanh_approx(GELU_A * (x + GELU_C * x * x * x));
+  return 0.5f * x * (1.0f + t);
+}
+__device__ __forceinline__ float gelu_tanh_grad_fast(float x) {
+  const float t = tanh_approx(GELU_A * (x + GELU_C * x * x * x));
+  return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * GELU_A * (1.0f + 3.0f * GELU_C * x * x);
+}
+
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ long long cdivll(long long a, long long b) { return (a + b - 1) / b; }

@@ -70,5 +70,7 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
 int gemm_f32_simt(cudaStream_t st, int M, int N, int K, const float* A, long long lda, bool a_mn,
                   const float* B, long long ldb, bool b_mn, EpiParams ep);
 
-// Column width of the logits tiles that EPI_CE_FWD partials refer to, for a given N.
+// Output tile width of the tcgen05 GEMM for a given N.
 int gemm_tc_tile_n(int N);
+// Number of per-row softmax partials EPI_CE_FWD writes for N columns (two per tile).
+int gemm_tc_ce_tiles(int N);

@@ -1,10 +1,11 @@
 // bf16 x bf16 -> fp32 GEMM on the sm_100a tensor cores (tcgen05.mma, accumulators in
 // TMEM), fed by TMA with a multi-stage mbarrier pipeline, with fused epilogues.
 //
-// Roles inside one persistent CTA (192 threads, one CTA per SM):
+// Roles inside one persistent CTA (320 threads, one CTA per SM):
 //   warp 0      : TMA producer (one elected lane) - stages of A and B tiles
 //   warp 1      : TMEM allocator + MMA issuer (one elected lane)
-//   warps 2..5  : epilogue - tcgen05.ld of the fp32 accumulator, fused math, stores
+//   warps 2..9  : epilogue - tcgen05.ld of the fp32 accumulator, fused math, stores;
+//                 two warps per TMEM lane quarter, each taking half of the tile's columns
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue of one
 // output tile overlaps the main loop of the next.
 //
@@ -20,7 +21,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;             // 64 bf16 = one 128-byte swizzle row
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_THREADS = 256;
 
 template <int BN>
 struct TileCfg {
@@ -169,7 +171,7 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         v[j] = alpha * v[j] + b[j];
-        g[j] = gelu_tanh_f(v[j]);
+        g[j] = gelu_tanh_fast(v[j]);
       }
       if (full) {
         store_bf16x32(u, v);
@@ -191,12 +193,12 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
         float uu[32];
         load_bf16x32(u, uu);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_f(uu[j]);
+        for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_fast(uu[j]);
         store_bf16x32(c, v);
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = __float2bfloat16_rn(alpha * v[j] * gelu_tanh_grad_f(__bfloat162float(u[j])));
+          if (j < nvalid) c[j] = __float2bfloat16_rn(alpha * v[j] * gelu_tanh_grad_fast(__bfloat162float(u[j])));
       }
       break;
     }
@@ -273,7 +275,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 128);
+      mbar_init(&tempty_bar[a], EPI_THREADS);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -362,6 +364,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;        // which half of the tile's columns
     const int row = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -374,7 +377,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int n_base = tn * BN;
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0x7fffffff};
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
         uint32_t r[32];
         tmem_ld32(tmem_base + acc * BN + c + (static_cast<uint32_t>(q * 32) << 16), r);
         tmem_wait_ld();
@@ -391,7 +394,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         p.sum = ce.sum;
         p.amax = ce.amax;
         p.aidx = ce.aidx;
-        ep.ce_part[(long long)m * ep.n_ctiles + tn] = p;
+        ep.ce_part[(long long)m * ep.n_ctiles + tn * 2 + half] = p;
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
@@ -476,6 +479,7 @@ int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, Til
 }  // namespace
 
 int gemm_tc_tile_n(int N) { return N > 128 ? 256 : 128; }
+int gemm_tc_ce_tiles(int N) { return cdiv(N, gemm_tc_tile_n(N)) * 2; }
 
 int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long lda, bool a_mn, const void* B,
                  long long ldb, bool b_mn, EpiParams ep, float* ws, size_t ws_elems, int num_sms) {
@@ -518,8 +522,8 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
     }
   }
   if (ep.kind == EPI_CE_FWD) {
-    run.n_ctiles = sched.n_tiles;
-    run.ce_tile_n = BN;
+    run.n_ctiles = sched.n_tiles * 2;
+    run.ce_tile_n = BN / 2;
   }
   if (BN == 256) {
     if (!a_mn && !b_mn) rc = launch_tc<256, false, false>(st, ta, tb, sched, run, num_sms);

@@ -360,7 +360,7 @@ int forward_impl(gpt2_ctx* c, int B, int T, bool with_targets) {
       RC(gemm(c, N, Vp, C, c->lnf, C, false, W(c, 0), C, false, e));
     }
     if (with_targets) {
-      const int ntiles = cdiv(Vp, gemm_tc_tile_n(Vp));
+      const int ntiles = gemm_tc_ce_tiles(Vp);
       PROF(PROF_CE, 0, 16.0 * Nd * ntiles + 16.0 * Nd);
       RC(launch_ce_finalize(st, c->ce_part, ntiles, c->zt, c->targets, N, g.vocab_size, c->lse, c->loss_row,
                             c->argmax));
@@ -612,7 +612,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
   AL(dalloc(c, &c->lnf_mean, N));
   AL(dalloc(c, &c->lnf_rstd, N));
   AL(dalloc_bytes(c, &c->logits, N * c->ldl * A));
-  AL(dalloc(c, &c->ce_part, N * (size_t)cdiv((int)Vp, 128)));
+  AL(dalloc(c, &c->ce_part, N * (size_t)gemm_tc_ce_tiles((int)Vp)));
   AL(dalloc(c, &c->zt, N));
   AL(dalloc(c, &c->lse, N));
   AL(dalloc(c, &c->loss_row, N));

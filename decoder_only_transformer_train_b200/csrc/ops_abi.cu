@@ -61,7 +61,7 @@ int gpt2op_layernorm_fwd(void* stream, int precision, const float* x, const floa
 }
 
 int64_t gpt2op_classifier_aux_floats(int N, int V) {
-  const int ntiles = cdiv(V, gemm_tc_tile_n(V));
+  const int ntiles = gemm_tc_ce_tiles(V);
   // partials (4 floats each), zt, loss_row, and 8 scalars
   return (int64_t)N * ntiles * 4 + 2LL * N + 8;
 }
@@ -73,7 +73,7 @@ int gpt2op_classifier_fwd_bwd(void* stream, const void* h, const void* W, const 
   if (N <= 0 || V <= 0 || C <= 0 || ldl < V || ldl % 8 || C % 8) return GPT2_ERR_SHAPE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int nsm = sm_count();
-  const int ntiles = cdiv(V, gemm_tc_tile_n(V));
+  const int ntiles = gemm_tc_ce_tiles(V);
   CePartial* part = reinterpret_cast<CePartial*>(aux_ws);
   float* zt = aux_ws + (size_t)N * ntiles * 4;
   float* loss_row = zt + N;
