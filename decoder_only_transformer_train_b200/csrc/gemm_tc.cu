@@ -87,26 +87,49 @@ struct CeRowState {
   int aidx;
 };
 
-// Epilogue of one 32-column chunk of one output row.
+// Global reads an epilogue chunk needs (bias, residual / accumulator / GELU input), issued
+// before the chunk's TMEM load so that their latencies overlap.
+__device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, int m, int n0, float (&b)[32],
+                                                  float (&pre)[32]) {
+  const int N = ep.N;
+  const bool full = (n0 + 32 <= N);
+  const int nvalid = full ? 32 : max(0, N - n0);
+  const bool use_bias = ep.bias != nullptr && (ep.kind == EPI_STORE_ACT || ep.kind == EPI_STORE_F32 ||
+                                               ep.kind == EPI_RESID_F32 || ep.kind == EPI_GELU_FWD);
+  if (use_bias && full) {
+    load_f32x32(ep.bias + n0, b);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) b[j] = (use_bias && j < nvalid) ? ep.bias[n0 + j] : 0.0f;
+  }
+  if (ep.kind == EPI_RESID_F32 || ep.kind == EPI_ACCUM_F32) {
+    const float* src = (ep.kind == EPI_RESID_F32)
+                           ? reinterpret_cast<const float*>(ep.aux) + (long long)m * ep.ld_aux + n0
+                           : reinterpret_cast<const float*>(ep.C) + (long long)m * ep.ldc + n0;
+    if (full) {
+      load_f32x32(src, pre);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) pre[j] = (j < nvalid) ? src[j] : 0.0f;
+    }
+  } else if (ep.kind == EPI_GELU_BWD) {
+    const bf16* u = reinterpret_cast<const bf16*>(ep.aux) + (long long)m * ep.ld_aux + n0;
+    if (full) {
+      load_bf16x32(u, pre);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) pre[j] = (j < nvalid) ? __bfloat162float(u[j]) : 0.0f;
+    }
+  }
+}
+
+// Epilogue of one 32-column chunk of one output row (b, pre from epilogue_prefetch).
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n0, float (&v)[32], int split,
-                                               CeRowState& ce) {
+                                               CeRowState& ce, const float (&b)[32], const float (&pre)[32]) {
   const int N = ep.N;
   const bool full = (n0 + 32 <= N);
   const int nvalid = full ? 32 : max(0, N - n0);
   const float alpha = ep.alpha;
-  float b[32];
-  if (ep.bias != nullptr && ep.kind != EPI_SPLITK && ep.kind != EPI_ACCUM_F32 && ep.kind != EPI_CE_FWD &&
-      ep.kind != EPI_GELU_BWD) {
-    if (full) {
-      load_f32x32(ep.bias + n0, b);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) b[j] = (j < nvalid) ? ep.bias[n0 + j] : 0.0f;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) b[j] = 0.0f;
-  }
 
   switch (ep.kind) {
     case EPI_STORE_ACT: {
@@ -133,34 +156,17 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
       }
       break;
     }
-    case EPI_ACCUM_F32: {
-      float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) {
-        float o[32];
-        load_f32x32(c, o);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] += alpha * v[j];
-        store_f32x32(c, o);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] += alpha * v[j];
-      }
-      break;
-    }
+    case EPI_ACCUM_F32:
     case EPI_RESID_F32: {
-      const float* r = reinterpret_cast<const float*>(ep.aux) + (long long)m * ep.ld_aux + n0;
-      float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) {
-        float o[32];
-        load_f32x32(r, o);
+      float o[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] += alpha * v[j] + b[j];
-        store_f32x32(c, o);
-      } else {
+      for (int j = 0; j < 32; ++j) o[j] = pre[j] + alpha * v[j] + b[j];
+      float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
+      if (full) store_f32x32(c, o);
+      else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = r[j] + alpha * v[j] + b[j];
+          if (j < nvalid) c[j] = o[j];
       }
       break;
     }
@@ -187,18 +193,14 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
       break;
     }
     case EPI_GELU_BWD: {
-      const bf16* u = reinterpret_cast<const bf16*>(ep.aux) + (long long)m * ep.ld_aux + n0;
       bf16* c = reinterpret_cast<bf16*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) {
-        float uu[32];
-        load_bf16x32(u, uu);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_fast(uu[j]);
-        store_bf16x32(c, v);
-      } else {
+      for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_fast(pre[j]);
+      if (full) store_bf16x32(c, v);
+      else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = __float2bfloat16_rn(alpha * v[j] * gelu_tanh_grad_fast(__bfloat162float(u[j])));
+          if (j < nvalid) c[j] = __float2bfloat16_rn(v[j]);
       }
       break;
     }
@@ -378,14 +380,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0x7fffffff};
 #pragma unroll 1
       for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+        const bool live = (m < ep.M && n_base + c < ep.N);
+        float bb[32], pre[32];
+        if (live) epilogue_prefetch(ep, m, n_base + c, bb, pre);
         uint32_t r[32];
         tmem_ld32(tmem_base + acc * BN + c + (static_cast<uint32_t>(q * 32) << 16), r);
         tmem_wait_ld();
-        if (m < ep.M && n_base + c < ep.N) {
+        if (live) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          epilogue_chunk(ep, m, n_base + c, v, split, ce);
+          epilogue_chunk(ep, m, n_base + c, v, split, ce, bb, pre);
         }
       }
       if (ep.kind == EPI_CE_FWD && m < ep.M) {

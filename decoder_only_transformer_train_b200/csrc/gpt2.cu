@@ -413,8 +413,10 @@ int backward_impl(gpt2_ctx* c) {
   const double ln_bwd_bytes = Nd * Cd * (4.0 * 4 + A) + 8.0 * Nd;
   {
     PROF(PROF_LN_BWD, 0, ln_bwd_bytes - 4.0 * Nd * Cd);
+    // the new dres is d loss / d x_L: its column sums are the last mlp.c_proj bias gradient
     RC(launch_layernorm_bwd(st, c->bf16, c->dy, xL, c->lnf_mean, c->lnf_rstd, P(c, lf), c->dres, c->dres_act, false,
-                            c->ln_part, c->ln_blocks, G(c, lf), G(c, lf + 1), N, C));
+                            c->ln_part, c->ln_blocks, G(c, lf), G(c, lf + 1), G(c, param_index(g, L - 1, MPROJ_B)), N,
+                            C));
   }
   const int ncs = colsum_chunks(N);
   for (int l = L - 1; l >= 0; --l) {
@@ -426,10 +428,6 @@ int backward_impl(gpt2_ctx* c) {
     {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * 4 * Cd * Cd, 0);
       RC(gemm(c, C, 4 * C, N, c->dres_act, C, true, a.fc_act, 4 * C, true, e));
-    }
-    {
-      PROF(PROF_BIAS, 0, 4.0 * Nd * Cd);
-      RC(launch_colsum(st, false, c->dres, C, N, C, c->colsum_part, ncs, G(c, pi(MPROJ_B))));
     }
     e = epi_make(EPI_GELU_BWD, c->d4c, 4 * C);
     e.aux = a.fc_pre;
@@ -454,18 +452,16 @@ int backward_impl(gpt2_ctx* c) {
     }
     {
       PROF(PROF_LN_BWD, 0, ln_bwd_bytes);
+      // the new dres is d loss / d x1: its column sums are this layer's attn.c_proj bias gradient
       RC(launch_layernorm_bwd(st, c->bf16, c->dy, a.x1, a.ln2_mean, a.ln2_rstd, P(c, pi(LN2_W)), c->dres,
-                              c->dres_act, true, c->ln_part, c->ln_blocks, G(c, pi(LN2_W)), G(c, pi(LN2_B)), N, C));
+                              c->dres_act, true, c->ln_part, c->ln_blocks, G(c, pi(LN2_W)), G(c, pi(LN2_B)),
+                              G(c, pi(PROJ_B)), N, C));
     }
     // ---- attention: x1 = x + attn(ln1 Wqkv^T + bqkv) Wp^T + bp
     e = epi_make(EPI_ACCUM_F32, G(c, pi(PROJ_W)), C);
     {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * Cd * Cd, 0);
       RC(gemm(c, C, C, N, c->dres_act, C, true, a.attn, C, true, e));
-    }
-    {
-      PROF(PROF_BIAS, 0, 4.0 * Nd * Cd);
-      RC(launch_colsum(st, false, c->dres, C, N, C, c->colsum_part, ncs, G(c, pi(PROJ_B))));
     }
     e = epi_make(EPI_STORE_ACT, c->dattn, C);
     {
@@ -492,8 +488,10 @@ int backward_impl(gpt2_ctx* c) {
     }
     {
       PROF(PROF_LN_BWD, 0, ln_bwd_bytes);
+      // the new dres is d loss / d x_l: the previous layer's mlp.c_proj bias gradient
+      float* db_prev = (l > 0) ? G(c, param_index(g, l - 1, MPROJ_B)) : nullptr;
       RC(launch_layernorm_bwd(st, c->bf16, c->dy, x, a.ln1_mean, a.ln1_rstd, P(c, pi(LN1_W)), c->dres, c->dres_act,
-                              true, c->ln_part, c->ln_blocks, G(c, pi(LN1_W)), G(c, pi(LN1_B)), N, C));
+                              true, c->ln_part, c->ln_blocks, G(c, pi(LN1_W)), G(c, pi(LN1_B)), db_prev, N, C));
     }
   }
   // token + position embedding
@@ -629,7 +627,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
   AL(dalloc_bytes(c, &c->dattn, N * C * A));
   AL(dalloc(c, &c->attnD, N * H));
   c->ln_blocks = layernorm_bwd_blocks(c->num_sms);
-  AL(dalloc(c, &c->ln_part, (size_t)c->ln_blocks * 2 * C));
+  AL(dalloc(c, &c->ln_part, (size_t)c->ln_blocks * 3 * C));
   AL(dalloc(c, &c->colsum_part, (size_t)colsum_chunks((int)N) * 4 * C));
   AL(dalloc(c, &c->enc_sorted, N));
   AL(dalloc(c, &c->enc_part, encoder_bwd_part_floats((int)N, (int)C)));

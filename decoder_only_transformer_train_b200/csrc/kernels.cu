@@ -95,9 +95,11 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const float* __restrict__ x
 
 // dx = rstd * (dxhat - mean(dxhat) - xhat * mean(dxhat * xhat)),  dxhat = dy * w;
 // dres = (accumulate ? dres : 0) + dx, also written in the activation type for the next
-// GEMM.  dw = sum_rows dy * xhat and db = sum_rows dy are accumulated in each warp's own
-// shared-memory slice (fixed row order: block b, warp w owns rows b*8+w + k*gridDim*8),
-// then summed over the 8 warps in order into one partial per block.
+// GEMM.  Column sums accumulated in each warp's own shared-memory slice, in a fixed row
+// order (block b, warp w owns rows b*8+w + k*gridDim*8), then over the 8 warps in order
+// into one partial per block:  dw = sum dy * xhat,  db = sum dy,  and the sum of the new
+// dres rows, which is the bias gradient of the Linear layer whose output this residual
+// stream position receives (attn.c_proj or mlp.c_proj).
 template <typename ActT, int CPL>
 __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
                                                         const float* __restrict__ mean, const float* __restrict__ rstd,
@@ -105,20 +107,24 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict_
                                                         ActT* __restrict__ dres_act, int accumulate,
                                                         float* __restrict__ part, int N) {
   constexpr int C = CPL * 32;
-  extern __shared__ float red[];   // [8][2C]
+  extern __shared__ float red[];   // [8][3C]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* mine = red + warp * 2 * C;
+  float* mine = red + warp * 3 * C;
 #pragma unroll
   for (int k = 0; k < CPL; ++k) {
     mine[lane + 32 * k] = 0.f;
     mine[C + lane + 32 * k] = 0.f;
+    mine[2 * C + lane + 32 * k] = 0.f;
   }
   for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
     const float* dyr = dy + (long long)row * C;
     const float* xr = x + (long long)row * C;
+    float* dr = dres + (long long)row * C;
     const float mu = mean[row], r = rstd[row];
-    float g[CPL], xh[CPL];
+    float g[CPL], xh[CPL], prev[CPL];
     float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) prev[k] = accumulate ? dr[lane + 32 * k] : 0.f;   // issued early
 #pragma unroll
     for (int k = 0; k < CPL; ++k) {
       const int c = lane + 32 * k;
@@ -132,42 +138,43 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict_
     }
     s1 = warp_sum(s1) * (1.0f / C);
     s2 = warp_sum(s2) * (1.0f / C);
-    float* dr = dres + (long long)row * C;
     ActT* da = dres_act + (long long)row * C;
 #pragma unroll
     for (int k = 0; k < CPL; ++k) {
       const int c = lane + 32 * k;
-      float o = r * (g[k] - s1 - xh[k] * s2);
-      if (accumulate) o += dr[c];
+      const float o = r * (g[k] - s1 - xh[k] * s2) + prev[k];
       dr[c] = o;
       st_f(da + c, o);
+      mine[2 * C + c] += o;
     }
   }
   __syncthreads();
-  for (int c = threadIdx.x; c < 2 * C; c += blockDim.x) {
+  for (int c = threadIdx.x; c < 3 * C; c += blockDim.x) {
     float s = 0.f;
 #pragma unroll
-    for (int wi = 0; wi < 8; ++wi) s += red[wi * 2 * C + c];
-    part[(long long)blockIdx.x * 2 * C + c] = s;
+    for (int wi = 0; wi < 8; ++wi) s += red[wi * 3 * C + c];
+    part[(long long)blockIdx.x * 3 * C + c] = s;
   }
 }
 
 __global__ void ln_param_reduce_kernel(const float* __restrict__ part, int nblocks, int C, float* __restrict__ dw,
-                                       float* __restrict__ db) {
+                                       float* __restrict__ db, float* __restrict__ dbias_out) {
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= 2 * C) return;
+  if (c >= 3 * C) return;
+  if (c >= 2 * C && dbias_out == nullptr) return;
   float s = 0.f;
   int b = 0;
   for (; b + 8 <= nblocks; b += 8) {   // loads first, then the sum in block order
     float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = part[(long long)(b + i) * 2 * C + c];
+    for (int i = 0; i < 8; ++i) v[i] = part[(long long)(b + i) * 3 * C + c];
 #pragma unroll
     for (int i = 0; i < 8; ++i) s += v[i];
   }
-  for (; b < nblocks; ++b) s += part[(long long)b * 2 * C + c];
+  for (; b < nblocks; ++b) s += part[(long long)b * 3 * C + c];
   if (c < C) dw[c] += s;
-  else db[c - C] += s;
+  else if (c < 2 * C) db[c - C] += s;
+  else dbias_out[c - 2 * C] += s;
 }
 
 // ================================================================ bias gradients
@@ -177,20 +184,39 @@ constexpr int COLSUM_ROWS = 256;
 template <typename T>
 __global__ void colsum_partial_kernel(const T* __restrict__ x, long long ldx, int M, int N,
                                       float* __restrict__ part) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+  const int n0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;   // 8 consecutive columns per thread
+  if (n0 >= N) return;
   const int m0 = blockIdx.y * COLSUM_ROWS, m1 = min(M, m0 + COLSUM_ROWS);
-  float s = 0.f;
-  int m = m0;
-  for (; m + 8 <= m1; m += 8) {   // loads first, then the sum in row order
-    float v[8];
+  float s[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = ld_f(x + (long long)(m + i) * ldx + n);
+  for (int i = 0; i < 8; ++i) s[i] = 0.f;
+  if (n0 + 8 <= N) {
+#pragma unroll 4
+    for (int m = m0; m < m1; ++m) {
+      const T* p = x + (long long)m * ldx + n0;
+      if (sizeof(T) == 2) {
+        const uint4 q = *reinterpret_cast<const uint4*>(p);
+        const uint32_t* u = reinterpret_cast<const uint32_t*>(&q);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s += v[i];
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = unpack_bf16x2(u[i]);
+          s[2 * i] += f.x;
+          s[2 * i + 1] += f.y;
+        }
+      } else {
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        const float4 b = *reinterpret_cast<const float4*>(p + 4);
+        s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
+        s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
+      }
+    }
+  } else {
+    for (int m = m0; m < m1; ++m)
+      for (int i = 0; i < 8 && n0 + i < N; ++i) s[i] += ld_f(x + (long long)m * ldx + n0 + i);
   }
-  for (; m < m1; ++m) s += ld_f(x + (long long)m * ldx + n);
-  part[(long long)blockIdx.y * N + n] = s;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    if (n0 + i < N) part[(long long)blockIdx.y * N + n0 + i] = s[i];
 }
 __global__ void colsum_reduce_kernel(const float* __restrict__ part, int nchunks, int N, float* __restrict__ out) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
@@ -597,7 +623,7 @@ int ln_fwd_dispatch(cudaStream_t st, const float* x, const float* w, const float
 template <typename ActT>
 int ln_bwd_dispatch(cudaStream_t st, const float* dy, const float* x, const float* mean, const float* rstd,
                     const float* w, float* dres, ActT* dres_act, int acc, float* part, int nblocks, int N, int C) {
-  const int smem = 8 * 2 * C * (int)sizeof(float);
+  const int smem = 8 * 3 * C * (int)sizeof(float);
   switch (C) {
 #define LNB(CPL)                                                                                               \
   case CPL * 32: {                                                                                             \
@@ -638,13 +664,13 @@ int layernorm_bwd_blocks(int num_sms) { return 2 * num_sms; }
 
 int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const float* dy, const float* x, const float* mean,
                          const float* rstd, const float* w, float* dres, void* dres_act, bool accumulate, float* part,
-                         int nblocks, float* dw, float* db, int N, int C) {
+                         int nblocks, float* dw, float* db, float* dbias_out, int N, int C) {
   int rc = is_bf16 ? ln_bwd_dispatch<bf16>(st, dy, x, mean, rstd, w, dres, reinterpret_cast<bf16*>(dres_act),
                                            accumulate, part, nblocks, N, C)
                    : ln_bwd_dispatch<float>(st, dy, x, mean, rstd, w, dres, reinterpret_cast<float*>(dres_act),
                                             accumulate, part, nblocks, N, C);
   if (rc) return rc;
-  ln_param_reduce_kernel<<<cdiv(2 * C, 256), 256, 0, st>>>(part, nblocks, C, dw, db);
+  ln_param_reduce_kernel<<<cdiv(3 * C, 256), 256, 0, st>>>(part, nblocks, C, dw, db, dbias_out);
   note_kernel_launches(1);
   return ok();
 }
@@ -653,9 +679,10 @@ int colsum_chunks(int M) { return cdiv(M, COLSUM_ROWS); }
 
 int launch_colsum(cudaStream_t st, bool is_bf16, const void* x, long long ldx, int M, int N, float* part,
                   int nchunks, float* out) {
-  dim3 grid(cdiv(N, 256), nchunks);
-  if (is_bf16) colsum_partial_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, part);
-  else colsum_partial_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, part);
+  if (N % 8 != 0 || ldx % 8 != 0) return -4;
+  dim3 grid(cdiv(N / 8, 128), nchunks);
+  if (is_bf16) colsum_partial_kernel<bf16><<<grid, 128, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, part);
+  else colsum_partial_kernel<float><<<grid, 128, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, part);
   colsum_reduce_kernel<<<cdiv(N, 256), 256, 0, st>>>(part, nchunks, N, out);
   note_kernel_launches(2);
   return ok();
