@@ -4,38 +4,38 @@
 // scores, mask, softmax and weighted sum fused in one kernel that never writes the T x T
 // matrix, using the online softmax (running max and sum).
 //
-// One CTA per (batch, head, 128-query tile), heaviest (latest) query tiles first.
-//   warp 0      : TMA producer - Q once, then K_j / V_j tiles of 128 keys (3 stages),
+// Persistent: one CTA per SM walks (batch, head, 128-query tile) items, heaviest (latest)
+// query tiles first; Q is double-buffered so the pipeline runs on across items.
+//   warp 0      : TMA producer - Q of each item, then its K_j / V_j tiles of 128 keys,
 //                 all straight out of the qkv activation [B*T, 3C]
-//   warp 1      : TMEM allocator + MMA issuer:  S_j = Q K_j^T  (128 x 128, TMEM)
-//                                                O_j = P_j V_j  (128 x 64,  TMEM)
-//   warps 2..9  : two softmax groups of four warps; group g takes the key tiles j with
-//                 j % 2 == g.  Thread r of a group owns query row r (= TMEM lane r): it
-//                 reads S_j, applies the causal mask, updates its running max / sum,
-//                 writes P_j (bf16) to shared memory in the 128-byte-swizzled K-major
-//                 layout the MMA reads, and folds O_j into its register accumulator.
-//                 At the end the two partial softmax states of each row are merged.
-// S, O and P are double-buffered by tile parity, so each group owns one buffer of each
-// and the MMAs of one group's tile overlap the other group's softmax.
+//   warp 1      : TMEM allocator + MMA issuer:  S_j = Q K_j^T    (128 x 128, TMEM)
+//                                                O  += P_j V_j    (128 x 64, TMEM)
+//   warps 2..9  : two softmax groups of four warps; the CTA's key tiles alternate between
+//                 them (global tile counter parity).  Thread r of a group owns query row r
+//                 (= TMEM lane r): it reads S_j, applies the causal mask, and writes
+//                 P_j = 2^(s*log2e/sqrt(hd) - m_ref) (bf16) to shared memory in the
+//                 128-byte-swizzled K-major layout the MMA reads.  Each group accumulates
+//                 its own O in TMEM; m_ref only moves when a row's max grows by more than
+//                 2^8, and then the thread rescales its O row in TMEM before the next MMA.
+//                 At the end of an item the two groups' (m_ref, l, O) are merged.
 #include <math.h>
 #include "sm100.cuh"
 #include "kernels.h"
 
 namespace {
 
-constexpr int QT = 128;          // queries per CTA
+constexpr int QT = 128;          // queries per item
 constexpr int KT = 128;          // keys per tile
 constexpr int HD = 64;
 constexpr int KV_STAGES = 3;
 constexpr int NUM_THREADS = 320;
 constexpr int TILE_BYTES = KT * HD * 2;        // 16 KB: one Q, K or V tile
 constexpr int P_BYTES = QT * KT * 2;           // 32 KB
-constexpr int MERGE_STRIDE = HD + 3;           // floats per row of the merge buffer (m, l, o[64])
-constexpr int MERGE_BYTES = QT * MERGE_STRIDE * 4;
-constexpr int SMEM_BYTES = TILE_BYTES + 2 * KV_STAGES * TILE_BYTES + 2 * P_BYTES + MERGE_BYTES + 512 + 1024;
+constexpr int SMEM_BYTES = 2 * TILE_BYTES + 2 * KV_STAGES * TILE_BYTES + 2 * P_BYTES + QT * 8 + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t S_COL = 0;                  // S buffers: columns [0, 256)
-constexpr uint32_t O_COL = 256;                // O buffers: columns [256, 384)
+constexpr uint32_t S_COL = 0;                  // S of group g: columns [128 g, 128 g + 128)
+constexpr uint32_t O_COL = 256;                // O of group g: columns [256 + 64 g, 256 + 64 g + 64)
+constexpr float RESCALE_THRESHOLD = 8.0f;      // log2 units
 
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -47,56 +47,60 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Item order shared by all roles: item t -> (query tile, batch*head), heaviest first.
+struct FwdItems {
+  int n_qt, BH, total;
+  __device__ __forceinline__ void get(int t, int& qt, int& bh) const {
+    qt = n_qt - 1 - t / BH;
+    bh = t % BH;
+  }
+};
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
                    int B, int T, int H, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + TILE_BYTES;
-  uint8_t* sV = sK + KV_STAGES * TILE_BYTES;
-  uint8_t* sP = sV + KV_STAGES * TILE_BYTES;
-  float* sMerge = reinterpret_cast<float*>(sP + 2 * P_BYTES);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + 2 * P_BYTES + MERGE_BYTES);
-  uint64_t* q_full = bars;                       // 1
-  uint64_t* kv_full = bars + 1;                  // KV_STAGES
+  uint8_t* sQ = smem;                                    // [2]
+  uint8_t* sK = sQ + 2 * TILE_BYTES;                     // [KV_STAGES]
+  uint8_t* sV = sK + KV_STAGES * TILE_BYTES;             // [KV_STAGES]
+  uint8_t* sP = sV + KV_STAGES * TILE_BYTES;             // [2]
+  float* sML = reinterpret_cast<float*>(sP + 2 * P_BYTES);   // [QT][2]: handed-over (m_ref, l)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sML + 2 * QT);
+  uint64_t* q_full = bars;                       // 2
+  uint64_t* q_empty = q_full + 2;                // 2
+  uint64_t* kv_full = q_empty + 2;               // KV_STAGES
   uint64_t* kv_empty = kv_full + KV_STAGES;      // KV_STAGES
-  uint64_t* s_full = kv_empty + KV_STAGES;       // 2
+  uint64_t* s_full = kv_empty + KV_STAGES;       // 2 (per group)
   uint64_t* s_empty = s_full + 2;                // 2
   uint64_t* p_full = s_empty + 2;                // 2
   uint64_t* p_empty = p_full + 2;                // 2
-  uint64_t* o_full = p_empty + 2;                // 2
-  uint64_t* o_empty = o_full + 2;                // 2
-  uint64_t* merge_bar = o_empty + 2;             // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_bar + 1);
+  uint64_t* o_done = p_empty + 2;                // 2
+  uint64_t* merge_full = o_done + 2;             // 1
+  uint64_t* merge_empty = merge_full + 1;        // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_empty + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_qt = cdiv(T, QT);
-  const int BH = B * H;
-  const int qt = n_qt - 1 - (int)(blockIdx.x / BH);     // heaviest tiles first
-  const int bh = (int)(blockIdx.x % BH);
-  const int b = bh / H, h = bh % H;
   const int C = H * HD;
-  const int q0 = qt * QT;
-  const int row0 = b * T;                               // first token row of this sequence
-  const int n_kv = qt + 1;
+  FwdItems items{cdiv(T, QT), B * H, cdiv(T, QT) * B * H};
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < KV_STAGES; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
       mbar_init(&s_empty[i], 128);
       mbar_init(&p_full[i], 128);
       mbar_init(&p_empty[i], 1);
-      mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 128);
+      mbar_init(&o_done[i], 1);
     }
-    mbar_init(merge_bar, 128);
+    for (int s = 0; s < KV_STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(merge_full, 128);
+    mbar_init(merge_empty, 128);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
@@ -113,14 +117,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------------- TMA producer
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      tma_load_2d(sQ, &tm_qkv, h * HD, row0 + q0, q_full);
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % KV_STAGES;
-        if (!mbar_wait(&kv_empty[s], ((j / KV_STAGES) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * TILE_BYTES);
-        tma_load_2d(sK + s * TILE_BYTES, &tm_qkv, C + h * HD, row0 + j * KT, &kv_full[s]);
-        tma_load_2d(sV + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + j * KT, &kv_full[s]);
+      int G = 0;                                   // global key-tile counter
+      bool ok = true;
+      for (int t = blockIdx.x, k = 0; t < items.total && ok; t += gridDim.x, ++k) {
+        int qt, bh;
+        items.get(t, qt, bh);
+        const int b = bh / H, h = bh % H, row0 = b * T;
+        const int qb = k & 1;
+        if (!mbar_wait(&q_empty[qb], ((k >> 1) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&q_full[qb], TILE_BYTES);
+        tma_load_2d(sQ + qb * TILE_BYTES, &tm_qkv, h * HD, row0 + qt * QT, &q_full[qb]);
+        for (int j = 0; j <= qt; ++j, ++G) {
+          const int s = G % KV_STAGES;
+          if (!mbar_wait(&kv_empty[s], ((G / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&kv_full[s], 2 * TILE_BYTES);
+          tma_load_2d(sK + s * TILE_BYTES, &tm_qkv, C + h * HD, row0 + j * KT, &kv_full[s]);
+          tma_load_2d(sV + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + j * KT, &kv_full[s]);
+        }
       }
     }
   } else if (warp == 1) {
@@ -128,161 +141,234 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = make_idesc_bf16(QT, KT, false, false);   // Q, K both K-major
       constexpr uint32_t idesc_o = make_idesc_bf16(QT, HD, false, true);    // P K-major, V MN-major
-      const uint32_t aQ = smem_u32(sQ);
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % KV_STAGES;
-        if (!mbar_wait(&kv_full[s], (j / KV_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait(&s_empty[j & 1], ((j >> 1) & 1) ^ 1, abort_flag)) return false;
+      // tile iterator over the CTA's flattened (item, j) sequence
+      struct It {
+        int t, k, qt, j, G;
+      };
+      auto valid = [&](const It& it) { return it.t < items.total; };
+      auto next = [&](It it) {
+        ++it.G;
+        if (++it.j > it.qt) {
+          it.j = 0;
+          it.t += gridDim.x;
+          ++it.k;
+          if (it.t < items.total) {
+            int bh;
+            items.get(it.t, it.qt, bh);
+          }
+        }
+        return it;
+      };
+      It cur{(int)blockIdx.x, 0, 0, 0, 0};
+      if (valid(cur)) {
+        int bh;
+        items.get(cur.t, cur.qt, bh);
+      }
+      int cs0 = 0, cs1 = 0;    // S issues per group
+      int co0 = 0, co1 = 0;    // O issues per group
+      bool ok = true;
+      auto issue_s = [&](const It& it) -> bool {
+        const int g = it.G & 1, s = it.G % KV_STAGES, qb = it.k & 1;
+        if (it.j == 0 && !mbar_wait(&q_full[qb], (it.k >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&kv_full[s], (it.G / KV_STAGES) & 1, abort_flag)) return false;
+        const int cs = g ? cs1 : cs0;
+        if (!mbar_wait(&s_empty[g], (cs & 1) ^ 1, abort_flag)) return false;
+        if (g) ++cs1; else ++cs0;
         tc_fence_after();
+        const uint32_t aQ = smem_u32(sQ + qb * TILE_BYTES);
         const uint32_t bK = smem_u32(sK + s * TILE_BYTES);
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k)
-          tc_mma_bf16(tmem + S_COL + (j & 1) * KT, make_sdesc_sw128(aQ + k * 32, 16, 1024),
-                      make_sdesc_sw128(bK + k * 32, 16, 1024), idesc_s, k > 0 ? 1u : 0u);
-        tc_commit(&s_full[j & 1]);
+        for (int kk = 0; kk < HD / 16; ++kk)
+          tc_mma_bf16(tmem + S_COL + g * KT, make_sdesc_sw128(aQ + kk * 32, 16, 1024),
+                      make_sdesc_sw128(bK + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        tc_commit(&s_full[g]);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < n_kv && ok; ++j) {
-        if (j + 1 < n_kv && !issue_s(j + 1)) break;
-        const int s = j % KV_STAGES;
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag)) break;
-        if (!mbar_wait(&o_empty[j & 1], ((j >> 1) & 1) ^ 1, abort_flag)) break;
+      if (valid(cur)) ok = issue_s(cur);
+      while (ok && valid(cur)) {
+        const It nx = next(cur);
+        if (valid(nx) && !issue_s(nx)) break;
+        const int g = cur.G & 1, s = cur.G % KV_STAGES;
+        const int co = g ? co1 : co0;
+        if (!mbar_wait(&p_full[g], co & 1, abort_flag)) break;
+        if (g) ++co1; else ++co0;
         tc_fence_after();
-        const uint32_t aP = smem_u32(sP + (j & 1) * P_BYTES);
+        const bool first_of_group = (cur.j < 2);          // the group's first tile of this item
+        const uint32_t aP = smem_u32(sP + g * P_BYTES);
         const uint32_t bV = smem_u32(sV + s * TILE_BYTES);
 #pragma unroll
-        for (int k = 0; k < KT / 16; ++k)
-          tc_mma_bf16(tmem + O_COL + (j & 1) * HD, make_sdesc_sw128(aP + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                      make_sdesc_sw128(bV + k * 2048, 8192, 1024), idesc_o, k > 0 ? 1u : 0u);
-        tc_commit(&o_full[j & 1]);
+        for (int kk = 0; kk < KT / 16; ++kk)
+          tc_mma_bf16(tmem + O_COL + g * HD, make_sdesc_sw128(aP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                      make_sdesc_sw128(bV + kk * 2048, 8192, 1024), idesc_o, (kk > 0 || !first_of_group) ? 1u : 0u);
         tc_commit(&kv_empty[s]);
-        tc_commit(&p_empty[j & 1]);
+        tc_commit(&p_empty[g]);
+        if (cur.j + 2 > cur.qt) tc_commit(&o_done[g]);    // the group's last tile of this item
+        if (cur.j == cur.qt) tc_commit(&q_empty[cur.k & 1]);
+        cur = nx;
       }
     }
   } else {
     // ------------------------------------------------------------------ softmax
-    const int grp = (warp - 2) >> 2;             // key tiles j with j % 2 == grp
+    const int grp = (warp - 2) >> 2;             // key tiles with global counter parity grp
     const int q = warp & 3;
-    const int r = q * 32 + lane;                 // query row within the tile
+    const int r = q * 32 + lane;                 // query row within the item
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const uint32_t s_col = S_COL + grp * KT, o_col = O_COL + grp * HD;
+    const uint32_t s_col = S_COL + grp * KT;
     uint8_t* prow = sP + grp * P_BYTES + r * 128;
-    float m = -INFINITY, l = 0.f, alpha_pending = 1.f;
-    float o[HD];
-#pragma unroll
-    for (int d = 0; d < HD; ++d) o[d] = 0.f;
+    int c = 0, d = 0, hcount = 0;                // this group's tiles, items, handovers
+    bool pending = false;                        // an O handover the finisher has not released yet
     bool ok = true;
-
-    auto fold_o = [&](int k) -> bool {          // o = o * alpha + O (this group's k-th tile)
-      if (!mbar_wait(&o_full[grp], k & 1, abort_flag)) return false;
-      tc_fence_after();
+    int G = 0;
+    for (int t = blockIdx.x; t < items.total && ok; t += gridDim.x) {
+      int qt, bh;
+      items.get(t, qt, bh);
+      const int n_kv = qt + 1;
+      const int G0 = G;
+      G += n_kv;
+      float m_ref = -INFINITY, l = 0.f;
+      bool has = false;
+      for (int j = ((G0 & 1) == grp) ? 0 : 1; j < n_kv; j += 2) {
+        if (!mbar_wait(&s_full[grp], c & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const bool diag = (j == qt);
+        // pass 1: row max, 64 columns per TMEM round trip (key j*KT+e after query qt*QT+r masked)
+        float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < HD; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + o_col + c, v);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < KT; c0 += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem + lane_off + s_col + c0, v0);
+          tmem_ld32(tmem + lane_off + s_col + c0 + 32, v1);
+          tmem_wait_ld();
 #pragma unroll
-        for (int d = 0; d < 32; ++d) o[c + d] = o[c + d] * alpha_pending + __uint_as_float(v[d]);
-      }
-      tc_fence_before();
-      mbar_arrive(&o_empty[grp]);
-      return true;
-    };
-
-    int k = 0;
-    for (int j = grp; j < n_kv && ok; j += 2, ++k) {
-      if (!mbar_wait(&s_full[grp], k & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const bool diag = (j == qt);
-      // pass 1: row max (key j*KT+c after query q0+r is masked on the diagonal tile)
-      float mx = -INFINITY;
+          for (int e = 0; e < 32; ++e) {
+            if (!(diag && c0 + e > r)) mx = fmaxf(mx, __uint_as_float(v0[e]));
+            if (!(diag && c0 + 32 + e > r)) mx = fmaxf(mx, __uint_as_float(v1[e]));
+          }
+        }
+        const float m_new = mx * scale_log2;
+        // the group's previous P.V MMA must be done: P buffer free, O stable
+        if (!mbar_wait(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (!has) {
+          m_ref = m_new;
+        } else if (m_new > m_ref + RESCALE_THRESHOLD) {
+          const float f = ex2(m_ref - m_new);
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < HD; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(tmem + lane_off + O_COL + grp * HD + c0, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+            tmem_st16(tmem + lane_off + O_COL + grp * HD + c0, v);
+          }
+          tmem_wait_st();
+          l *= f;
+          m_ref = m_new;
+        }
+        // pass 2: P = 2^(s*scale*log2e - m_ref) to shared memory, row sum
+        float sum = 0.f;
 #pragma unroll 1
-      for (int c0 = 0; c0 < KT; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + s_col + c0, v);
-        tmem_wait_ld();
+        for (int c0 = 0; c0 < KT; c0 += 64) {
+          uint32_t v[64];
+          tmem_ld32(tmem + lane_off + s_col + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(tmem + lane_off + s_col + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_wait_ld();
 #pragma unroll
-        for (int d = 0; d < 32; ++d) {
-          const float x = (diag && c0 + d > r) ? -INFINITY : __uint_as_float(v[d]);
-          mx = fmaxf(mx, x);
+          for (int g8 = 0; g8 < 8; ++g8) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int col = c0 + g8 * 8 + e;
+              p[e] = (diag && col > r) ? 0.f : ex2(__uint_as_float(v[g8 * 8 + e]) * scale_log2 - m_ref);
+              sum += p[e];
+            }
+            uint4 w;
+            w.x = pack_bf16x2(p[0], p[1]);
+            w.y = pack_bf16x2(p[2], p[3]);
+            w.z = pack_bf16x2(p[4], p[5]);
+            w.w = pack_bf16x2(p[6], p[7]);
+            const int chunk = c0 >> 6, gi = g8;
+            *reinterpret_cast<uint4*>(prow + chunk * 16384 + ((gi ^ (r & 7)) << 4)) = w;
+          }
         }
+        l += sum;
+        tc_fence_before();
+        mbar_arrive(&s_empty[grp]);
+        // an O row handed over at the previous item must be read before this group's next MMA
+        if (pending) {
+          if (!mbar_wait(merge_empty, (hcount & 1) ^ 1, abort_flag)) { ok = false; break; }
+          pending = false;
+        }
+        fence_async_smem();
+        mbar_arrive(&p_full[grp]);
+        has = true;
+        ++c;
       }
-      const float m_new = fmaxf(m, mx * scale_log2);
-      const float alpha = ex2(m - m_new);
-      // pass 2: P = 2^(s*scale*log2e - m_new), row sum, P_j to shared memory once the
-      // MMA of this group's previous tile is done reading the buffer
-      if (!mbar_wait(&p_empty[grp], (k & 1) ^ 1, abort_flag)) { ok = false; break; }
-      float sum = 0.f;
+      if (!ok) break;
+      if (has) {
+        if (!mbar_wait(&o_done[grp], d & 1, abort_flag)) { ok = false; break; }
+        ++d;
+      }
+      const int finisher = (G0 + n_kv - 1) & 1;
+      const bool both = n_kv >= 2;
+      if (grp != finisher) {
+        if (both) {
+          // hand (m_ref, l) over; O stays in this group's TMEM columns for the finisher
+          if (pending && !mbar_wait(merge_empty, (hcount & 1) ^ 1, abort_flag)) { ok = false; break; }
+          sML[r * 2] = m_ref;
+          sML[r * 2 + 1] = l;
+          mbar_arrive(merge_full);
+          pending = true;
+          ++hcount;
+        }
+      } else {
+        const int qi = qt * QT + r;
+        float m1 = -INFINITY, l1 = 0.f;
+        if (both) {
+          if (!mbar_wait(merge_full, hcount & 1, abort_flag)) { ok = false; break; }
+          m1 = sML[r * 2];
+          l1 = sML[r * 2 + 1];
+        }
+        tc_fence_after();
+        const float M = fmaxf(m_ref, m1);
+        const float a0 = ex2(m_ref - M), a1 = both ? ex2(m1 - M) : 0.f;
+        const float inv = 1.0f / (l * a0 + l1 * a1);
+        const int b = bh / H, h = bh % H;
+        bf16* orow = out + (long long)(b * T + qi) * C + h * HD;
 #pragma unroll 1
-      for (int c0 = 0; c0 < KT; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + s_col + c0, v);
-        tmem_wait_ld();
-        float p[32];
+        for (int c0 = 0; c0 < HD; c0 += 16) {
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tmem + lane_off + O_COL + grp * HD + c0, v0);
+          if (both) tmem_ld16(tmem + lane_off + O_COL + (grp ^ 1) * HD + c0, v1);
+          tmem_wait_ld();
+          if (qi < T) {
 #pragma unroll
-        for (int d = 0; d < 32; ++d) {
-          const float x = (diag && c0 + d > r) ? -INFINITY : __uint_as_float(v[d]);
-          p[d] = ex2(x * scale_log2 - m_new);
-          sum += p[d];
+            for (int g8 = 0; g8 < 2; ++g8) {
+              float o[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int idx = g8 * 8 + e;
+                o[e] = (__uint_as_float(v0[idx]) * a0 + (both ? __uint_as_float(v1[idx]) * a1 : 0.f)) * inv;
+              }
+              uint4 w;
+              w.x = pack_bf16x2(o[0], o[1]);
+              w.y = pack_bf16x2(o[2], o[3]);
+              w.z = pack_bf16x2(o[4], o[5]);
+              w.w = pack_bf16x2(o[6], o[7]);
+              reinterpret_cast<uint4*>(orow + c0)[g8] = w;
+            }
+          }
         }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint4 w;
-          w.x = pack_bf16x2(p[g * 8 + 0], p[g * 8 + 1]);
-          w.y = pack_bf16x2(p[g * 8 + 2], p[g * 8 + 3]);
-          w.z = pack_bf16x2(p[g * 8 + 4], p[g * 8 + 5]);
-          w.w = pack_bf16x2(p[g * 8 + 6], p[g * 8 + 7]);
-          const int gi = ((c0 & 63) >> 3) + g;
-          *reinterpret_cast<uint4*>(prow + (c0 >> 6) * 16384 + ((gi ^ (r & 7)) << 4)) = w;
+        if (qi < T) lse[(long long)bh * T + qi] = (M + log2f(l * a0 + l1 * a1)) * 0.6931471805599453f;
+        if (both) {
+          tc_fence_before();
+          mbar_arrive(merge_empty);
+          ++hcount;
         }
-      }
-      tc_fence_before();
-      mbar_arrive(&s_empty[grp]);
-      fence_async_smem();
-      mbar_arrive(&p_full[grp]);
-      l = l * alpha + sum;
-      m = m_new;
-      if (k > 0 && !fold_o(k - 1)) { ok = false; break; }
-      alpha_pending = alpha;
-    }
-    if (ok && k > 0) ok = fold_o(k - 1);
-    // merge the two groups' partial states of row r: group 1 hands its (m, l, o) over
-    float* mrow = sMerge + r * MERGE_STRIDE;
-    if (grp == 1) {
-      if (ok) {
-        mrow[0] = m;
-        mrow[1] = l;
-#pragma unroll
-        for (int d = 0; d < HD; ++d) mrow[2 + d] = o[d];
-      }
-      mbar_arrive(merge_bar);
-    } else {
-      ok = ok && mbar_wait(merge_bar, 0, abort_flag);
-      const int qi = q0 + r;
-      if (ok && qi < T) {
-        const float m1 = mrow[0], l1 = mrow[1];
-        const float M = fmaxf(m, m1);
-        const float a0 = ex2(m - M), a1 = ex2(m1 - M);
-        const float L = l * a0 + l1 * a1;
-        const float inv = 1.0f / L;
-        bf16* orow = out + (long long)(row0 + qi) * C + h * HD;
-#pragma unroll
-        for (int g = 0; g < HD / 8; ++g) {
-          float v[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = (o[g * 8 + e] * a0 + mrow[2 + g * 8 + e] * a1) * inv;
-          uint4 w;
-          w.x = pack_bf16x2(v[0], v[1]);
-          w.y = pack_bf16x2(v[2], v[3]);
-          w.z = pack_bf16x2(v[4], v[5]);
-          w.w = pack_bf16x2(v[6], v[7]);
-          reinterpret_cast<uint4*>(orow)[g] = w;
-        }
-        lse[(long long)bh * T + qi] = (M + log2f(L)) * 0.6931471805599453f;
       }
     }
+    if (ok && pending) mbar_wait(merge_empty, (hcount & 1) ^ 1, abort_flag);
   }
 
   tc_fence_before();
@@ -335,7 +421,11 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
       return -3;
     attr = true;
   }
-  const int grid = cdiv(T, QT) * B * H;
+  int dev = 0, nsm = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int total = cdiv(T, QT) * B * H;
+  const int grid = total < nsm ? total : nsm;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, reinterpret_cast<bf16*>(out), lse, B, T, H,
                                                             scale_log2);

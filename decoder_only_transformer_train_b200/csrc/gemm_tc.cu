@@ -26,13 +26,13 @@ constexpr int EPI_THREADS = 256;
 
 template <int BN>
 struct TileCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;   // +1024: manual alignment
-  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;   // power of two >= 2*BN
 };
 
 struct TileSched {
@@ -87,49 +87,26 @@ struct CeRowState {
   int aidx;
 };
 
-// Global reads an epilogue chunk needs (bias, residual / accumulator / GELU input), issued
-// before the chunk's TMEM load so that their latencies overlap.
-__device__ __forceinline__ void epilogue_prefetch(const EpiParams& ep, int m, int n0, float (&b)[32],
-                                                  float (&pre)[32]) {
-  const int N = ep.N;
-  const bool full = (n0 + 32 <= N);
-  const int nvalid = full ? 32 : max(0, N - n0);
-  const bool use_bias = ep.bias != nullptr && (ep.kind == EPI_STORE_ACT || ep.kind == EPI_STORE_F32 ||
-                                               ep.kind == EPI_RESID_F32 || ep.kind == EPI_GELU_FWD);
-  if (use_bias && full) {
-    load_f32x32(ep.bias + n0, b);
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) b[j] = (use_bias && j < nvalid) ? ep.bias[n0 + j] : 0.0f;
-  }
-  if (ep.kind == EPI_RESID_F32 || ep.kind == EPI_ACCUM_F32) {
-    const float* src = (ep.kind == EPI_RESID_F32)
-                           ? reinterpret_cast<const float*>(ep.aux) + (long long)m * ep.ld_aux + n0
-                           : reinterpret_cast<const float*>(ep.C) + (long long)m * ep.ldc + n0;
-    if (full) {
-      load_f32x32(src, pre);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) pre[j] = (j < nvalid) ? src[j] : 0.0f;
-    }
-  } else if (ep.kind == EPI_GELU_BWD) {
-    const bf16* u = reinterpret_cast<const bf16*>(ep.aux) + (long long)m * ep.ld_aux + n0;
-    if (full) {
-      load_bf16x32(u, pre);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) pre[j] = (j < nvalid) ? __bfloat162float(u[j]) : 0.0f;
-    }
-  }
-}
-
-// Epilogue of one 32-column chunk of one output row (b, pre from epilogue_prefetch).
+// Epilogue of one 32-column chunk of one output row.
 __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n0, float (&v)[32], int split,
-                                               CeRowState& ce, const float (&b)[32], const float (&pre)[32]) {
+                                               CeRowState& ce) {
   const int N = ep.N;
   const bool full = (n0 + 32 <= N);
   const int nvalid = full ? 32 : max(0, N - n0);
   const float alpha = ep.alpha;
+  float b[32];
+  if (ep.bias != nullptr && ep.kind != EPI_SPLITK && ep.kind != EPI_ACCUM_F32 && ep.kind != EPI_CE_FWD &&
+      ep.kind != EPI_GELU_BWD) {
+    if (full) {
+      load_f32x32(ep.bias + n0, b);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) b[j] = (j < nvalid) ? ep.bias[n0 + j] : 0.0f;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) b[j] = 0.0f;
+  }
 
   switch (ep.kind) {
     case EPI_STORE_ACT: {
@@ -156,17 +133,34 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
       }
       break;
     }
-    case EPI_ACCUM_F32:
-    case EPI_RESID_F32: {
-      float o[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) o[j] = pre[j] + alpha * v[j] + b[j];
+    case EPI_ACCUM_F32: {
       float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) store_f32x32(c, o);
-      else {
+      if (full) {
+        float o[32];
+        load_f32x32(c, o);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] += alpha * v[j];
+        store_f32x32(c, o);
+      } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = o[j];
+          if (j < nvalid) c[j] += alpha * v[j];
+      }
+      break;
+    }
+    case EPI_RESID_F32: {
+      const float* r = reinterpret_cast<const float*>(ep.aux) + (long long)m * ep.ld_aux + n0;
+      float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
+      if (full) {
+        float o[32];
+        load_f32x32(r, o);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] += alpha * v[j] + b[j];
+        store_f32x32(c, o);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (j < nvalid) c[j] = r[j] + alpha * v[j] + b[j];
       }
       break;
     }
@@ -193,14 +187,18 @@ __device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n
       break;
     }
     case EPI_GELU_BWD: {
+      const bf16* u = reinterpret_cast<const bf16*>(ep.aux) + (long long)m * ep.ld_aux + n0;
       bf16* c = reinterpret_cast<bf16*>(ep.C) + (long long)m * ep.ldc + n0;
+      if (full) {
+        float uu[32];
+        load_bf16x32(u, uu);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_fast(pre[j]);
-      if (full) store_bf16x32(c, v);
-      else {
+        for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_fast(uu[j]);
+        store_bf16x32(c, v);
+      } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = __float2bfloat16_rn(v[j]);
+          if (j < nvalid) c[j] = __float2bfloat16_rn(alpha * v[j] * gelu_tanh_grad_fast(__bfloat162float(u[j])));
       }
       break;
     }
@@ -380,17 +378,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0x7fffffff};
 #pragma unroll 1
       for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
-        const bool live = (m < ep.M && n_base + c < ep.N);
-        float bb[32], pre[32];
-        if (live) epilogue_prefetch(ep, m, n_base + c, bb, pre);
         uint32_t r[32];
         tmem_ld32(tmem_base + acc * BN + c + (static_cast<uint32_t>(q * 32) << 16), r);
         tmem_wait_ld();
-        if (live) {
+        if (m < ep.M && n_base + c < ep.N) {
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          epilogue_chunk(ep, m, n_base + c, v, split, ce, bb, pre);
+          epilogue_chunk(ep, m, n_base + c, v, split, ce);
         }
       }
       if (ep.kind == EPI_CE_FWD && m < ep.M) {
@@ -486,16 +481,56 @@ int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, Til
 int gemm_tc_tile_n(int N) { return N > 128 ? 256 : 128; }
 int gemm_tc_ce_tiles(int N) { return cdiv(N, gemm_tc_tile_n(N)) * 2; }
 
+namespace {
+// Picks the output tile width (128, 192 or 256 columns) and the number of K splits from a
+// small cost model in MMA clock cycles: the busiest SM's tiles x the tile's main loop
+// (narrower tiles re-read more operand bytes per FLOP, hence the efficiency factor), plus
+// for split-K the extra fp32 traffic of the partials and their reduction.
+struct TileChoice {
+  int bn, splits;
+};
+TileChoice choose_tiles(int M, int N, int K, bool can_split, size_t ws_elems, int num_sms, bool fixed_bn) {
+  const int m_tiles = cdiv(M, BM);
+  const int nk = cdiv(K, BK);
+  const int bns[3] = {256, 192, 128};
+  const double eff[3] = {1.0, 0.96, 0.88};
+  TileChoice best{gemm_tc_tile_n(N), 1};
+  double best_cost = 1e300;
+  for (int i = 0; i < 3; ++i) {
+    const int bn = bns[i];
+    if (fixed_bn && bn != gemm_tc_tile_n(N)) continue;
+    if (bn > 128 && N <= 128) continue;
+    const int tiles = m_tiles * cdiv(N, bn);
+    for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
+      if (sp > 1 && (nk / sp < 8 || (size_t)sp * M * N > ws_elems)) break;
+      const int kb = cdiv(nk, sp);
+      const double per_tile = (double)bn * kb * 2.0 / eff[i] + 1500.0;   // MMA clks of a 128 x bn x 64kb tile + overhead
+      const double waves = (double)cdiv(tiles * sp, num_sms);
+      double cost = waves * per_tile;
+      if (sp > 1) cost += (double)(sp + 2) * M * N * 4.0 / 6.0e12 * 1.9e9 + 3000.0;   // partial traffic + reduce launch
+      if (cost < best_cost * 0.999) {
+        best_cost = cost;
+        best = TileChoice{bn, sp};
+      }
+    }
+  }
+  return best;
+}
+}  // namespace
+
 int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long lda, bool a_mn, const void* B,
                  long long ldb, bool b_mn, EpiParams ep, float* ws, size_t ws_elems, int num_sms) {
   if (M <= 0 || N <= 0) return 0;
   if (K <= 0) return -1;
   if (a_mn && !b_mn) return -1;   // not needed by any Linear-layer product
-  const int BN = gemm_tc_tile_n(N);
   ep.M = M;
   ep.N = N;
   // alignment of the vectorised epilogue accesses
   if (ep.kind != EPI_SPLITK && (ep.ldc % 8) != 0) return -1;
+  const bool can_split = (ep.kind == EPI_ACCUM_F32 && ws != nullptr);
+  // the softmax partials of EPI_CE_FWD are laid out per 256/128-column tile
+  const TileChoice tc = choose_tiles(M, N, K, can_split, ws_elems, num_sms, ep.kind == EPI_CE_FWD);
+  const int BN = tc.bn;
   CUtensorMap ta, tb;
   int rc;
   if (!a_mn) rc = encode_bf16_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, BK, BM);
@@ -512,33 +547,28 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   sched.splits = 1;
   sched.kb_per_split = sched.nk;
   EpiParams run = ep;
-  const int mn_tiles = sched.m_tiles * sched.n_tiles;
   bool split = false;
-  if (ep.kind == EPI_ACCUM_F32 && ws != nullptr && mn_tiles < num_sms && sched.nk >= 16) {
-    int s = cdiv(num_sms, mn_tiles);
-    s = min(s, sched.nk / 8);
-    while (s > 1 && (size_t)s * (size_t)M * (size_t)N > ws_elems) --s;
-    if (s > 1) {
-      sched.kb_per_split = cdiv(sched.nk, s);
-      sched.splits = cdiv(sched.nk, sched.kb_per_split);
-      run.kind = EPI_SPLITK;
-      run.ws = ws;
-      split = true;
-    }
+  if (tc.splits > 1) {
+    sched.kb_per_split = cdiv(sched.nk, tc.splits);
+    sched.splits = cdiv(sched.nk, sched.kb_per_split);
+    run.kind = EPI_SPLITK;
+    run.ws = ws;
+    split = true;
   }
   if (ep.kind == EPI_CE_FWD) {
     run.n_ctiles = sched.n_tiles * 2;
     run.ce_tile_n = BN / 2;
   }
-  if (BN == 256) {
-    if (!a_mn && !b_mn) rc = launch_tc<256, false, false>(st, ta, tb, sched, run, num_sms);
-    else if (!a_mn && b_mn) rc = launch_tc<256, false, true>(st, ta, tb, sched, run, num_sms);
-    else rc = launch_tc<256, true, true>(st, ta, tb, sched, run, num_sms);
-  } else {
-    if (!a_mn && !b_mn) rc = launch_tc<128, false, false>(st, ta, tb, sched, run, num_sms);
-    else if (!a_mn && b_mn) rc = launch_tc<128, false, true>(st, ta, tb, sched, run, num_sms);
-    else rc = launch_tc<128, true, true>(st, ta, tb, sched, run, num_sms);
-  }
+#define LAUNCH_BN(BNV)                                                                           \
+  do {                                                                                           \
+    if (!a_mn && !b_mn) rc = launch_tc<BNV, false, false>(st, ta, tb, sched, run, num_sms);     \
+    else if (!a_mn && b_mn) rc = launch_tc<BNV, false, true>(st, ta, tb, sched, run, num_sms);  \
+    else rc = launch_tc<BNV, true, true>(st, ta, tb, sched, run, num_sms);                       \
+  } while (0)
+  if (BN == 256) LAUNCH_BN(256);
+  else if (BN == 192) LAUNCH_BN(192);
+  else LAUNCH_BN(128);
+#undef LAUNCH_BN
   if (rc) return rc;
   if (split) {
     const long long total = (long long)M * N;

@@ -178,22 +178,27 @@ __global__ void ln_param_reduce_kernel(const float* __restrict__ part, int nbloc
 }
 
 // ================================================================ bias gradients
-// out[n] += sum_m x[m, n], rows in chunks of COLSUM_ROWS summed in order, then chunks
-// summed in order.
-constexpr int COLSUM_ROWS = 256;
+// out[n] += sum_m x[m, n]: partial sums over COLSUM_CHUNKS row chunks, each in a fixed
+// order, then the chunks summed in order.
+constexpr int COLSUM_CHUNKS = 8;   // row chunks (partials per column)
+// Block: 8 column groups of 8 columns x 32 row lanes.  Thread (cx, ry) sums rows
+// ry, ry+32, ... of its chunk for columns c0..c0+7 with 16-byte loads; the 32 row lanes are
+// then added in order through shared memory.
 template <typename T>
-__global__ void colsum_partial_kernel(const T* __restrict__ x, long long ldx, int M, int N,
-                                      float* __restrict__ part) {
-  const int n0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;   // 8 consecutive columns per thread
-  if (n0 >= N) return;
-  const int m0 = blockIdx.y * COLSUM_ROWS, m1 = min(M, m0 + COLSUM_ROWS);
+__global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict__ x, long long ldx, int M, int N,
+                                                             float* __restrict__ part) {
+  __shared__ float red[32][65];
+  const int cx = threadIdx.x & 7, ry = threadIdx.x >> 3;
+  const int c0 = blockIdx.x * 64 + cx * 8;
+  const int rows = cdiv(M, COLSUM_CHUNKS);
+  const int m0 = blockIdx.y * rows, m1 = min(M, m0 + rows);
   float s[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) s[i] = 0.f;
-  if (n0 + 8 <= N) {
+  if (c0 + 8 <= N) {
 #pragma unroll 4
-    for (int m = m0; m < m1; ++m) {
-      const T* p = x + (long long)m * ldx + n0;
+    for (int m = m0 + ry; m < m1; m += 32) {
+      const T* p = x + (long long)m * ldx + c0;
       if (sizeof(T) == 2) {
         const uint4 q = *reinterpret_cast<const uint4*>(p);
         const uint32_t* u = reinterpret_cast<const uint32_t*>(&q);
@@ -211,12 +216,19 @@ __global__ void colsum_partial_kernel(const T* __restrict__ x, long long ldx, in
       }
     }
   } else {
-    for (int m = m0; m < m1; ++m)
-      for (int i = 0; i < 8 && n0 + i < N; ++i) s[i] += ld_f(x + (long long)m * ldx + n0 + i);
+    for (int m = m0 + ry; m < m1; m += 32)
+      for (int i = 0; i < 8 && c0 + i < N; ++i) s[i] += ld_f(x + (long long)m * ldx + c0 + i);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (n0 + i < N) part[(long long)blockIdx.y * N + n0 + i] = s[i];
+  for (int i = 0; i < 8; ++i) red[ry][cx * 8 + i] = s[i];
+  __syncthreads();
+  if (threadIdx.x < 64) {
+    const int c = blockIdx.x * 64 + threadIdx.x;
+    float t = 0.f;
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) t += red[r][threadIdx.x];
+    if (c < N) part[(long long)blockIdx.y * N + c] = t;
+  }
 }
 __global__ void colsum_reduce_kernel(const float* __restrict__ part, int nchunks, int N, float* __restrict__ out) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
@@ -675,14 +687,14 @@ int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const float* dy, const f
   return ok();
 }
 
-int colsum_chunks(int M) { return cdiv(M, COLSUM_ROWS); }
+int colsum_chunks(int M) { return COLSUM_CHUNKS; }
 
 int launch_colsum(cudaStream_t st, bool is_bf16, const void* x, long long ldx, int M, int N, float* part,
                   int nchunks, float* out) {
-  if (N % 8 != 0 || ldx % 8 != 0) return -4;
-  dim3 grid(cdiv(N / 8, 128), nchunks);
-  if (is_bf16) colsum_partial_kernel<bf16><<<grid, 128, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, part);
-  else colsum_partial_kernel<float><<<grid, 128, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, part);
+  if (N % 8 != 0 || ldx % 8 != 0 || nchunks != COLSUM_CHUNKS) return -4;
+  dim3 grid(cdiv(N, 64), nchunks);
+  if (is_bf16) colsum_partial_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, part);
+  else colsum_partial_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, part);
   colsum_reduce_kernel<<<cdiv(N, 256), 256, 0, st>>>(part, nchunks, N, out);
   note_kernel_launches(2);
   return ok();

@@ -94,8 +94,24 @@ def test_gemm_split_k_weight_gradient_shape_is_deterministic():
     assert torch.equal(outs[0], outs[1])
 
 
+@pytest.mark.parametrize("M,N,K", [(3072, 768, 4096), (2304, 768, 4096), (768, 3072, 4096), (768, 768, 8192)])
+def test_gemm_weight_gradient_shapes_tile_choices(M, N, K):
+    """dW += dY^T X on the weight-gradient shapes, where the launcher picks 128/192/256-wide
+    tiles and split-K by its cost model."""
+    dY = bf16_round(_randn((M, K), 71 + M))
+    X = bf16_round(_randn((N, K), 73 + N))
+    Ad, lda = _layout(dY, True)
+    Bd, ldb = _layout(X, True)
+    ws = torch.empty(8 * 4 * 768 * 768, dtype=torch.float32, device="cuda")
+    C = torch.full((M, N), 0.25, dtype=torch.float32, device="cuda")
+    BD.gemm_bf16(Ad, Bd, C, M, N, K, lda, ldb, N, True, True, epilogue=2, alpha=0.5, workspace=ws)
+    torch.cuda.synchronize()
+    assert rel_l2(C.cpu() - 0.25, 0.5 * (dY @ X.T)) < 2e-5
+
+
 # ------------------------------------------------------------------ attention
-ATTN_CASES = [(2, 64, 4, 16), (1, 200, 2, 64), (2, 256, 3, 64), (1, 1, 2, 64), (3, 130, 1, 32)]
+ATTN_CASES = [(2, 64, 4, 16), (1, 200, 2, 64), (2, 256, 3, 64), (1, 1, 2, 64), (3, 130, 1, 32), (2, 1024, 12, 64),
+              (3, 384, 100, 64)]
 
 
 @pytest.mark.parametrize("prec", [BD.GPT2_FP32, BD.GPT2_BF16])
