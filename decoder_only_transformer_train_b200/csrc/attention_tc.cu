@@ -46,6 +46,107 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Paired fp32 arithmetic (one instruction for two lanes of data): a*b+c and a+b.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// Row max of a 128-column S tile in TMEM (64 columns per round trip); on the diagonal
+// tile the keys after query row r are left out.
+template <bool DIAG>
+__device__ __forceinline__ float s_row_max(uint32_t taddr, int r) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c0 = 0; c0 < 128; c0 += 64) {
+    uint32_t v0[32], v1[32];
+    tmem_ld32(taddr + c0, v0);
+    tmem_ld32(taddr + c0 + 32, v1);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      if (DIAG) {
+        const float a = (c0 + e > r) ? -INFINITY : __uint_as_float(v0[e]);
+        const float b = (c0 + e + 1 > r) ? -INFINITY : __uint_as_float(v0[e + 1]);
+        const float c = (c0 + 32 + e > r) ? -INFINITY : __uint_as_float(v1[e]);
+        const float d = (c0 + 33 + e > r) ? -INFINITY : __uint_as_float(v1[e + 1]);
+        mx = max3f(mx, a, b);
+        mx = max3f(mx, c, d);
+      } else {
+        mx = max3f(mx, __uint_as_float(v0[e]), __uint_as_float(v0[e + 1]));
+        mx = max3f(mx, __uint_as_float(v1[e]), __uint_as_float(v1[e + 1]));
+      }
+    }
+  }
+  return mx;
+}
+
+// P = 2^(s * scale_log2 - m_ref) for a 128-column S row, written as bf16 into row r of a
+// 128 x 128 K-major SW128 operand; returns the row sum of P.
+template <bool DIAG>
+__device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint8_t* prow) {
+  float2 sum = make_float2(0.f, 0.f);
+  const float2 sc = make_float2(scale_log2, scale_log2);
+  const float2 nm = make_float2(-m_ref, -m_ref);
+#pragma unroll 1
+  for (int c0 = 0; c0 < 128; c0 += 64) {
+    uint32_t v[64];
+    tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
+    tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+    tmem_wait_ld();
+#pragma unroll
+    for (int g8 = 0; g8 < 8; ++g8) {
+      float p[8];
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        const float2 x = ffma2(make_float2(__uint_as_float(v[g8 * 8 + e]), __uint_as_float(v[g8 * 8 + e + 1])), sc, nm);
+        p[e] = ex2(x.x);
+        p[e + 1] = ex2(x.y);
+        if (DIAG) {
+          const int col = c0 + g8 * 8 + e;
+          if (col > r) p[e] = 0.f;
+          if (col + 1 > r) p[e + 1] = 0.f;
+        }
+        sum = fadd2(sum, make_float2(p[e], p[e + 1]));
+      }
+      uint4 w;
+      w.x = pack_bf16x2(p[0], p[1]);
+      w.y = pack_bf16x2(p[2], p[3]);
+      w.z = pack_bf16x2(p[4], p[5]);
+      w.w = pack_bf16x2(p[6], p[7]);
+      *reinterpret_cast<uint4*>(prow + (c0 >> 6) * 16384 + ((g8 ^ (r & 7)) << 4)) = w;
+    }
+  }
+  return sum.x + sum.y;
+}
 
 // Item order shared by all roles: item t -> (query tile, batch*head), heaviest first.
 struct FwdItems {
@@ -231,20 +332,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         if (!mbar_wait(&s_full[grp], c & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const bool diag = (j == qt);
-        // pass 1: row max, 64 columns per TMEM round trip (key j*KT+e after query qt*QT+r masked)
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c0 = 0; c0 < KT; c0 += 64) {
-          uint32_t v0[32], v1[32];
-          tmem_ld32(tmem + lane_off + s_col + c0, v0);
-          tmem_ld32(tmem + lane_off + s_col + c0 + 32, v1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            if (!(diag && c0 + e > r)) mx = fmaxf(mx, __uint_as_float(v0[e]));
-            if (!(diag && c0 + 32 + e > r)) mx = fmaxf(mx, __uint_as_float(v1[e]));
-          }
-        }
+        const uint32_t srow = tmem + lane_off + s_col;
+        const float mx = diag ? s_row_max<true>(srow, r) : s_row_max<false>(srow, r);
         const float m_new = mx * scale_log2;
         // the group's previous P.V MMA must be done: P buffer free, O stable
         if (!mbar_wait(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -267,31 +356,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
           m_ref = m_new;
         }
         // pass 2: P = 2^(s*scale*log2e - m_ref) to shared memory, row sum
-        float sum = 0.f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < KT; c0 += 64) {
-          uint32_t v[64];
-          tmem_ld32(tmem + lane_off + s_col + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-          tmem_ld32(tmem + lane_off + s_col + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-          tmem_wait_ld();
-#pragma unroll
-          for (int g8 = 0; g8 < 8; ++g8) {
-            float p[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int col = c0 + g8 * 8 + e;
-              p[e] = (diag && col > r) ? 0.f : ex2(__uint_as_float(v[g8 * 8 + e]) * scale_log2 - m_ref);
-              sum += p[e];
-            }
-            uint4 w;
-            w.x = pack_bf16x2(p[0], p[1]);
-            w.y = pack_bf16x2(p[2], p[3]);
-            w.z = pack_bf16x2(p[4], p[5]);
-            w.w = pack_bf16x2(p[6], p[7]);
-            const int chunk = c0 >> 6, gi = g8;
-            *reinterpret_cast<uint4*>(prow + chunk * 16384 + ((gi ^ (r & 7)) << 4)) = w;
-          }
-        }
+        const float sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, prow)
+                               : p_row_store<false>(srow, r, scale_log2, m_ref, prow);
         l += sum;
         tc_fence_before();
         mbar_arrive(&s_empty[grp]);
@@ -644,26 +710,59 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         uint32_t us[32], ud[32];
         tmem_ld32(tmem + lane_off + S_C + c0, us);
         tmem_ld32(tmem + lane_off + DP_C + c0, ud);
-        tmem_wait_ld();
-        float pv[32], dz[32];
+        // per-column scalars (MODE 0: the 32 queries of this chunk), fetched while TMEM loads
+        float nl[32], nd[32];                    // -lse*log2(e) and -D
+        bool col_mask = false;                   // some column of this chunk is past T
+        if (MODE == 0) {
+          const int q0c = t * 128 + c0;
+          if ((T & 3) == 0 && q0c + 32 <= T) {
+            const float4* l4 = reinterpret_cast<const float4*>(lse_bh + q0c);
+            const float4* d4 = reinterpret_cast<const float4*>(D_bh + q0c);
 #pragma unroll
-        for (int d = 0; d < 32; ++d) {
-          const int c = c0 + d;
-          float p, Dv;
-          bool masked;
-          if (MODE == 0) {           // row r = key, column c = query (queries past T are masked)
-            const int qi = t * 128 + c;
-            masked = (diag && (c < r)) || qi >= T;
-            const int qc = masked ? 0 : qi;
-            p = ex2(__uint_as_float(us[d]) * scale_log2 - __ldg(lse_bh + qc) * LOG2E);
-            Dv = __ldg(D_bh + qc);
-          } else {                   // row r = query, column c = key
-            masked = diag && (c > r);
-            p = ex2(__uint_as_float(us[d]) * scale_log2 - row_lse2);
-            Dv = row_D;
+            for (int i = 0; i < 8; ++i) {
+              const float4 a = __ldg(l4 + i), bq = __ldg(d4 + i);
+              nl[4 * i] = -a.x * LOG2E; nl[4 * i + 1] = -a.y * LOG2E; nl[4 * i + 2] = -a.z * LOG2E; nl[4 * i + 3] = -a.w * LOG2E;
+              nd[4 * i] = -bq.x; nd[4 * i + 1] = -bq.y; nd[4 * i + 2] = -bq.z; nd[4 * i + 3] = -bq.w;
+            }
+          } else {
+            col_mask = true;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int qi = q0c + e;
+              nl[e] = (qi < T) ? -__ldg(lse_bh + qi) * LOG2E : 0.f;
+              nd[e] = (qi < T) ? -__ldg(D_bh + qi) : 0.f;
+            }
           }
-          pv[d] = masked ? 0.f : p;
-          dz[d] = masked ? 0.f : p * (__uint_as_float(ud[d]) - Dv);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            nl[e] = -row_lse2;
+            nd[e] = -row_D;
+          }
+        }
+        tmem_wait_ld();
+        const bool need_mask = diag || col_mask;
+        float pv[32], dz[32];
+        const float2 sc = make_float2(scale_log2, scale_log2);
+#pragma unroll
+        for (int d = 0; d < 32; d += 2) {
+          const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc,
+                                 make_float2(nl[d], nl[d + 1]));
+          float2 pp = make_float2(ex2(x.x), ex2(x.y));
+          if (need_mask) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int c = c0 + d + h2;
+              const bool masked = (MODE == 0) ? ((diag && c < r) || t * 128 + c >= T) : (diag && c > r);
+              if (masked) (h2 ? pp.y : pp.x) = 0.f;
+            }
+          }
+          const float2 g = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])),
+                                           make_float2(nd[d], nd[d + 1])));
+          pv[d] = pp.x;
+          pv[d + 1] = pp.y;
+          dz[d] = g.x;
+          dz[d + 1] = g.y;
         }
         if (MODE == 0) store_32_sw128(sP, r, c0, pv);
         store_32_sw128(sDS, r, c0, dz);
