@@ -508,11 +508,11 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
 // accumulates dQ over the key tiles at or before it.
 namespace {
 
-constexpr int BWD_THREADS = 320;   // producer, MMA, 8 elementwise warps
+constexpr int BWD_THREADS = 576;   // producer, MMA, 16 elementwise warps (4 per TMEM lane quarter)
 constexpr int BWD_STAGES = 2;
 // smem: 2 resident tiles (K_j,V_j or Q_i,dO_i) + BWD_STAGES x 2 streamed tiles + 2 P-like
 // 128x128 bf16 operands + barriers
-constexpr int BWD_SMEM = 2 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + 512 + 1024;
+constexpr int BWD_SMEM = 2 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + BWD_STAGES * 1024 + 512 + 1024;
 
 // Writes 32 bf16 values (columns col0 .. col0+31, col0 a multiple of 32) into row r of a
 // 128 x 128 K-major operand stored as two 64-column chunks of 128-byte swizzled rows.
@@ -545,7 +545,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   uint8_t* sB = sA + BWD_STAGES * TILE_BYTES;            // streamed: dO_i (MODE 0) / V_j (MODE 1)
   uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P^T (MODE 0) ; unused (MODE 1)
   uint8_t* sDS = sP + P_BYTES;                           // dZ^T (MODE 0) / dZ (MODE 1)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + P_BYTES);
+  float* sScal = reinterpret_cast<float*>(sDS + P_BYTES); // [BWD_STAGES][lse 128 | D 128] (MODE 0)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sScal + BWD_STAGES * 256);
   uint64_t* r_full = bars;                               // resident tiles loaded
   uint64_t* t_full = bars + 1;                           // [BWD_STAGES]
   uint64_t* t_empty = t_full + BWD_STAGES;               // [BWD_STAGES]
@@ -579,8 +580,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       mbar_init(&t_empty[s], 1);
     }
     mbar_init(sd_full, 1);
-    mbar_init(sd_empty, 256);
-    mbar_init(ps_full, 256);
+    mbar_init(sd_empty, 512);
+    mbar_init(ps_full, 512);
     mbar_init(ps_empty, 1);
     mbar_init(acc_full, 1);
     *abort_flag = 0;
@@ -612,7 +613,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         const int s = n % BWD_STAGES;
         const int t = it0 + n;
         if (!mbar_wait(&t_empty[s], ((n / BWD_STAGES) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&t_full[s], 2 * TILE_BYTES);
+        const bool scal_bulk = (MODE == 0) && (T % 4 == 0) && (t * 128 + 128 <= T);
+        mbar_arrive_expect_tx(&t_full[s], 2 * TILE_BYTES + (scal_bulk ? 1024 : 0));
+        if (scal_bulk) {
+          bulk_load(sScal + s * 256, lse + (long long)bh * T + t * 128, 512, &t_full[s]);
+          bulk_load(sScal + s * 256 + 128, Dbuf + (long long)bh * T + t * 128, 512, &t_full[s]);
+        }
         if (MODE == 0) {
           tma_load_2d(sA + s * TILE_BYTES, &tm_qkv, h * HD, row0 + t * 128, &t_full[s]);      // Q_i
           tma_load_2d(sB + s * TILE_BYTES, &tm_do, h * HD, row0 + t * 128, &t_full[s]);       // dO_i
@@ -685,7 +691,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   } else {
     // ------------------------------------------------------------------ elementwise
     const int q = warp & 3;
-    const int half = (warp - 2) >> 2;            // columns [64*half, 64*half + 64) of each tile
+    const int part = (warp - 2) >> 2;            // columns [32*part, 32*part + 32) of each tile
     const int r = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float LOG2E = 1.4426950408889634f;
@@ -702,73 +708,62 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       const int t = it0 + n;
       if (!mbar_wait(sd_full, n & 1, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      // this thread's 32 columns of S and dP, then the TMEM buffer is released at once
+      const int c0 = part * 32;
+      uint32_t us[32], ud[32];
+      tmem_ld32(tmem + lane_off + S_C + c0, us);
+      tmem_ld32(tmem + lane_off + DP_C + c0, ud);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(sd_empty);
+      const int s = n % BWD_STAGES;
+      const bool scal_bulk = (MODE == 0) && (T % 4 == 0) && (t * 128 + 128 <= T);
+      if (scal_bulk && !mbar_wait(&t_full[s], (n / BWD_STAGES) & 1, abort_flag)) { ok = false; break; }
+      const float* lse_s = sScal + s * 256;
+      const float* D_s = lse_s + 128;
       // the previous tile's MMAs must be done reading the P / dZ operands
       if (!mbar_wait(ps_empty, (n & 1) ^ 1, abort_flag)) { ok = false; break; }
       const bool diag = (t == tile);
-#pragma unroll 1
-      for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 32) {
-        uint32_t us[32], ud[32];
-        tmem_ld32(tmem + lane_off + S_C + c0, us);
-        tmem_ld32(tmem + lane_off + DP_C + c0, ud);
-        // per-column scalars (MODE 0: the 32 queries of this chunk), fetched while TMEM loads
-        float nl[32], nd[32];                    // -lse*log2(e) and -D
-        bool col_mask = false;                   // some column of this chunk is past T
+      const bool need_mask = diag || (MODE == 0 && t * 128 + 128 > T);
+      const float2 sc = make_float2(scale_log2, scale_log2);
+      float pv[32], dz[32];
+#pragma unroll
+      for (int d = 0; d < 32; d += 2) {
+        const int c = c0 + d;
+        float2 nl, nd;
         if (MODE == 0) {
-          const int q0c = t * 128 + c0;
-          if ((T & 3) == 0 && q0c + 32 <= T) {
-            const float4* l4 = reinterpret_cast<const float4*>(lse_bh + q0c);
-            const float4* d4 = reinterpret_cast<const float4*>(D_bh + q0c);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 a = __ldg(l4 + i), bq = __ldg(d4 + i);
-              nl[4 * i] = -a.x * LOG2E; nl[4 * i + 1] = -a.y * LOG2E; nl[4 * i + 2] = -a.z * LOG2E; nl[4 * i + 3] = -a.w * LOG2E;
-              nd[4 * i] = -bq.x; nd[4 * i + 1] = -bq.y; nd[4 * i + 2] = -bq.z; nd[4 * i + 3] = -bq.w;
-            }
+          if (scal_bulk) {
+            const float2 lv = *reinterpret_cast<const float2*>(lse_s + c);
+            const float2 dv = *reinterpret_cast<const float2*>(D_s + c);
+            nl = make_float2(-lv.x * LOG2E, -lv.y * LOG2E);
+            nd = make_float2(-dv.x, -dv.y);
           } else {
-            col_mask = true;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int qi = q0c + e;
-              nl[e] = (qi < T) ? -__ldg(lse_bh + qi) * LOG2E : 0.f;
-              nd[e] = (qi < T) ? -__ldg(D_bh + qi) : 0.f;
-            }
+            const int qi = t * 128 + c;
+            nl = make_float2(qi < T ? -__ldg(lse_bh + qi) * LOG2E : 0.f, qi + 1 < T ? -__ldg(lse_bh + qi + 1) * LOG2E : 0.f);
+            nd = make_float2(qi < T ? -__ldg(D_bh + qi) : 0.f, qi + 1 < T ? -__ldg(D_bh + qi + 1) : 0.f);
           }
         } else {
+          nl = make_float2(-row_lse2, -row_lse2);
+          nd = make_float2(-row_D, -row_D);
+        }
+        const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
+        float2 pp = make_float2(ex2(x.x), ex2(x.y));
+        if (need_mask) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            nl[e] = -row_lse2;
-            nd[e] = -row_D;
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int cm = c + h2;
+            const bool masked = (MODE == 0) ? ((diag && cm < r) || t * 128 + cm >= T) : (diag && cm > r);
+            if (masked) (h2 ? pp.y : pp.x) = 0.f;
           }
         }
-        tmem_wait_ld();
-        const bool need_mask = diag || col_mask;
-        float pv[32], dz[32];
-        const float2 sc = make_float2(scale_log2, scale_log2);
-#pragma unroll
-        for (int d = 0; d < 32; d += 2) {
-          const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc,
-                                 make_float2(nl[d], nl[d + 1]));
-          float2 pp = make_float2(ex2(x.x), ex2(x.y));
-          if (need_mask) {
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int c = c0 + d + h2;
-              const bool masked = (MODE == 0) ? ((diag && c < r) || t * 128 + c >= T) : (diag && c > r);
-              if (masked) (h2 ? pp.y : pp.x) = 0.f;
-            }
-          }
-          const float2 g = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])),
-                                           make_float2(nd[d], nd[d + 1])));
-          pv[d] = pp.x;
-          pv[d + 1] = pp.y;
-          dz[d] = g.x;
-          dz[d + 1] = g.y;
-        }
-        if (MODE == 0) store_32_sw128(sP, r, c0, pv);
-        store_32_sw128(sDS, r, c0, dz);
+        const float2 g = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])), nd));
+        pv[d] = pp.x;
+        pv[d + 1] = pp.y;
+        dz[d] = g.x;
+        dz[d + 1] = g.y;
       }
-      tc_fence_before();
-      mbar_arrive(sd_empty);
+      if (MODE == 0) store_32_sw128(sP, r, c0, pv);
+      store_32_sw128(sDS, r, c0, dz);
       fence_async_smem();
       mbar_arrive(ps_full);
     }
@@ -780,16 +775,16 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       const int nacc = (MODE == 0) ? 2 : 1;
       for (int a = 0; a < nacc; ++a) {
         // MODE 0: a=0 dV (column block 2C), a=1 dK (column block C, times scale); MODE 1: dQ (times scale).
-        // Each warp of a lane quarter writes 32 of the 64 head columns.
-        const uint32_t col = ((a == 0) ? A0_C : A1_C) + half * 32;
+        // Each of the 4 warps of a lane quarter writes 16 of the 64 head columns.
+        const uint32_t col = ((a == 0) ? A0_C : A1_C) + part * 16;
         const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
-        bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C)) + half * 32;
-        uint32_t u[32];
-        tmem_ld32(tmem + lane_off + col, u);
+        bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C)) + part * 16;
+        uint32_t u[16];
+        tmem_ld16(tmem + lane_off + col, u);
         tmem_wait_ld();
         if (gi < T) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
+          for (int g = 0; g < 2; ++g) {
             uint4 w;
             w.x = pack_bf16x2(__uint_as_float(u[g * 8 + 0]) * mul, __uint_as_float(u[g * 8 + 1]) * mul);
             w.y = pack_bf16x2(__uint_as_float(u[g * 8 + 2]) * mul, __uint_as_float(u[g * 8 + 3]) * mul);
