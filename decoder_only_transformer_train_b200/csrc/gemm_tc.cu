@@ -4,8 +4,13 @@
 // Roles inside one persistent CTA (320 threads, one CTA per SM):
 //   warp 0      : TMA producer (one elected lane) - stages of A and B tiles
 //   warp 1      : TMEM allocator + MMA issuer (one elected lane)
-//   warps 2..9  : epilogue - tcgen05.ld of the fp32 accumulator, fused math, stores;
-//                 two warps per TMEM lane quarter, each taking half of the tile's columns
+//   warps 2..9  : epilogue - tcgen05.ld of the fp32 accumulator, fused math; two warps
+//                 per TMEM lane quarter, each taking half of the tile's columns.  Each warp
+//                 owns a 32-row slab: thread r computes row r, writes it into a small
+//                 64-byte-swizzled shared buffer, and one lane moves the 32 x 64-byte box
+//                 to global memory with a TMA store (inputs the epilogue needs - residual,
+//                 accumulator, GELU pre-activation - arrive the same way by TMA load), so
+//                 global traffic is in full lines rather than per-row 16-byte pieces.
 // The accumulator is double-buffered in TMEM (2 x BN columns) so the epilogue of one
 // output tile overlaps the main loop of the next.
 //
@@ -24,245 +29,168 @@ constexpr int BK = 64;             // 64 bf16 = one 128-byte swizzle row
 constexpr int NUM_THREADS = 320;
 constexpr int EPI_THREADS = 256;
 
+constexpr int BOX_BYTES = 2048;     // one epilogue staging box: 32 rows x 64 bytes
+
 template <int BN>
 struct TileCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 5 : 6);
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 4 : 6);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STG_BYTES = 8 * 2 * BOX_BYTES;   // 8 epilogue warps x 2 boxes
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;   // +1024: manual alignment
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES + 1024;   // +1024: manual alignment
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;   // power of two >= 2*BN
 };
 
+// Tile order: with few column tiles (n_fast) the column tiles of one row block are
+// neighbours, so the CTAs working on them at the same time share each A tile (read once
+// from HBM); otherwise the row tiles of one column block are neighbours and share B.
 struct TileSched {
-  int m_tiles, n_tiles, splits, nk, kb_per_split;
+  int m_tiles, n_tiles, splits, nk, kb_per_split, n_fast;
   __device__ __forceinline__ int num_tiles() const { return m_tiles * n_tiles * splits; }
   __device__ __forceinline__ void decode(int t, int& tm, int& tn, int& split, int& kb0, int& kb1) const {
     const int mn = m_tiles * n_tiles;
     split = t / mn;
     const int r = t - split * mn;
-    tm = r % m_tiles;
-    tn = r / m_tiles;
+    if (n_fast) {
+      tn = r % n_tiles;
+      tm = r / n_tiles;
+    } else {
+      tm = r % m_tiles;
+      tn = r / m_tiles;
+    }
     kb0 = split * kb_per_split;
     kb1 = min(nk, kb0 + kb_per_split);
   }
 };
-
-__device__ __forceinline__ void load_f32x32(const float* p, float (&o)[32]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float4 q = reinterpret_cast<const float4*>(p)[i];
-    o[4 * i] = q.x; o[4 * i + 1] = q.y; o[4 * i + 2] = q.z; o[4 * i + 3] = q.w;
-  }
-}
-__device__ __forceinline__ void store_f32x32(float* p, const float (&o)[32]) {
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    reinterpret_cast<float4*>(p)[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
-}
-__device__ __forceinline__ void store_bf16x32(bf16* p, const float (&o)[32]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 q;
-    q.x = pack_bf16x2(o[8 * i + 0], o[8 * i + 1]);
-    q.y = pack_bf16x2(o[8 * i + 2], o[8 * i + 3]);
-    q.z = pack_bf16x2(o[8 * i + 4], o[8 * i + 5]);
-    q.w = pack_bf16x2(o[8 * i + 6], o[8 * i + 7]);
-    reinterpret_cast<uint4*>(p)[i] = q;
-  }
-}
-__device__ __forceinline__ void load_bf16x32(const bf16* p, float (&o)[32]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 q = reinterpret_cast<const uint4*>(p)[i];
-    float2 a = unpack_bf16x2(q.x), b = unpack_bf16x2(q.y), c = unpack_bf16x2(q.z), d = unpack_bf16x2(q.w);
-    o[8 * i + 0] = a.x; o[8 * i + 1] = a.y; o[8 * i + 2] = b.x; o[8 * i + 3] = b.y;
-    o[8 * i + 4] = c.x; o[8 * i + 5] = c.y; o[8 * i + 6] = d.x; o[8 * i + 7] = d.y;
-  }
-}
 
 struct CeRowState {
   float mx, sum, amax;
   int aidx;
 };
 
-// Epilogue of one 32-column chunk of one output row.
-__device__ __forceinline__ void epilogue_chunk(const EpiParams& ep, int m, int n0, float (&v)[32], int split,
-                                               CeRowState& ce) {
-  const int N = ep.N;
-  const bool full = (n0 + 32 <= N);
-  const int nvalid = full ? 32 : max(0, N - n0);
-  const float alpha = ep.alpha;
-  float b[32];
-  if (ep.bias != nullptr && ep.kind != EPI_SPLITK && ep.kind != EPI_ACCUM_F32 && ep.kind != EPI_CE_FWD &&
-      ep.kind != EPI_GELU_BWD) {
-    if (full) {
-      load_f32x32(ep.bias + n0, b);
-    } else {
+// Softmax partials of the cross-entropy for one 32-column chunk of one logits row, from
+// the fp32 accumulator.
+__device__ __forceinline__ void ce_row_chunk(const EpiParams& ep, int m, int n0, const float (&v)[32], CeRowState& ce) {
+  const int nvalid = min(32, ep.N - n0);
+  float cmax = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) b[j] = (j < nvalid) ? ep.bias[n0 + j] : 0.0f;
+  for (int j = 0; j < 32; ++j)
+    if (j < nvalid) {
+      if (v[j] > ce.amax) { ce.amax = v[j]; ce.aidx = n0 + j; }
+      cmax = fmaxf(cmax, v[j]);
     }
-  } else {
+  const float nmx = fmaxf(ce.mx, cmax);
+  float s = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) b[j] = 0.0f;
-  }
-
-  switch (ep.kind) {
-    case EPI_STORE_ACT: {
+  for (int j = 0; j < 32; ++j)
+    if (j < nvalid) s += __expf(v[j] - nmx);
+  ce.sum = ce.sum * __expf(ce.mx - nmx) + s;
+  ce.mx = nmx;
+  const int y = ep.targets[m];
+  if (y >= n0 && y < n0 + nvalid) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] + b[j];
-      bf16* c = reinterpret_cast<bf16*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) store_bf16x32(c, v);
-      else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = __float2bfloat16_rn(v[j]);
-      }
-      break;
-    }
-    case EPI_STORE_F32: {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] + b[j];
-      float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) store_f32x32(c, v);
-      else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = v[j];
-      }
-      break;
-    }
-    case EPI_ACCUM_F32: {
-      float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) {
-        float o[32];
-        load_f32x32(c, o);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] += alpha * v[j];
-        store_f32x32(c, o);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] += alpha * v[j];
-      }
-      break;
-    }
-    case EPI_RESID_F32: {
-      const float* r = reinterpret_cast<const float*>(ep.aux) + (long long)m * ep.ld_aux + n0;
-      float* c = reinterpret_cast<float*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) {
-        float o[32];
-        load_f32x32(r, o);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] += alpha * v[j] + b[j];
-        store_f32x32(c, o);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = r[j] + alpha * v[j] + b[j];
-      }
-      break;
-    }
-    case EPI_GELU_FWD: {
-      bf16* u = reinterpret_cast<bf16*>(ep.aux_out) + (long long)m * ep.ld_aux_out + n0;
-      bf16* c = reinterpret_cast<bf16*>(ep.C) + (long long)m * ep.ldc + n0;
-      float g[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        v[j] = alpha * v[j] + b[j];
-        g[j] = gelu_tanh_fast(v[j]);
-      }
-      if (full) {
-        store_bf16x32(u, v);
-        store_bf16x32(c, g);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) {
-            u[j] = __float2bfloat16_rn(v[j]);
-            c[j] = __float2bfloat16_rn(g[j]);
-          }
-      }
-      break;
-    }
-    case EPI_GELU_BWD: {
-      const bf16* u = reinterpret_cast<const bf16*>(ep.aux) + (long long)m * ep.ld_aux + n0;
-      bf16* c = reinterpret_cast<bf16*>(ep.C) + (long long)m * ep.ldc + n0;
-      if (full) {
-        float uu[32];
-        load_bf16x32(u, uu);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] * gelu_tanh_grad_fast(uu[j]);
-        store_bf16x32(c, v);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = __float2bfloat16_rn(alpha * v[j] * gelu_tanh_grad_fast(__bfloat162float(u[j])));
-      }
-      break;
-    }
-    case EPI_CE_FWD: {
-      bf16* c = reinterpret_cast<bf16*>(ep.C) + (long long)m * ep.ldc + n0;
-      float cmax = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        v[j] *= alpha;
-        if (j < nvalid) {
-          if (v[j] > ce.amax) { ce.amax = v[j]; ce.aidx = n0 + j; }
-          cmax = fmaxf(cmax, v[j]);
-        }
-      }
-      if (nvalid > 0) {
-        const float nmx = fmaxf(ce.mx, cmax);
-        float s = 0.0f;
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) s += __expf(v[j] - nmx);
-        ce.sum = ce.sum * __expf(ce.mx - nmx) + s;
-        ce.mx = nmx;
-        const int y = ep.targets[m];
-        if (y >= n0 && y < n0 + nvalid) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (n0 + j == y) ep.zt[m] = v[j];
-        }
-      }
-      if (full) store_bf16x32(c, v);
-      else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) c[j] = __float2bfloat16_rn(v[j]);
-      }
-      break;
-    }
-    case EPI_SPLITK: {
-      float* w = ep.ws + ((long long)split * ep.M + m) * (long long)N + n0;
-      if (full && (N % 4 == 0)) store_f32x32(w, v);
-      else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (j < nvalid) w[j] = v[j];
-      }
-      break;
-    }
-    default:
-      break;
+    for (int j = 0; j < 32; ++j)
+      if (n0 + j == y) ep.zt[m] = v[j];
   }
 }
+
+// Byte offset of 16-byte granule g (0..3) of row r in a 32 x 64-byte box stored with the
+// TMA 64-byte swizzle (granule index XOR bits 7-8 of the address).
+__device__ __forceinline__ uint32_t box_off(int r, int g) { return r * 64 + ((g ^ ((r >> 1) & 3)) << 4); }
+
+__device__ __forceinline__ void box_put_bf16(uint8_t* box, int r, const float* v) {   // 32 values
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+    w.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+    w.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+    w.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+    *reinterpret_cast<uint4*>(box + box_off(r, g)) = w;
+  }
+}
+__device__ __forceinline__ void box_get_bf16(const uint8_t* box, int r, float* v) {   // 32 values
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const uint4 w = *reinterpret_cast<const uint4*>(box + box_off(r, g));
+    const float2 a = unpack_bf16x2(w.x), b = unpack_bf16x2(w.y), c = unpack_bf16x2(w.z), d = unpack_bf16x2(w.w);
+    v[8 * g + 0] = a.x; v[8 * g + 1] = a.y; v[8 * g + 2] = b.x; v[8 * g + 3] = b.y;
+    v[8 * g + 4] = c.x; v[8 * g + 5] = c.y; v[8 * g + 6] = d.x; v[8 * g + 7] = d.y;
+  }
+}
+__device__ __forceinline__ void box_put_f32(uint8_t* box, int r, const float* v) {    // 16 values
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    *reinterpret_cast<float4*>(box + box_off(r, g)) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+}
+__device__ __forceinline__ void box_get_f32(const uint8_t* box, int r, float* v) {    // 16 values
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const float4 w = *reinterpret_cast<const float4*>(box + box_off(r, g));
+    v[4 * g] = w.x; v[4 * g + 1] = w.y; v[4 * g + 2] = w.z; v[4 * g + 3] = w.w;
+  }
+}
+
+__device__ __forceinline__ bool kind_has_bias(int kind) {
+  return kind == EPI_STORE_ACT || kind == EPI_STORE_F32 || kind == EPI_RESID_F32 || kind == EPI_GELU_FWD;
+}
+__device__ __forceinline__ bool kind_out_bf16(int kind) {
+  return kind == EPI_STORE_ACT || kind == EPI_GELU_FWD || kind == EPI_GELU_BWD || kind == EPI_CE_FWD;
+}
+
+// Per-warp epilogue state: two staging boxes used alternately, and the warp's mbarrier for
+// TMA loads of epilogue inputs.
+struct EpiWarp {
+  uint8_t* box0;
+  uint8_t* box1;
+  uint64_t* bar;
+  uint32_t bar_phase;
+  int cur;
+  volatile int* abort_flag;
+  int lane;
+  // wait until the box about to be reused is no longer read by an earlier TMA store
+  __device__ __forceinline__ uint8_t* acquire() {
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+    return cur ? box1 : box0;
+  }
+  __device__ __forceinline__ bool load(uint8_t* b, const CUtensorMap* map, int x, int y) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, BOX_BYTES);
+      tma_load_2d(b, map, x, y, bar);
+    }
+    const bool ok = mbar_wait(bar, bar_phase, abort_flag);
+    bar_phase ^= 1;
+    return ok;
+  }
+  __device__ __forceinline__ void store(uint8_t* b, const CUtensorMap* map, int x, int y) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(map, x, y, b);
+      bulk_commit_group();
+    }
+    cur ^= 1;
+  }
+};
 
 template <int BN, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               TileSched sched, EpiParams ep) {
+               const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmIn,
+               const __grid_constant__ CUtensorMap tmOut2, TileSched sched, EpiParams ep) {
   using Cfg = TileCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint8_t* stg = smem + Cfg::STAGES * Cfg::STAGE_BYTES;                       // epilogue boxes
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(stg + Cfg::STG_BYTES);
   uint64_t* empty_bar = full_bar + Cfg::STAGES;
   uint64_t* tfull_bar = empty_bar + Cfg::STAGES;
   uint64_t* tempty_bar = tfull_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + 2);
+  uint64_t* epi_bar = tempty_bar + 2;             // [8] one per epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -277,10 +205,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_init(&tfull_bar[a], 1);
       mbar_init(&tempty_bar[a], EPI_THREADS);
     }
+    for (int w = 0; w < 8; ++w) mbar_init(&epi_bar[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmOut);
+    tma_prefetch_desc(&tmIn);
+    tma_prefetch_desc(&tmOut2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -366,29 +298,112 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;        // which half of the tile's columns
     const int row = q * 32 + lane;
+    const int ew = warp - 2;
+    EpiWarp E;
+    E.box0 = stg + (ew * 2) * BOX_BYTES;
+    E.box1 = stg + (ew * 2 + 1) * BOX_BYTES;
+    E.bar = &epi_bar[ew];
+    E.bar_phase = 0;
+    E.cur = 0;
+    E.abort_flag = abort_flag;
+    E.lane = lane;
+    const int kind = ep.kind;
+    const bool out_bf16 = kind_out_bf16(kind);
+    const bool use_bias = ep.bias != nullptr && kind_has_bias(kind);
+    const float alpha = ep.alpha;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
       int tm, tn, split, kb0, kb1;
       sched.decode(t, tm, tn, split, kb0, kb1);
       if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const int m = tm * BM + row;
+      const int m_warp = tm * BM + q * 32;                      // first row of this warp's slab
+      const int y_out = (kind == EPI_SPLITK) ? split * ep.ld_aux + m_warp : m_warp;   // ws rows per split: ld_aux
       const int n_base = tn * BN;
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0x7fffffff};
 #pragma unroll 1
-      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2); c += 32) {
+      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2) && ok; c += 32) {
         uint32_t r[32];
         tmem_ld32(tmem_base + acc * BN + c + (static_cast<uint32_t>(q * 32) << 16), r);
         tmem_wait_ld();
-        if (m < ep.M && n_base + c < ep.N) {
-          float v[32];
+        const int n0 = n_base + c;
+        if (n0 >= ep.N || m_warp >= ep.M) continue;            // warp-uniform
+        float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          epilogue_chunk(ep, m, n_base + c, v, split, ce);
+        for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+        if (kind == EPI_CE_FWD && m < ep.M) ce_row_chunk(ep, m, n0, v, ce);
+        if (out_bf16) {
+          float b[32];
+          if (use_bias && n0 + 32 <= ep.N) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 q4 = reinterpret_cast<const float4*>(ep.bias + n0)[i];
+              b[4 * i] = q4.x; b[4 * i + 1] = q4.y; b[4 * i + 2] = q4.z; b[4 * i + 3] = q4.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) b[j] = (use_bias && n0 + j < ep.N) ? ep.bias[n0 + j] : 0.f;
+          }
+          if (kind == EPI_GELU_FWD) {
+            float u[32], g[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              u[j] = alpha * v[j] + b[j];
+              g[j] = gelu_tanh_fast(u[j]);
+            }
+            uint8_t* bx = E.acquire();
+            box_put_bf16(bx, lane, u);
+            E.store(bx, &tmOut2, n0, m_warp);
+            bx = E.acquire();
+            box_put_bf16(bx, lane, g);
+            E.store(bx, &tmOut, n0, m_warp);
+          } else if (kind == EPI_GELU_BWD) {
+            uint8_t* bx = E.acquire();
+            if (!E.load(bx, &tmIn, n0, m_warp)) { ok = false; break; }
+            float u[32];
+            box_get_bf16(bx, lane, u);
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] = alpha * v[j] * gelu_tanh_grad_fast(u[j]);
+            box_put_bf16(bx, lane, u);
+            E.store(bx, &tmOut, n0, m_warp);
+          } else {   // EPI_STORE_ACT, EPI_CE_FWD
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] + b[j];
+            uint8_t* bx = E.acquire();
+            box_put_bf16(bx, lane, v);
+            E.store(bx, &tmOut, n0, m_warp);
+          }
+        } else {
+          // fp32 output: two 16-column boxes
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int n1 = n0 + hh * 16;
+            if (!ok || n1 >= ep.N) continue;
+            float o[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float bj = (use_bias && n1 + j < ep.N) ? ep.bias[n1 + j] : 0.f;
+              o[j] = (kind == EPI_SPLITK) ? v[hh * 16 + j] : alpha * v[hh * 16 + j] + bj;
+            }
+            uint8_t* bx = E.acquire();
+            if (kind == EPI_RESID_F32 || kind == EPI_ACCUM_F32) {
+              if (!E.load(bx, (kind == EPI_RESID_F32) ? &tmIn : &tmOut, n1, m_warp)) { ok = false; continue; }
+              float in[16];
+              box_get_f32(bx, lane, in);
+              __syncwarp();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) o[j] += in[j];
+            }
+            box_put_f32(bx, lane, o);
+            E.store(bx, &tmOut, n1, y_out);
+          }
         }
       }
-      if (ep.kind == EPI_CE_FWD && m < ep.M) {
+      if (kind == EPI_CE_FWD && m < ep.M) {
         CePartial p;
         p.max = ce.mx;
         p.sum = ce.sum;
@@ -401,6 +416,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (lane == 0) bulk_wait_group<0>();      // every store of this warp has landed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -413,14 +430,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 }
 
 // split-K reduction in fixed split order: C[m,n] += alpha * sum_s ws[s][m][n]
+// ws holds `splits` partial products of Mpad rows each (row-major, N columns).
 __global__ void splitk_reduce_kernel(float* __restrict__ C, long long ldc, const float* __restrict__ ws, int M,
-                                     int N, int splits, float alpha) {
+                                     int Mpad, int N, int splits, float alpha) {
   const long long total = (long long)M * N;
+  const long long per_split = (long long)Mpad * N;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const int m = (int)(i / N), n = (int)(i % N);
     float s = 0.0f;
-    for (int k = 0; k < splits; ++k) s += ws[(long long)k * total + i];
+    for (int k = 0; k < splits; ++k) s += ws[(long long)k * per_split + i];
     C[(long long)m * ldc + n] += alpha * s;
   }
 }
@@ -442,25 +461,36 @@ PFN_tmapEncodeTiled get_encode_fn() {
   return fn;
 }
 
-// bf16 2-D tensor map: `inner` contiguous elements per row, `outer` rows, row pitch ld.
-int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-                   uint32_t box_inner, uint32_t box_outer) {
+// 2-D tensor map: `inner` contiguous elements per row, `outer` rows, row pitch ld elements.
+int encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int esize, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t ld, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   PFN_tmapEncodeTiled fn = get_encode_fn();
   if (fn == nullptr) return -3;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (ld * 2) % 16 != 0) return -1;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (ld * esize) % 16 != 0) return -1;
   cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
+  cuuint64_t strides[1] = {ld * (uint64_t)esize};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? 0 : -3;
+}
+int encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+                   uint32_t box_inner, uint32_t box_outer) {
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, ld, box_inner, box_outer,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+// Epilogue box map: 32 rows x 64 bytes (32 bf16 or 16 fp32 columns), 64-byte swizzle.
+int encode_epi_box(CUtensorMap* map, bool bf16_elems, const void* base, uint64_t cols, uint64_t rows, uint64_t ld) {
+  return bf16_elems ? encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, cols, rows, ld, 32, 32,
+                                CU_TENSOR_MAP_SWIZZLE_64B)
+                    : encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, cols, rows, ld, 16, 32,
+                                CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 template <int BN, bool A_MN, bool B_MN>
-int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, TileSched sched, const EpiParams& ep,
-              int num_sms) {
+int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
+              const CUtensorMap& tin, const CUtensorMap& tout2, TileSched sched, const EpiParams& ep, int num_sms) {
   using Cfg = TileCfg<BN>;
   auto kern = gemm_tc_kernel<BN, A_MN, B_MN>;
   static bool attr_set = false;
@@ -471,7 +501,7 @@ int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, Til
   }
   const int tiles = sched.m_tiles * sched.n_tiles * sched.splits;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  kern<<<grid, NUM_THREADS, Cfg::SMEM, st>>>(ta, tb, sched, ep);
+  kern<<<grid, NUM_THREADS, Cfg::SMEM, st>>>(ta, tb, tout, tin, tout2, sched, ep);
   note_kernel_launches(1);
   return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
@@ -502,7 +532,7 @@ TileChoice choose_tiles(int M, int N, int K, bool can_split, size_t ws_elems, in
     if (bn > 128 && N <= 128) continue;
     const int tiles = m_tiles * cdiv(N, bn);
     for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
-      if (sp > 1 && (nk / sp < 8 || (size_t)sp * M * N > ws_elems)) break;
+      if (sp > 1 && (nk / sp < 8 || (size_t)sp * cdiv(M, BM) * BM * N > ws_elems)) break;
       const int kb = cdiv(nk, sp);
       const double per_tile = (double)bn * kb * 2.0 / eff[i] + 1500.0;   // MMA clks of a 128 x bn x 64kb tile + overhead
       const double waves = (double)cdiv(tiles * sp, num_sms);
@@ -546,6 +576,7 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   sched.nk = cdiv(K, BK);
   sched.splits = 1;
   sched.kb_per_split = sched.nk;
+  sched.n_fast = sched.n_tiles <= 8 ? 1 : 0;
   EpiParams run = ep;
   bool split = false;
   if (tc.splits > 1) {
@@ -559,11 +590,34 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
     run.n_ctiles = sched.n_tiles * 2;
     run.ce_tile_n = BN / 2;
   }
-#define LAUNCH_BN(BNV)                                                                           \
-  do {                                                                                           \
-    if (!a_mn && !b_mn) rc = launch_tc<BNV, false, false>(st, ta, tb, sched, run, num_sms);     \
-    else if (!a_mn && b_mn) rc = launch_tc<BNV, false, true>(st, ta, tb, sched, run, num_sms);  \
-    else rc = launch_tc<BNV, true, true>(st, ta, tb, sched, run, num_sms);                       \
+  // epilogue tensor maps: output, input (residual / accumulator / GELU pre-activation),
+  // second output (GELU pre-activation); unused ones repeat the output map
+  CUtensorMap tout, tin, tout2;
+  const int Mpad = cdiv(M, BM) * BM;
+  if (split) {
+    run.ld_aux = Mpad;   // rows per split in the workspace
+    rc = encode_epi_box(&tout, false, ws, (uint64_t)N, (uint64_t)sched.splits * Mpad, (uint64_t)N);
+  } else {
+    const bool ob = (ep.kind == EPI_STORE_ACT || ep.kind == EPI_GELU_FWD || ep.kind == EPI_GELU_BWD ||
+                     ep.kind == EPI_CE_FWD);
+    rc = encode_epi_box(&tout, ob, ep.C, (uint64_t)N, (uint64_t)M, (uint64_t)ep.ldc);
+  }
+  if (rc) return rc;
+  tin = tout;
+  tout2 = tout;
+  if (!split && ep.kind == EPI_RESID_F32)
+    rc = encode_epi_box(&tin, false, ep.aux, (uint64_t)N, (uint64_t)M, (uint64_t)ep.ld_aux);
+  else if (!split && ep.kind == EPI_GELU_BWD)
+    rc = encode_epi_box(&tin, true, ep.aux, (uint64_t)N, (uint64_t)M, (uint64_t)ep.ld_aux);
+  if (rc) return rc;
+  if (ep.kind == EPI_GELU_FWD)
+    rc = encode_epi_box(&tout2, true, ep.aux_out, (uint64_t)N, (uint64_t)M, (uint64_t)ep.ld_aux_out);
+  if (rc) return rc;
+#define LAUNCH_BN(BNV)                                                                                     \
+  do {                                                                                                     \
+    if (!a_mn && !b_mn) rc = launch_tc<BNV, false, false>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);      \
+    else if (!a_mn && b_mn) rc = launch_tc<BNV, false, true>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);   \
+    else rc = launch_tc<BNV, true, true>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);                       \
   } while (0)
   if (BN == 256) LAUNCH_BN(256);
   else if (BN == 192) LAUNCH_BN(192);
@@ -576,7 +630,7 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
     long long nb = cdivll(total, threads);
     if (nb > (long long)num_sms * 8) nb = (long long)num_sms * 8;
     const int blocks = (int)nb;
-    splitk_reduce_kernel<<<blocks, threads, 0, st>>>(reinterpret_cast<float*>(ep.C), ep.ldc, ws, M, N,
+    splitk_reduce_kernel<<<blocks, threads, 0, st>>>(reinterpret_cast<float*>(ep.C), ep.ldc, ws, M, Mpad, N,
                                                      sched.splits, ep.alpha);
     note_kernel_launches(1);
     if (cudaGetLastError() != cudaSuccess) return -3;
