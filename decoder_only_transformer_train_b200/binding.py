@@ -59,6 +59,7 @@ _PROTOS = {
     "gpt2op_gemm_bf16": (_i, [_vp, _i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _f, _vp, _i64]),
     "gpt2op_attention_fwd": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i]),
     "gpt2op_attention_bwd": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
+    "gpt2op_attention_bwd_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
     "gpt2op_layernorm_fwd": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i]),
     "gpt2op_classifier_aux_floats": (_i64, [_i, _i]),
     "gpt2op_classifier_fwd_bwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -266,6 +267,19 @@ def attention_fwd(qkv, out, lse, B, T, H, head_dim, precision, stream=None):
 def attention_bwd(qkv, out, dout, lse, Dbuf, dqkv, B, T, H, head_dim, precision, stream=None):
     _check(lib().gpt2op_attention_bwd(_stream(stream), precision, _ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse),
                                       _ptr(Dbuf), _ptr(dqkv), B, T, H, head_dim))
+
+
+# Largest B*H*T gpt2op_attention_bwd_noalloc accepts (size of its fixed row-sum array).
+NOALLOC_ATTN_MAX_ROWS = 262144
+
+
+def attention_bwd_noalloc(qkv, out, dout, lse, dqkv, B, T, H, head_dim, precision, stream=None):
+    """attention_bwd without a scratch argument: D lives in the library's fixed array."""
+    rc = lib().gpt2op_attention_bwd_noalloc(_stream(stream), precision, _ptr(qkv), _ptr(out), _ptr(dout),
+                                            _ptr(lse), _ptr(dqkv), B, T, H, head_dim)
+    if rc != GPT2_OK and B * H * T > NOALLOC_ATTN_MAX_ROWS:
+        raise Gpt2Error(rc, f"B*H*T = {B * H * T} exceeds the fixed scratch of {NOALLOC_ATTN_MAX_ROWS} rows")
+    _check(rc)
 
 
 def layernorm_fwd(x, w, b, y, mean, rstd, N, C, precision, stream=None):

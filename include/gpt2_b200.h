@@ -168,6 +168,25 @@ int gpt2op_attention_fwd(void* stream, int precision, const void* qkv, void* out
 int gpt2op_attention_bwd(void* stream, int precision, const void* qkv, const void* out, const void* dout,
                          const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int head_dim);
 
+/* The same backward with no scratch argument and no device allocation.  The pages have
+ * no counterpart: it is an interface for callers that cannot allocate (a C caller with no
+ * allocator of its own, or one whose device memory a caching allocator has reserved
+ * up front and that cannot afford the device-wide synchronisation of cudaFree).
+ * D = rowsum(dO * O) goes to one fixed f32 array of GPT2OP_NOALLOC_ATTN_MAX_ROWS entries
+ * (1 MiB) compiled into the library, one per device.
+ *   - Arguments, layouts and results are those of gpt2op_attention_bwd minus Dbuf.
+ *   - GPT2_ERR_SHAPE if B, T, H or head_dim <= 0 or B*H*T > GPT2OP_NOALLOC_ATTN_MAX_ROWS;
+ *     this check runs before any CUDA call.  GPT2_ERR_ARG for a null pointer or an
+ *     unknown precision.
+ *   - The first call on each device looks up the array's address (cudaGetSymbolAddress)
+ *     and caches it; make that first call before any stream capture begins.
+ *   - Nothing needs to start at zero: the call writes every row sum before reading it.
+ *   - The array is shared by all callers in the process: calls whose executions overlap
+ *     on one device (different streams, concurrent host threads) race on it. */
+#define GPT2OP_NOALLOC_ATTN_MAX_ROWS 262144
+int gpt2op_attention_bwd_noalloc(void* stream, int precision, const void* qkv, const void* out, const void* dout,
+                                 const float* lse, void* dqkv, int B, int T, int H, int head_dim);
+
 /* LayerNorm forward over rows of x (f32 [N, C]): y (bf16 or f32 by precision), mean and
  * rstd (f32 [N]); eps 1e-5, biased variance (nn.LayerNorm defaults). */
 int gpt2op_layernorm_fwd(void* stream, int precision, const float* x, const float* w, const float* b, void* y,
