@@ -66,33 +66,53 @@ struct TileSched {
 };
 
 struct CeRowState {
-  float mx, sum, amax;
+  float mx, sum, amax, zt;
   int aidx;
 };
 
+constexpr float CE_LOG2E = 1.4426950408889634f;
+
 // Softmax partials of the cross-entropy for one 32-column chunk of one logits row, from
-// the fp32 accumulator.
-__device__ __forceinline__ void ce_row_chunk(const EpiParams& ep, int m, int n0, const float (&v)[32], CeRowState& ce) {
-  const int nvalid = min(32, ep.N - n0);
-  float cmax = -INFINITY;
+// the fp32 accumulator: running max and sum of exp(v - max) (online rescaling), the first
+// column reaching the running maximum (argmax), and the target column's logit.  Columns
+// at or past N (nvalid < 32) count as -inf.
+__device__ __forceinline__ void ce_row_chunk(int n0, int nvalid, int y, const float (&v)[32], CeRowState& ce) {
+  float w[32];
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (j < nvalid) {
-      if (v[j] > ce.amax) { ce.amax = v[j]; ce.aidx = n0 + j; }
-      cmax = fmaxf(cmax, v[j]);
-    }
+  for (int j = 0; j < 32; ++j) w[j] = (j < nvalid) ? v[j] : -INFINITY;
+  // chunk max as a shallow tree of 3-input maxima
+  float t[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) t[i] = max3f(w[3 * i], w[3 * i + 1], w[3 * i + 2]);
+  t[10] = fmaxf(w[30], w[31]);
+  const float cmax = fmaxf(max3f(max3f(t[0], t[1], t[2]), max3f(t[3], t[4], t[5]), max3f(t[6], t[7], t[8])),
+                           fmaxf(t[9], t[10]));
+  if (cmax > ce.amax) {   // strictly greater: an earlier column keeps a tie
+    uint32_t mask = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) mask |= (w[j] == cmax ? 1u : 0u) << j;
+    ce.amax = cmax;
+    ce.aidx = n0 + __ffs(mask) - 1;
+  }
   const float nmx = fmaxf(ce.mx, cmax);
-  float s = 0.0f;
+  const float2 l2e = make_float2(CE_LOG2E, CE_LOG2E);
+  const float2 off = make_float2(-nmx * CE_LOG2E, -nmx * CE_LOG2E);
+  float2 acc[4];
 #pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (j < nvalid) s += __expf(v[j] - nmx);
-  ce.sum = ce.sum * __expf(ce.mx - nmx) + s;
+  for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    const float2 x = ffma2(make_float2(w[j], w[j + 1]), l2e, off);   // (v - max) log2 e
+    acc[(j >> 1) & 3] = fadd2(acc[(j >> 1) & 3], make_float2(ex2(x.x), ex2(x.y)));
+  }
+  const float2 s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+  ce.sum = ce.sum * ex2((ce.mx - nmx) * CE_LOG2E) + (s2.x + s2.y);
   ce.mx = nmx;
-  const int y = ep.targets[m];
-  if (y >= n0 && y < n0 + nvalid) {
+  const int jt = y - n0;
+  if (jt >= 0 && jt < nvalid) {
 #pragma unroll
     for (int j = 0; j < 32; ++j)
-      if (n0 + j == y) ep.zt[m] = v[j];
+      if (j == jt) ce.zt = v[j];
   }
 }
 
@@ -323,7 +343,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int m_warp = tm * BM + q * 32;                      // first row of this warp's slab
       const int y_out = (kind == EPI_SPLITK) ? split * ep.ld_aux + m_warp : m_warp;   // ws rows per split: ld_aux
       const int n_base = tn * BN;
-      CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0x7fffffff};
+      CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0.0f, 0x7fffffff};
+      const int y_row = (kind == EPI_CE_FWD && m < ep.M) ? ep.targets[m] : -1;
 #pragma unroll 1
       for (int c = half * (BN / 2); c < (half + 1) * (BN / 2) && ok; c += 32) {
         uint32_t r[32];
@@ -334,7 +355,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (kind == EPI_CE_FWD && m < ep.M) ce_row_chunk(ep, m, n0, v, ce);
+        if (kind == EPI_CE_FWD && m < ep.M) ce_row_chunk(n0, min(32, ep.N - n0), y_row, v, ce);
         if (out_bf16) {
           float b[32];
           if (use_bias && n0 + 32 <= ep.N) {
@@ -410,6 +431,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         p.amax = ce.amax;
         p.aidx = ce.aidx;
         ep.ce_part[(long long)m * ep.n_ctiles + tn * 2 + half] = p;
+        const int n_lo = n_base + half * (BN / 2);
+        if (y_row >= n_lo && y_row < min(n_lo + BN / 2, ep.N)) ep.zt[m] = ce.zt;
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[acc]);
@@ -430,17 +453,40 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 }
 
 // split-K reduction in fixed split order: C[m,n] += alpha * sum_s ws[s][m][n]
-// ws holds `splits` partial products of Mpad rows each (row-major, N columns).
-__global__ void splitk_reduce_kernel(float* __restrict__ C, long long ldc, const float* __restrict__ ws, int M,
-                                     int Mpad, int N, int splits, float alpha) {
-  const long long total = (long long)M * N;
+// ws holds `splits` (<= 8) partial products of Mpad rows each (row-major, N columns).  Each
+// thread handles 4 consecutive columns with 16-byte accesses (N % 4 == 0, ldc % 4 == 0 and a
+// 16-byte aligned C, which the fp32 tensor maps of the split path already require) and has
+// all the splits' loads in flight before it adds them in split order.
+__global__ void __launch_bounds__(256) splitk_reduce_kernel(float* __restrict__ C, long long ldc,
+                                                            const float* __restrict__ ws, int M, int Mpad, int N,
+                                                            int splits, float alpha) {
+  const int nq = N >> 2;
+  const long long total = (long long)M * nq;
   const long long per_split = (long long)Mpad * N;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
-    const int m = (int)(i / N), n = (int)(i % N);
-    float s = 0.0f;
-    for (int k = 0; k < splits; ++k) s += ws[(long long)k * per_split + i];
-    C[(long long)m * ldc + n] += alpha * s;
+    const int m = (int)(i / nq), q = (int)(i - (long long)m * nq);
+    const float* src = ws + (long long)m * N + 4 * q;
+    float4 v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k < splits) v[k] = __ldcs(reinterpret_cast<const float4*>(src + k * per_split));
+    float4 acc = v[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k)
+      if (k < splits) {
+        acc.x += v[k].x;
+        acc.y += v[k].y;
+        acc.z += v[k].z;
+        acc.w += v[k].w;
+      }
+    float4* dst = reinterpret_cast<float4*>(C + (long long)m * ldc + 4 * q);
+    float4 c = *dst;
+    c.x += alpha * acc.x;
+    c.y += alpha * acc.y;
+    c.z += alpha * acc.z;
+    c.w += alpha * acc.w;
+    *dst = c;
   }
 }
 
@@ -532,7 +578,7 @@ TileChoice choose_tiles(int M, int N, int K, bool can_split, size_t ws_elems, in
     if (bn > 128 && N <= 128) continue;
     const int tiles = m_tiles * cdiv(N, bn);
     for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
-      if (sp > 1 && (nk / sp < 8 || (size_t)sp * cdiv(M, BM) * BM * N > ws_elems)) break;
+      if (sp > 1 && (nk / sp < 8 || N % 4 != 0 || (size_t)sp * cdiv(M, BM) * BM * N > ws_elems)) break;
       const int kb = cdiv(nk, sp);
       const double per_tile = (double)bn * kb * 2.0 / eff[i] + 1500.0;   // MMA clks of a 128 x bn x 64kb tile + overhead
       const double waves = (double)cdiv(tiles * sp, num_sms);
@@ -557,7 +603,8 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   ep.N = N;
   // alignment of the vectorised epilogue accesses
   if (ep.kind != EPI_SPLITK && (ep.ldc % 8) != 0) return -1;
-  const bool can_split = (ep.kind == EPI_ACCUM_F32 && ws != nullptr);
+  const bool can_split = (ep.kind == EPI_ACCUM_F32 && ws != nullptr && (reinterpret_cast<uintptr_t>(ep.C) % 16) == 0 &&
+                         (reinterpret_cast<uintptr_t>(ws) % 16) == 0);
   // the softmax partials of EPI_CE_FWD are laid out per 256/128-column tile
   const TileChoice tc = choose_tiles(M, N, K, can_split, ws_elems, num_sms, ep.kind == EPI_CE_FWD);
   const int BN = tc.bn;
@@ -625,7 +672,7 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
 #undef LAUNCH_BN
   if (rc) return rc;
   if (split) {
-    const long long total = (long long)M * N;
+    const long long total = (long long)M * (N / 4);
     const int threads = 256;
     long long nb = cdivll(total, threads);
     if (nb > (long long)num_sms * 8) nb = (long long)num_sms * 8;

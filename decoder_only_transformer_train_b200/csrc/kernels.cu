@@ -157,24 +157,42 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict_
   }
 }
 
-__global__ void ln_param_reduce_kernel(const float* __restrict__ part, int nblocks, int C, float* __restrict__ dw,
-                                       float* __restrict__ db, float* __restrict__ dbias_out) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= 3 * C) return;
-  if (c >= 2 * C && dbias_out == nullptr) return;
+// Block: 32 columns x 16 row groups.  Row group r sums partial rows r, r+16, r+32, ... in
+// that order (8 loads in flight), then the 16 group sums are added in group order, so the
+// result does not depend on timing.
+constexpr int LNP_GROUPS = 16;
+__global__ void __launch_bounds__(32 * LNP_GROUPS) ln_param_reduce_kernel(const float* __restrict__ part, int nblocks,
+                                                                         int C, float* __restrict__ dw,
+                                                                         float* __restrict__ db,
+                                                                         float* __restrict__ dbias_out) {
+  __shared__ float red[LNP_GROUPS][33];
+  const int lane = threadIdx.x & 31, r = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
+  const int ncols = dbias_out ? 3 * C : 2 * C;
+  const long long ld = 3LL * C;
   float s = 0.f;
-  int b = 0;
-  for (; b + 8 <= nblocks; b += 8) {   // loads first, then the sum in block order
-    float v[8];
+  if (c < ncols) {
+    for (int b0 = r; b0 < nblocks; b0 += LNP_GROUPS * 8) {
+      float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = part[(long long)(b + i) * 3 * C + c];
+      for (int i = 0; i < 8; ++i) {
+        const int b = b0 + LNP_GROUPS * i;
+        v[i] = (b < nblocks) ? part[(long long)b * ld + c] : 0.f;
+      }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s += v[i];
+      for (int i = 0; i < 8; ++i) s += v[i];
+    }
   }
-  for (; b < nblocks; ++b) s += part[(long long)b * 3 * C + c];
-  if (c < C) dw[c] += s;
-  else if (c < 2 * C) db[c - C] += s;
-  else dbias_out[c - 2 * C] += s;
+  red[r][lane] = s;
+  __syncthreads();
+  if (r == 0 && c < ncols) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < LNP_GROUPS; ++i) t += red[i][lane];
+    if (c < C) dw[c] += t;
+    else if (c < 2 * C) db[c - C] += t;
+    else dbias_out[c - 2 * C] += t;
+  }
 }
 
 // ================================================================ bias gradients
@@ -682,7 +700,8 @@ int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const float* dy, const f
                    : ln_bwd_dispatch<float>(st, dy, x, mean, rstd, w, dres, reinterpret_cast<float*>(dres_act),
                                             accumulate, part, nblocks, N, C);
   if (rc) return rc;
-  ln_param_reduce_kernel<<<cdiv(3 * C, 256), 256, 0, st>>>(part, nblocks, C, dw, db, dbias_out);
+  ln_param_reduce_kernel<<<cdiv(dbias_out ? 3 * C : 2 * C, 32), 32 * LNP_GROUPS, 0, st>>>(part, nblocks, C, dw, db,
+                                                                                         dbias_out);
   note_kernel_launches(1);
   return ok();
 }
