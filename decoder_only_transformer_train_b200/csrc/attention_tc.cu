@@ -504,8 +504,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   uint8_t* sR1 = sR0 + TILE_BYTES;                       // resident: V_j (MODE 0) / dO_i (MODE 1)
   uint8_t* sA = sR1 + TILE_BYTES;                        // streamed: Q_i (MODE 0) / K_j (MODE 1)
   uint8_t* sB = sA + BWD_STAGES * TILE_BYTES;            // streamed: dO_i (MODE 0) / V_j (MODE 1)
-  uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P^T (MODE 0) ; unused (MODE 1)
-  uint8_t* sDS = sP + P_BYTES;                           // dZ^T (MODE 0) / dZ (MODE 1)
+  uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P (MODE 0) ; unused (MODE 1)
+  uint8_t* sDS = sP + P_BYTES;                           // dZ, a query per row
   float* sScal = reinterpret_cast<float*>(sDS + P_BYTES); // [BWD_STAGES][lse 128 | D 128] (MODE 0)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sScal + BWD_STAGES * 256);
   uint64_t* r_full = bars;                               // resident tiles loaded
@@ -593,7 +593,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_sq = make_idesc_bf16(128, 128, false, false);   // 128x128, K=64, both K-major
-      constexpr uint32_t idesc_acc = make_idesc_bf16(128, HD, false, true);    // 128x64, K=128, B MN-major
+      constexpr uint32_t idesc_acc = make_idesc_bf16(128, HD, MODE == 0, true);  // 128x64, K=128, B MN-major;
+                                                                                 // A MN-major in MODE 0
       bool ok = mbar_wait(r_full, 0, abort_flag);
       const uint32_t r0 = smem_u32(sR0), r1 = smem_u32(sR1);
       auto issue_sd = [&](int n) -> bool {
@@ -605,10 +606,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           if (MODE == 0) {
-            // S^T = K_j Q_i^T ; dP^T = V_j dO_i^T
-            tc_mma_bf16(tmem + S_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
+            // S = Q_i K_j^T ; dP = dO_i V_j^T   (rows: the streamed query tile)
+            tc_mma_bf16(tmem + S_C, make_sdesc_sw128(a + k * 32, 16, 1024), make_sdesc_sw128(r0 + k * 32, 16, 1024),
                         idesc_sq, k > 0 ? 1u : 0u);
-            tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024), make_sdesc_sw128(bq + k * 32, 16, 1024),
+            tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(bq + k * 32, 16, 1024), make_sdesc_sw128(r1 + k * 32, 16, 1024),
                         idesc_sq, k > 0 ? 1u : 0u);
           } else {
             // S = Q_i K_j^T ; dP = dO_i V_j^T
@@ -633,10 +634,12 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         for (int k = 0; k < 8; ++k) {
           const uint32_t koff = (k >> 2) * 16384 + (k & 3) * 32;
           if (MODE == 0) {
-            // dV += P^T dO_i ; dK += dZ^T Q_i   (B operands MN-major: [128 queries x 64])
-            tc_mma_bf16(tmem + A0_C, make_sdesc_sw128(smem_u32(sP) + koff, 16, 1024),
+            // dV += P^T dO_i ; dK += dZ^T Q_i.  P and dZ are stored with a query per row (keys in
+            // two 64-column halves 16 KB apart), which read as MN-major A operands (M = keys,
+            // K = queries: 16 query rows = 2 KB per step); B operands MN-major: [128 queries x 64]
+            tc_mma_bf16(tmem + A0_C, make_sdesc_sw128(smem_u32(sP) + k * 2048, 16384, 1024),
                         make_sdesc_sw128(bq + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
-            tc_mma_bf16(tmem + A1_C, make_sdesc_sw128(dsA + koff, 16, 1024),
+            tc_mma_bf16(tmem + A1_C, make_sdesc_sw128(dsA + k * 2048, 16384, 1024),
                         make_sdesc_sw128(a + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
           } else {
             // dQ += dZ K_j
@@ -685,35 +688,35 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       // the previous tile's MMAs must be done reading the P / dZ operands
       if (!mbar_wait(ps_empty, (n & 1) ^ 1, abort_flag)) { ok = false; break; }
       const bool diag = (t == tile);
-      const bool need_mask = diag || (MODE == 0 && t * 128 + 128 > T);
+      // both kernels hold S with a query per row (thread r); MODE 0 streams the query tiles,
+      // so its row's lse and D change with t
+      bool row_out = false;   // a query row past T (MODE 0, last tile only)
+      if (MODE == 0) {
+        const int qi = t * 128 + r;
+        row_out = qi >= T;
+        if (scal_bulk) {
+          row_lse2 = lse_s[r] * LOG2E;
+          row_D = D_s[r];
+        } else {
+          row_lse2 = row_out ? 0.f : __ldg(lse_bh + qi) * LOG2E;
+          row_D = row_out ? 0.f : __ldg(D_bh + qi);
+        }
+      }
+      const bool need_mask = diag || row_out;
       const float2 sc = make_float2(scale_log2, scale_log2);
+      const float2 nl = make_float2(-row_lse2, -row_lse2);
+      const float2 nd = make_float2(-row_D, -row_D);
       float pv[32], dz[32];
 #pragma unroll
       for (int d = 0; d < 32; d += 2) {
         const int c = c0 + d;
-        float2 nl, nd;
-        if (MODE == 0) {
-          if (scal_bulk) {
-            const float2 lv = *reinterpret_cast<const float2*>(lse_s + c);
-            const float2 dv = *reinterpret_cast<const float2*>(D_s + c);
-            nl = make_float2(-lv.x * LOG2E, -lv.y * LOG2E);
-            nd = make_float2(-dv.x, -dv.y);
-          } else {
-            const int qi = t * 128 + c;
-            nl = make_float2(qi < T ? -__ldg(lse_bh + qi) * LOG2E : 0.f, qi + 1 < T ? -__ldg(lse_bh + qi + 1) * LOG2E : 0.f);
-            nd = make_float2(qi < T ? -__ldg(D_bh + qi) : 0.f, qi + 1 < T ? -__ldg(D_bh + qi + 1) : 0.f);
-          }
-        } else {
-          nl = make_float2(-row_lse2, -row_lse2);
-          nd = make_float2(-row_D, -row_D);
-        }
         const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
         float2 pp = make_float2(ex2(x.x), ex2(x.y));
         if (need_mask) {
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int cm = c + h2;
-            const bool masked = (MODE == 0) ? ((diag && cm < r) || t * 128 + cm >= T) : (diag && cm > r);
+            const bool masked = row_out || (diag && cm > r);   // causal: key cm after query r
             if (masked) (h2 ? pp.y : pp.x) = 0.f;
           }
         }
