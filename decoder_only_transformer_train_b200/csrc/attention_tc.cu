@@ -471,28 +471,47 @@ namespace {
 
 constexpr int BWD_THREADS = 576;   // producer, MMA, 16 elementwise warps (4 per TMEM lane quarter)
 constexpr int BWD_STAGES = 2;
-// smem: 2 resident tiles (K_j,V_j or Q_i,dO_i) + BWD_STAGES x 2 streamed tiles + 2 P-like
-// 128x128 bf16 operands + barriers
-constexpr int BWD_SMEM = 2 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + BWD_STAGES * 1024 + 512 + 1024;
+// smem: two buffers of the 2 resident tiles (K_j,V_j or Q_i,dO_i: this item's and the next
+// one's), BWD_STAGES x 2 streamed tiles, the 128x128 bf16 operands (P and dZ) and barriers
+constexpr int BWD_SMEM = 4 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + 512 + 1024;
+static_assert(BWD_SMEM <= 232448, "attention backward shared memory");
 
-// Writes 32 bf16 values (columns col0 .. col0+31, col0 a multiple of 32) into row r of a
-// 128 x 128 K-major operand stored as two 64-column chunks of 128-byte swizzled rows.
-__device__ __forceinline__ void store_32_sw128(uint8_t* base, int r, int col0, const float* v) {
+// Writes 32 bf16 values, packed in pairs (columns col0 .. col0+31, col0 a multiple of 32),
+// into row r of a 128 x 128 operand stored as two 64-column halves of 128-byte swizzled rows.
+__device__ __forceinline__ void store_32_sw128(uint8_t* base, int r, int col0, const uint32_t* w16) {
   uint8_t* row = base + (col0 >> 6) * 16384 + r * 128;
   const int g0 = (col0 & 63) >> 3;
 #pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    uint4 w;
-    w.x = pack_bf16x2(v[g * 8 + 0], v[g * 8 + 1]);
-    w.y = pack_bf16x2(v[g * 8 + 2], v[g * 8 + 3]);
-    w.z = pack_bf16x2(v[g * 8 + 4], v[g * 8 + 5]);
-    w.w = pack_bf16x2(v[g * 8 + 6], v[g * 8 + 7]);
-    *reinterpret_cast<uint4*>(row + (((g0 + g) ^ (r & 7)) << 4)) = w;
-  }
+  for (int g = 0; g < 4; ++g)
+    *reinterpret_cast<uint4*>(row + (((g0 + g) ^ (r & 7)) << 4)) =
+        make_uint4(w16[g * 4 + 0], w16[g * 4 + 1], w16[g * 4 + 2], w16[g * 4 + 3]);
 }
 
-// MODE 0: dK/dV kernel (CTA = key tile j; streams Q_i, dO_i for i >= j)
-// MODE 1: dQ kernel    (CTA = query tile i; streams K_j, V_j for j <= i)
+// Work items of the backward: (128-row tile, batch*head), heaviest first.
+//   MODE 0 (dK/dV): item = key tile j, streams the query tiles i >= j  (n_t - j of them)
+//   MODE 1 (dQ):    item = query tile i, streams the key tiles j <= i  (i + 1 of them)
+struct BwdItem {
+  int tile, bh, it0, it1;
+};
+template <int MODE>
+__device__ __forceinline__ BwdItem bwd_item(int idx, int BH, int n_t) {
+  BwdItem w;
+  w.tile = (MODE == 0) ? idx / BH : n_t - 1 - idx / BH;
+  w.bh = idx % BH;
+  w.it0 = (MODE == 0) ? w.tile : 0;
+  w.it1 = (MODE == 0) ? n_t : w.tile + 1;
+  return w;
+}
+// Item of a CTA's k-th turn: a snake over the grid (turn k takes items k*G .. k*G + G - 1,
+// odd turns in reverse), which evens out the heaviest-first item sizes across CTAs.
+__device__ __forceinline__ int bwd_turn_item(int k) {
+  return k * (int)gridDim.x + ((k & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
+}
+
+// MODE 0: dK/dV kernel;  MODE 1: dQ kernel.  Persistent: each CTA walks its items in turn.
+// Both hold S and dP with a query per TMEM lane.  Resident tiles and the TMEM accumulators
+// are double-buffered across items, so the next item's loads and first S / dP products
+// overlap the current item's last tile and epilogue.
 template <int MODE>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
@@ -500,51 +519,49 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
                    int T, int H, float scale, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sR0 = smem;                                   // resident: K_j (MODE 0) / Q_i (MODE 1)
-  uint8_t* sR1 = sR0 + TILE_BYTES;                       // resident: V_j (MODE 0) / dO_i (MODE 1)
-  uint8_t* sA = sR1 + TILE_BYTES;                        // streamed: Q_i (MODE 0) / K_j (MODE 1)
+  uint8_t* sRes = smem;                                  // [2][K_j,V_j (MODE 0) / Q_i,dO_i (MODE 1)]
+  uint8_t* sA = sRes + 4 * TILE_BYTES;                   // streamed: Q_i (MODE 0) / K_j (MODE 1)
   uint8_t* sB = sA + BWD_STAGES * TILE_BYTES;            // streamed: dO_i (MODE 0) / V_j (MODE 1)
-  uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P (MODE 0) ; unused (MODE 1)
+  uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P (MODE 0), a query per row
   uint8_t* sDS = sP + P_BYTES;                           // dZ, a query per row
-  float* sScal = reinterpret_cast<float*>(sDS + P_BYTES); // [BWD_STAGES][lse 128 | D 128] (MODE 0)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sScal + BWD_STAGES * 256);
-  uint64_t* r_full = bars;                               // resident tiles loaded
-  uint64_t* t_full = bars + 1;                           // [BWD_STAGES]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + P_BYTES);
+  uint64_t* r_full = bars;                               // [2] resident tiles loaded
+  uint64_t* r_empty = r_full + 2;                        // [2] resident tiles no longer read
+  uint64_t* t_full = r_empty + 2;                        // [BWD_STAGES]
   uint64_t* t_empty = t_full + BWD_STAGES;               // [BWD_STAGES]
   uint64_t* sd_full = t_empty + BWD_STAGES;              // S and dP in TMEM
   uint64_t* sd_empty = sd_full + 1;                      // S and dP read out
   uint64_t* ps_full = sd_empty + 1;                      // operands in smem
   uint64_t* ps_empty = ps_full + 1;                      // operands consumed
-  uint64_t* acc_full = ps_empty + 1;                     // accumulation done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+  uint64_t* acc_full = ps_empty + 1;                     // [2] an item's accumulation done
+  uint64_t* acc_empty = acc_full + 2;                    // [2] an item's accumulators read out
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_t = cdiv(T, 128);
   const int BH = B * H;
-  // heaviest CTAs first: key tile 0 (MODE 0) / the last query tile (MODE 1) loop longest
-  const int tile = (MODE == 0) ? (int)(blockIdx.x / BH) : n_t - 1 - (int)(blockIdx.x / BH);
-  const int bh = (int)(blockIdx.x % BH);
-  const int b = bh / H, h = bh % H;
+  const int n_items = n_t * BH;
   const int C = H * HD;
-  const int row0 = b * T;
-  const int it0 = (MODE == 0) ? tile : 0;                // streamed tiles [it0, it1)
-  const int it1 = (MODE == 0) ? n_t : tile + 1;
-  const int n_it = it1 - it0;
-  // TMEM columns: S [0,128), dP [128,256), acc0 [256,320) (dV or dQ), acc1 [320,384) (dK)
-  const uint32_t S_C = 0, DP_C = 128, A0_C = 256, A1_C = 320;
+  // TMEM columns: S [0,128), dP [128,256); accumulator buffer a at 256 + 128 a:
+  // acc0 (dV or dQ) 64 columns, acc1 (dK) the next 64
+  const uint32_t S_C = 0, DP_C = 128, ACC_C = 256;
 
   if (threadIdx.x == 0) {
-    mbar_init(r_full, 1);
-    for (int s = 0; s < BWD_STAGES; ++s) {
-      mbar_init(&t_full[s], 1);
-      mbar_init(&t_empty[s], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&r_full[i], 1);
+      mbar_init(&r_empty[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], 512);
+    }
+    for (int i = 0; i < BWD_STAGES; ++i) {
+      mbar_init(&t_full[i], 1);
+      mbar_init(&t_empty[i], 1);
     }
     mbar_init(sd_full, 1);
     mbar_init(sd_empty, 512);
     mbar_init(ps_full, 512);
     mbar_init(ps_empty, 1);
-    mbar_init(acc_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
@@ -562,47 +579,53 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   if (warp == 0) {
     if (lane == 0) {
       // ---------------------------------------------------------------- TMA producer
-      mbar_arrive_expect_tx(r_full, 2 * TILE_BYTES);
-      if (MODE == 0) {
-        tma_load_2d(sR0, &tm_qkv, C + h * HD, row0 + tile * 128, r_full);       // K_j
-        tma_load_2d(sR1, &tm_qkv, 2 * C + h * HD, row0 + tile * 128, r_full);   // V_j
-      } else {
-        tma_load_2d(sR0, &tm_qkv, h * HD, row0 + tile * 128, r_full);           // Q_i
-        tma_load_2d(sR1, &tm_do, h * HD, row0 + tile * 128, r_full);            // dO_i
-      }
-      for (int n = 0; n < n_it; ++n) {
-        const int s = n % BWD_STAGES;
-        const int t = it0 + n;
-        if (!mbar_wait(&t_empty[s], ((n / BWD_STAGES) & 1) ^ 1, abort_flag)) break;
-        const bool scal_bulk = (MODE == 0) && (T % 4 == 0) && (t * 128 + 128 <= T);
-        mbar_arrive_expect_tx(&t_full[s], 2 * TILE_BYTES + (scal_bulk ? 1024 : 0));
-        if (scal_bulk) {
-          bulk_load(sScal + s * 256, lse + (long long)bh * T + t * 128, 512, &t_full[s]);
-          bulk_load(sScal + s * 256 + 128, Dbuf + (long long)bh * T + t * 128, 512, &t_full[s]);
-        }
+      int g = 0;   // streamed tiles issued by this CTA (stage ring position)
+      for (int k = 0;; ++k) {
+        const int idx = bwd_turn_item(k);
+        if (idx >= n_items) break;
+        const BwdItem w = bwd_item<MODE>(idx, BH, n_t);
+        const int row0 = (w.bh / H) * T, h = w.bh % H;
+        const int rb = k & 1;
+        if (!mbar_wait(&r_empty[rb], ((k >> 1) & 1) ^ 1, abort_flag)) break;
+        uint8_t* r0 = sRes + rb * 2 * TILE_BYTES;
+        mbar_arrive_expect_tx(&r_full[rb], 2 * TILE_BYTES);
         if (MODE == 0) {
-          tma_load_2d(sA + s * TILE_BYTES, &tm_qkv, h * HD, row0 + t * 128, &t_full[s]);      // Q_i
-          tma_load_2d(sB + s * TILE_BYTES, &tm_do, h * HD, row0 + t * 128, &t_full[s]);       // dO_i
+          tma_load_2d(r0, &tm_qkv, C + h * HD, row0 + w.tile * 128, &r_full[rb]);                  // K_j
+          tma_load_2d(r0 + TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + w.tile * 128, &r_full[rb]);  // V_j
         } else {
-          tma_load_2d(sA + s * TILE_BYTES, &tm_qkv, C + h * HD, row0 + t * 128, &t_full[s]);  // K_j
-          tma_load_2d(sB + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + t * 128, &t_full[s]);  // V_j
+          tma_load_2d(r0, &tm_qkv, h * HD, row0 + w.tile * 128, &r_full[rb]);                      // Q_i
+          tma_load_2d(r0 + TILE_BYTES, &tm_do, h * HD, row0 + w.tile * 128, &r_full[rb]);           // dO_i
         }
+        bool ok = true;
+        for (int t = w.it0; t < w.it1; ++t, ++g) {
+          const int st = g % BWD_STAGES;
+          if (!mbar_wait(&t_empty[st], ((g / BWD_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&t_full[st], 2 * TILE_BYTES);
+          if (MODE == 0) {
+            tma_load_2d(sA + st * TILE_BYTES, &tm_qkv, h * HD, row0 + t * 128, &t_full[st]);          // Q_i
+            tma_load_2d(sB + st * TILE_BYTES, &tm_do, h * HD, row0 + t * 128, &t_full[st]);           // dO_i
+          } else {
+            tma_load_2d(sA + st * TILE_BYTES, &tm_qkv, C + h * HD, row0 + t * 128, &t_full[st]);      // K_j
+            tma_load_2d(sB + st * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + t * 128, &t_full[st]);  // V_j
+          }
+        }
+        if (!ok) break;
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_sq = make_idesc_bf16(128, 128, false, false);   // 128x128, K=64, both K-major
+      constexpr uint32_t idesc_sq = make_idesc_bf16(128, 128, false, false);     // 128x128, K=64, both K-major
       constexpr uint32_t idesc_acc = make_idesc_bf16(128, HD, MODE == 0, true);  // 128x64, K=128, B MN-major;
                                                                                  // A MN-major in MODE 0
-      bool ok = mbar_wait(r_full, 0, abort_flag);
-      const uint32_t r0 = smem_u32(sR0), r1 = smem_u32(sR1);
-      auto issue_sd = [&](int n) -> bool {
-        const int s = n % BWD_STAGES;
-        if (!mbar_wait(&t_full[s], (n / BWD_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait(sd_empty, (n & 1) ^ 1, abort_flag)) return false;
+      // S / dP of the CTA's g-th streamed tile, read against resident buffer rb
+      auto issue_sd = [&](int g, int rb) -> bool {
+        const int st = g % BWD_STAGES;
+        if (!mbar_wait(&t_full[st], (g / BWD_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait(sd_empty, (g & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t a = smem_u32(sA + s * TILE_BYTES), bq = smem_u32(sB + s * TILE_BYTES);
+        const uint32_t a = smem_u32(sA + st * TILE_BYTES), bq = smem_u32(sB + st * TILE_BYTES);
+        const uint32_t r0 = smem_u32(sRes + rb * 2 * TILE_BYTES), r1 = r0 + TILE_BYTES;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
           if (MODE == 0) {
@@ -612,7 +635,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
             tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(bq + k * 32, 16, 1024), make_sdesc_sw128(r1 + k * 32, 16, 1024),
                         idesc_sq, k > 0 ? 1u : 0u);
           } else {
-            // S = Q_i K_j^T ; dP = dO_i V_j^T
+            // S = Q_i K_j^T ; dP = dO_i V_j^T   (rows: the resident query tile)
             tc_mma_bf16(tmem + S_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
                         idesc_sq, k > 0 ? 1u : 0u);
             tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024), make_sdesc_sw128(bq + k * 32, 16, 1024),
@@ -622,35 +645,57 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         tc_commit(sd_full);
         return true;
       };
-      if (ok) ok = issue_sd(0);
-      for (int n = 0; n < n_it && ok; ++n) {
-        if (n + 1 < n_it && !issue_sd(n + 1)) break;
-        const int s = n % BWD_STAGES;
-        if (!mbar_wait(ps_full, n & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a = smem_u32(sA + s * TILE_BYTES), bq = smem_u32(sB + s * TILE_BYTES);
-        const uint32_t dsA = smem_u32(sDS);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t koff = (k >> 2) * 16384 + (k & 3) * 32;
-          if (MODE == 0) {
-            // dV += P^T dO_i ; dK += dZ^T Q_i.  P and dZ are stored with a query per row (keys in
-            // two 64-column halves 16 KB apart), which read as MN-major A operands (M = keys,
-            // K = queries: 16 query rows = 2 KB per step); B operands MN-major: [128 queries x 64]
-            tc_mma_bf16(tmem + A0_C, make_sdesc_sw128(smem_u32(sP) + k * 2048, 16384, 1024),
-                        make_sdesc_sw128(bq + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
-            tc_mma_bf16(tmem + A1_C, make_sdesc_sw128(dsA + k * 2048, 16384, 1024),
-                        make_sdesc_sw128(a + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
-          } else {
-            // dQ += dZ K_j
-            tc_mma_bf16(tmem + A0_C, make_sdesc_sw128(dsA + koff, 16, 1024),
-                        make_sdesc_sw128(a + k * 2048, 8192, 1024), idesc_acc, (n > 0 || k > 0) ? 1u : 0u);
+      bool ok = true;
+      int g = 0;
+      int idx = bwd_turn_item(0);
+      if (idx < n_items) ok = mbar_wait(&r_full[0], 0, abort_flag) && issue_sd(0, 0);
+      for (int k = 0; idx < n_items && ok; ++k) {
+        const BwdItem w = bwd_item<MODE>(idx, BH, n_t);
+        const int n_it = w.it1 - w.it0;
+        const int nidx = bwd_turn_item(k + 1);
+        const int ab = k & 1;
+        const uint32_t acc0 = tmem + ACC_C + ab * 128, acc1 = acc0 + 64;
+        for (int n = 0; n < n_it && ok; ++n, ++g) {
+          // S / dP one tile ahead, possibly the next item's first
+          if (n + 1 < n_it) {
+            ok = issue_sd(g + 1, k & 1);
+          } else if (nidx < n_items) {
+            ok = mbar_wait(&r_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag) && issue_sd(g + 1, (k + 1) & 1);
           }
+          if (!ok) break;
+          // the accumulator buffer must have been read out by item k - 2's epilogue
+          if (n == 0 && !mbar_wait(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int st = g % BWD_STAGES;
+          if (!mbar_wait(ps_full, g & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(sA + st * TILE_BYTES), bq = smem_u32(sB + st * TILE_BYTES);
+          const uint32_t dsA = smem_u32(sDS);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t accum = (n > 0 || kk > 0) ? 1u : 0u;
+            if (MODE == 0) {
+              // dV += P^T dO_i ; dK += dZ^T Q_i.  P and dZ are stored with a query per row (keys in
+              // two 64-column halves 16 KB apart), which read as MN-major A operands (M = keys,
+              // K = queries: 16 query rows = 2 KB per step); B operands MN-major: [128 queries x 64]
+              tc_mma_bf16(acc0, make_sdesc_sw128(smem_u32(sP) + kk * 2048, 16384, 1024),
+                          make_sdesc_sw128(bq + kk * 2048, 8192, 1024), idesc_acc, accum);
+              tc_mma_bf16(acc1, make_sdesc_sw128(dsA + kk * 2048, 16384, 1024),
+                          make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc, accum);
+            } else {
+              // dQ += dZ K_j   (A K-major: 16 keys = 32 bytes per step within a 64-key half)
+              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
+              tc_mma_bf16(acc0, make_sdesc_sw128(dsA + koff, 16, 1024), make_sdesc_sw128(a + kk * 2048, 8192, 1024),
+                          idesc_acc, accum);
+            }
+          }
+          tc_commit(&t_empty[st]);
+          tc_commit(ps_empty);
         }
-        tc_commit(&t_empty[s]);
-        tc_commit(ps_empty);
+        if (!ok) break;
+        tc_commit(&acc_full[ab]);
+        tc_commit(&r_empty[k & 1]);
+        idx = nidx;
       }
-      if (ok) tc_commit(acc_full);
     }
   } else {
     // ------------------------------------------------------------------ elementwise
@@ -659,102 +704,101 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
     const int r = q * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float LOG2E = 1.4426950408889634f;
-    float row_lse2 = 0.f, row_D = 0.f;
-    if (MODE == 1) {
-      const int qi = tile * 128 + r;
-      row_lse2 = (qi < T) ? lse[(long long)bh * T + qi] * LOG2E : 0.f;
-      row_D = (qi < T) ? Dbuf[(long long)bh * T + qi] : 0.f;
-    }
+    const int c0 = part * 32;
+    const float2 sc = make_float2(scale_log2, scale_log2);
     bool ok = true;
-    const float* lse_bh = lse + (long long)bh * T;
-    const float* D_bh = Dbuf + (long long)bh * T;
-    for (int n = 0; n < n_it && ok; ++n) {
-      const int t = it0 + n;
-      if (!mbar_wait(sd_full, n & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      // this thread's 32 columns of S and dP, then the TMEM buffer is released at once
-      const int c0 = part * 32;
-      uint32_t us[32], ud[32];
-      tmem_ld32(tmem + lane_off + S_C + c0, us);
-      tmem_ld32(tmem + lane_off + DP_C + c0, ud);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(sd_empty);
-      const int s = n % BWD_STAGES;
-      const bool scal_bulk = (MODE == 0) && (T % 4 == 0) && (t * 128 + 128 <= T);
-      if (scal_bulk && !mbar_wait(&t_full[s], (n / BWD_STAGES) & 1, abort_flag)) { ok = false; break; }
-      const float* lse_s = sScal + s * 256;
-      const float* D_s = lse_s + 128;
-      // the previous tile's MMAs must be done reading the P / dZ operands
-      if (!mbar_wait(ps_empty, (n & 1) ^ 1, abort_flag)) { ok = false; break; }
-      const bool diag = (t == tile);
-      // both kernels hold S with a query per row (thread r); MODE 0 streams the query tiles,
-      // so its row's lse and D change with t
-      bool row_out = false;   // a query row past T (MODE 0, last tile only)
-      if (MODE == 0) {
-        const int qi = t * 128 + r;
-        row_out = qi >= T;
-        if (scal_bulk) {
-          row_lse2 = lse_s[r] * LOG2E;
-          row_D = D_s[r];
-        } else {
+    int g = 0;
+    for (int k = 0; ok; ++k) {
+      const int idx = bwd_turn_item(k);
+      if (idx >= n_items) break;
+      const BwdItem w = bwd_item<MODE>(idx, BH, n_t);
+      const int row0 = (w.bh / H) * T, h = w.bh % H;
+      const float* lse_bh = lse + (long long)w.bh * T;
+      const float* D_bh = Dbuf + (long long)w.bh * T;
+      float row_lse2 = 0.f, row_D = 0.f;
+      if (MODE == 1) {
+        const int qi = w.tile * 128 + r;
+        row_lse2 = (qi < T) ? __ldg(lse_bh + qi) * LOG2E : 0.f;
+        row_D = (qi < T) ? __ldg(D_bh + qi) : 0.f;
+      }
+      for (int t = w.it0; t < w.it1; ++t, ++g) {
+        // MODE 0 streams the query tiles, so its row's lse and D change with t: load them
+        // before waiting for the scores
+        bool row_out = false;   // a query row past T (MODE 0, last tile only)
+        if (MODE == 0) {
+          const int qi = t * 128 + r;
+          row_out = qi >= T;
           row_lse2 = row_out ? 0.f : __ldg(lse_bh + qi) * LOG2E;
           row_D = row_out ? 0.f : __ldg(D_bh + qi);
         }
-      }
-      const bool need_mask = diag || row_out;
-      const float2 sc = make_float2(scale_log2, scale_log2);
-      const float2 nl = make_float2(-row_lse2, -row_lse2);
-      const float2 nd = make_float2(-row_D, -row_D);
-      float pv[32], dz[32];
-#pragma unroll
-      for (int d = 0; d < 32; d += 2) {
-        const int c = c0 + d;
-        const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
-        float2 pp = make_float2(ex2(x.x), ex2(x.y));
-        if (need_mask) {
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int cm = c + h2;
-            const bool masked = row_out || (diag && cm > r);   // causal: key cm after query r
-            if (masked) (h2 ? pp.y : pp.x) = 0.f;
-          }
-        }
-        const float2 g = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])), nd));
-        pv[d] = pp.x;
-        pv[d + 1] = pp.y;
-        dz[d] = g.x;
-        dz[d + 1] = g.y;
-      }
-      if (MODE == 0) store_32_sw128(sP, r, c0, pv);
-      store_32_sw128(sDS, r, c0, dz);
-      fence_async_smem();
-      mbar_arrive(ps_full);
-    }
-    // ---- epilogue: accumulators -> dqkv (bf16)
-    if (ok && mbar_wait(acc_full, 0, abort_flag)) {
-      tc_fence_after();
-      const int gi = tile * 128 + r;
-      bf16* row = dqkv + (long long)(row0 + gi) * (3 * C) + h * HD;
-      const int nacc = (MODE == 0) ? 2 : 1;
-      for (int a = 0; a < nacc; ++a) {
-        // MODE 0: a=0 dV (column block 2C), a=1 dK (column block C, times scale); MODE 1: dQ (times scale).
-        // Each of the 4 warps of a lane quarter writes 16 of the 64 head columns.
-        const uint32_t col = ((a == 0) ? A0_C : A1_C) + part * 16;
-        const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
-        bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C)) + part * 16;
-        uint32_t u[16];
-        tmem_ld16(tmem + lane_off + col, u);
+        if (!mbar_wait(sd_full, g & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        // this thread's 32 columns of S and dP, then the TMEM buffer is released at once
+        uint32_t us[32], ud[32];
+        tmem_ld32(tmem + lane_off + S_C + c0, us);
+        tmem_ld32(tmem + lane_off + DP_C + c0, ud);
         tmem_wait_ld();
-        if (gi < T) {
+        tc_fence_before();
+        mbar_arrive(sd_empty);
+        const bool diag = (t == w.tile);
+        const bool need_mask = diag || row_out;
+        const float2 nl = make_float2(-row_lse2, -row_lse2);
+        const float2 nd = make_float2(-row_D, -row_D);
+        uint32_t pw[16], dw[16];
 #pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(u[g * 8 + 0]) * mul, __uint_as_float(u[g * 8 + 1]) * mul);
-            w.y = pack_bf16x2(__uint_as_float(u[g * 8 + 2]) * mul, __uint_as_float(u[g * 8 + 3]) * mul);
-            w.z = pack_bf16x2(__uint_as_float(u[g * 8 + 4]) * mul, __uint_as_float(u[g * 8 + 5]) * mul);
-            w.w = pack_bf16x2(__uint_as_float(u[g * 8 + 6]) * mul, __uint_as_float(u[g * 8 + 7]) * mul);
-            reinterpret_cast<uint4*>(dst)[g] = w;
+        for (int d = 0; d < 32; d += 2) {
+          const int c = c0 + d;
+          const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
+          float2 pp = make_float2(ex2(x.x), ex2(x.y));
+          if (need_mask) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int cm = c + h2;
+              const bool masked = row_out || (diag && cm > r);   // causal: key cm after query r
+              if (masked) (h2 ? pp.y : pp.x) = 0.f;
+            }
+          }
+          const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])), nd));
+          pw[d >> 1] = pack_bf16x2(pp.x, pp.y);
+          dw[d >> 1] = pack_bf16x2(gz.x, gz.y);
+        }
+        // the previous tile's MMAs must be done reading the P / dZ operands
+        if (!mbar_wait(ps_empty, (g & 1) ^ 1, abort_flag)) { ok = false; break; }
+        if (MODE == 0) store_32_sw128(sP, r, c0, pw);
+        store_32_sw128(sDS, r, c0, dw);
+        fence_async_smem();
+        mbar_arrive(ps_full);
+      }
+      if (!ok) break;
+      // ---- epilogue: accumulators -> dqkv (bf16); the buffer is released before the stores
+      const int ab = k & 1;
+      if (!mbar_wait(&acc_full[ab], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t u0[16], u1[16];
+      const uint32_t acc0 = tmem + lane_off + ACC_C + ab * 128 + part * 16;
+      tmem_ld16(acc0, u0);
+      if (MODE == 0) tmem_ld16(acc0 + 64, u1);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
+      const int gi = w.tile * 128 + r;
+      if (gi < T) {
+        bf16* row = dqkv + (long long)(row0 + gi) * (3 * C) + h * HD + part * 16;
+        // MODE 0: dV (column block 2C) and dK (column block C, times scale); MODE 1: dQ (times scale).
+        // Each of the 4 warps of a lane quarter writes 16 of the 64 head columns.
+#pragma unroll
+        for (int a = 0; a < ((MODE == 0) ? 2 : 1); ++a) {
+          const uint32_t* u = (a == 0) ? u0 : u1;
+          const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
+          bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C));
+#pragma unroll
+          for (int gq = 0; gq < 2; ++gq) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(u[gq * 8 + 0]) * mul, __uint_as_float(u[gq * 8 + 1]) * mul);
+            v.y = pack_bf16x2(__uint_as_float(u[gq * 8 + 2]) * mul, __uint_as_float(u[gq * 8 + 3]) * mul);
+            v.z = pack_bf16x2(__uint_as_float(u[gq * 8 + 4]) * mul, __uint_as_float(u[gq * 8 + 5]) * mul);
+            v.w = pack_bf16x2(__uint_as_float(u[gq * 8 + 6]) * mul, __uint_as_float(u[gq * 8 + 7]) * mul);
+            reinterpret_cast<uint4*>(dst)[gq] = v;
           }
         }
       }
@@ -804,7 +848,15 @@ int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const
       return -3;
     attr = true;
   }
-  const int grid = cdiv(T, 128) * B * H;
+  static int nsm = 0;
+  if (nsm == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (nsm <= 0) nsm = 148;
+  }
+  const int items = cdiv(T, 128) * B * H;
+  const int grid = items < nsm ? items : nsm;   // persistent: one CTA per SM
   const float scale = 1.0f / sqrtf((float)HD);
   const float scale_log2 = 1.4426950408889634f * scale;
   attn_bwd_tc_kernel<0><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv), B, T,
