@@ -470,7 +470,7 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
 namespace {
 
 constexpr int BWD_THREADS = 576;   // producer, MMA, 16 elementwise warps (4 per TMEM lane quarter)
-constexpr int BWD_STAGES = 2;
+constexpr int BWD_STAGES = 3;
 // smem: two buffers of the 2 resident tiles (K_j,V_j or Q_i,dO_i: this item's and the next
 // one's), BWD_STAGES x 2 streamed tiles, the 128x128 bf16 operands (P and dZ) and barriers
 constexpr int BWD_SMEM = 4 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + 512 + 1024;
@@ -706,13 +706,51 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
     const float LOG2E = 1.4426950408889634f;
     const int c0 = part * 32;
     const float2 sc = make_float2(scale_log2, scale_log2);
+    // Epilogue of the CTA's k-th item: accumulators -> dqkv (bf16).  The TMEM buffer is
+    // released before the global stores.
+    auto epilogue = [&](const BwdItem& w, int k) -> bool {
+      const int ab = k & 1;
+      if (!mbar_wait(&acc_full[ab], (k >> 1) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const int gi = w.tile * 128 + r;
+      const int row0 = (w.bh / H) * T, h = w.bh % H;
+      bf16* row = dqkv + (long long)(row0 + gi) * (3 * C) + h * HD + part * 16;
+      // MODE 0: dV (column block 2C) and dK (column block C, times scale); MODE 1: dQ (times scale).
+      // Each of the 4 warps of a lane quarter writes 16 of the 64 head columns; the TMEM
+      // buffer is released after the last read, before the last stores.
+#pragma unroll
+      for (int a = 0; a < ((MODE == 0) ? 2 : 1); ++a) {
+        uint32_t u[16];
+        tmem_ld16(tmem + lane_off + ACC_C + ab * 128 + a * 64 + part * 16, u);
+        tmem_wait_ld();
+        if (a + 1 == ((MODE == 0) ? 2 : 1)) {
+          tc_fence_before();
+          mbar_arrive(&acc_empty[ab]);
+        }
+        const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
+        if (gi < T) {
+          bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C));
+#pragma unroll
+          for (int gq = 0; gq < 2; ++gq) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(u[gq * 8 + 0]) * mul, __uint_as_float(u[gq * 8 + 1]) * mul);
+            v.y = pack_bf16x2(__uint_as_float(u[gq * 8 + 2]) * mul, __uint_as_float(u[gq * 8 + 3]) * mul);
+            v.z = pack_bf16x2(__uint_as_float(u[gq * 8 + 4]) * mul, __uint_as_float(u[gq * 8 + 5]) * mul);
+            v.w = pack_bf16x2(__uint_as_float(u[gq * 8 + 6]) * mul, __uint_as_float(u[gq * 8 + 7]) * mul);
+            reinterpret_cast<uint4*>(dst)[gq] = v;
+          }
+        }
+      }
+      return true;
+    };
     bool ok = true;
     int g = 0;
-    for (int k = 0; ok; ++k) {
+    BwdItem prev{};
+    int k = 0;
+    for (;; ++k) {
       const int idx = bwd_turn_item(k);
       if (idx >= n_items) break;
       const BwdItem w = bwd_item<MODE>(idx, BH, n_t);
-      const int row0 = (w.bh / H) * T, h = w.bh % H;
       const float* lse_bh = lse + (long long)w.bh * T;
       const float* D_bh = Dbuf + (long long)w.bh * T;
       float row_lse2 = 0.f, row_D = 0.f;
@@ -768,41 +806,14 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         store_32_sw128(sDS, r, c0, dw);
         fence_async_smem();
         mbar_arrive(ps_full);
+        // the previous item's epilogue runs once this item's first tile is handed over, so
+        // its wait for the last accumulation overlaps this item's products
+        if (t == w.it0 && k > 0 && !epilogue(prev, k - 1)) { ok = false; break; }
       }
       if (!ok) break;
-      // ---- epilogue: accumulators -> dqkv (bf16); the buffer is released before the stores
-      const int ab = k & 1;
-      if (!mbar_wait(&acc_full[ab], (k >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t u0[16], u1[16];
-      const uint32_t acc0 = tmem + lane_off + ACC_C + ab * 128 + part * 16;
-      tmem_ld16(acc0, u0);
-      if (MODE == 0) tmem_ld16(acc0 + 64, u1);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&acc_empty[ab]);
-      const int gi = w.tile * 128 + r;
-      if (gi < T) {
-        bf16* row = dqkv + (long long)(row0 + gi) * (3 * C) + h * HD + part * 16;
-        // MODE 0: dV (column block 2C) and dK (column block C, times scale); MODE 1: dQ (times scale).
-        // Each of the 4 warps of a lane quarter writes 16 of the 64 head columns.
-#pragma unroll
-        for (int a = 0; a < ((MODE == 0) ? 2 : 1); ++a) {
-          const uint32_t* u = (a == 0) ? u0 : u1;
-          const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
-          bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C));
-#pragma unroll
-          for (int gq = 0; gq < 2; ++gq) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(u[gq * 8 + 0]) * mul, __uint_as_float(u[gq * 8 + 1]) * mul);
-            v.y = pack_bf16x2(__uint_as_float(u[gq * 8 + 2]) * mul, __uint_as_float(u[gq * 8 + 3]) * mul);
-            v.z = pack_bf16x2(__uint_as_float(u[gq * 8 + 4]) * mul, __uint_as_float(u[gq * 8 + 5]) * mul);
-            v.w = pack_bf16x2(__uint_as_float(u[gq * 8 + 6]) * mul, __uint_as_float(u[gq * 8 + 7]) * mul);
-            reinterpret_cast<uint4*>(dst)[gq] = v;
-          }
-        }
-      }
+      prev = w;
     }
+    if (ok && k > 0) epilogue(prev, k - 1);
   }
 
   tc_fence_before();
