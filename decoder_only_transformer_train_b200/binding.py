@@ -57,6 +57,8 @@ _PROTOS = {
     "gpt2_synchronize": (_i, [_vp]),
     "gpt2_last_error": (ctypes.c_char_p, [_vp]),
     "gpt2op_gemm_bf16": (_i, [_vp, _i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _f, _vp, _i64]),
+    "gpt2op_gemm_bf16_fused": (_i, [_vp, _i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, ctypes.c_float,
+                                    _vp, _i64, _vp, _i64]),
     "gpt2op_attention_fwd": (_i, [_vp, _i, _vp, _vp, _vp, _i, _i, _i, _i]),
     "gpt2op_attention_bwd": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
     "gpt2op_attention_bwd_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
@@ -257,6 +259,14 @@ def gemm_bf16(A, B, C, M, N, K, lda, ldb, ldc, a_mn=False, b_mn=False, epilogue=
     ws = workspace.numel() if workspace is not None else 0
     _check(lib().gpt2op_gemm_bf16(_stream(stream), M, N, K, _ptr(A), lda, int(a_mn), _ptr(B), ldb, int(b_mn),
                                   _ptr(C), ldc, epilogue, _ptr(bias), alpha, _ptr(workspace), ws))
+
+
+def gemm_bf16_fused(A, B, C, M, N, K, lda, ldb, ldc, a_mn, b_mn, epilogue, bias=None, alpha=1.0, aux=None,
+                    ld_aux=0, aux_out=None, ld_aux_out=0, stream=None):
+    """Epilogue 3 (residual), 4 (GELU, keeps the pre-activation in aux_out), 5 (GELU grad)."""
+    _check(lib().gpt2op_gemm_bf16_fused(_stream(stream), M, N, K, _ptr(A), lda, int(a_mn), _ptr(B), ldb, int(b_mn),
+                                        _ptr(C), ldc, epilogue, _ptr(bias), alpha, _ptr(aux), ld_aux, _ptr(aux_out),
+                                        ld_aux_out))
 
 
 def attention_fwd(qkv, out, lse, B, T, H, head_dim, precision, stream=None):

@@ -17,6 +17,38 @@ namespace {
 
 constexpr int AT = 64;   // rows per tile
 
+// Same for bf16 with head size 64: a warp per token row (all heads), 16-byte loads; lane l
+// takes the 8-channel groups l, l + 32, ... and the 8 lanes of a head add by shuffles.
+__global__ void __launch_bounds__(256) attn_bwd_D_bf16_hd64(const bf16* __restrict__ out, const bf16* __restrict__ dout,
+                                                            float* __restrict__ Dbuf, int Tn, int H, long long ntok) {
+  const long long tok = blockIdx.x * 8LL + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (tok >= ntok) return;                     // warp-uniform
+  const int groups = H * 8;                    // 8-channel groups per row
+  const uint4* o = reinterpret_cast<const uint4*>(out) + tok * groups;
+  const uint4* g = reinterpret_cast<const uint4*>(dout) + tok * groups;
+  const long long b = tok / Tn;
+  const int t = (int)(tok - b * Tn);
+  for (int base = 0; base < groups; base += 32) {
+    const int c8 = base + lane;
+    float s = 0.f;
+    if (c8 < groups) {
+      const uint4 a = __ldcs(o + c8), d = __ldcs(g + c8);
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, dw[4] = {d.x, d.y, d.z, d.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 af = unpack_bf16x2(aw[i]), df = unpack_bf16x2(dw[i]);
+        s = fmaf(af.x, df.x, s);
+        s = fmaf(af.y, df.y, s);
+      }
+    }
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    if (c8 < groups && (lane & 7) == 0) Dbuf[(b * H + (c8 >> 3)) * Tn + t] = s;
+  }
+}
+
 template <typename T, int HD>
 __global__ void __launch_bounds__(AT) attn_fwd_simt(const T* __restrict__ qkv, T* __restrict__ out,
                                                     float* __restrict__ lse, int Tn, int H, float scale) {
@@ -276,9 +308,16 @@ int launch_attn_fwd(cudaStream_t st, bool is_bf16, const void* qkv, void* out, f
 int launch_attn_bwd(cudaStream_t st, bool is_bf16, const void* qkv, const void* out, const void* dout,
                     const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd) {
   if (is_bf16 && hd == 64) {
-    dim3 gD(cdiv(T * H, 8), B);
-    attn_bwd_D<bf16><<<gD, 256, 0, st>>>(reinterpret_cast<const bf16*>(out), reinterpret_cast<const bf16*>(dout),
-                                         Dbuf, T, H, hd);
+    const long long ntok = (long long)B * T;
+    if ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(dout)) % 16 == 0) {
+      attn_bwd_D_bf16_hd64<<<(unsigned)cdivll(ntok, 8), 256, 0, st>>>(reinterpret_cast<const bf16*>(out),
+                                                                       reinterpret_cast<const bf16*>(dout), Dbuf, T, H,
+                                                                       ntok);
+    } else {
+      dim3 gD(cdiv(T * H, 8), B);
+      attn_bwd_D<bf16><<<gD, 256, 0, st>>>(reinterpret_cast<const bf16*>(out), reinterpret_cast<const bf16*>(dout),
+                                           Dbuf, T, H, hd);
+    }
     note_kernel_launches(1);
     if (cudaGetLastError() != cudaSuccess) return -3;
     return launch_attn_bwd_tc(st, qkv, dout, lse, Dbuf, dqkv, B, T, H, hd);

@@ -36,6 +36,34 @@ int gpt2op_gemm_bf16(void* stream, int M, int N, int K, const void* A, int64_t l
   return rc == 0 ? GPT2_OK : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA);
 }
 
+int gpt2op_gemm_bf16_fused(void* stream, int M, int N, int K, const void* A, int64_t lda, int a_mn_major,
+                           const void* B, int64_t ldb, int b_mn_major, void* C, int64_t ldc, int epilogue,
+                           const float* bias, float alpha, const void* aux, int64_t ld_aux, void* aux_out,
+                           int64_t ld_aux_out) {
+  if (A == nullptr || B == nullptr || C == nullptr) return GPT2_ERR_ARG;
+  if (M < 0 || N < 0 || K <= 0) return GPT2_ERR_SHAPE;
+  int kind;
+  switch (epilogue) {
+    case 3: kind = EPI_RESID_F32; break;
+    case 4: kind = EPI_GELU_FWD; break;
+    case 5: kind = EPI_GELU_BWD; break;
+    default: return GPT2_ERR_ARG;
+  }
+  if ((kind == EPI_RESID_F32 || kind == EPI_GELU_BWD) && aux == nullptr) return GPT2_ERR_ARG;
+  if (kind == EPI_GELU_FWD && aux_out == nullptr) return GPT2_ERR_ARG;
+  if ((aux && ld_aux % 8) || (aux_out && ld_aux_out % 8)) return GPT2_ERR_ARG;
+  EpiParams e = epi_make(kind, C, ldc);
+  e.bias = (kind == EPI_GELU_BWD) ? nullptr : bias;
+  e.alpha = alpha;
+  e.aux = aux;
+  e.ld_aux = ld_aux;
+  e.aux_out = aux_out;
+  e.ld_aux_out = ld_aux_out;
+  int rc = gemm_bf16_tc(reinterpret_cast<cudaStream_t>(stream), M, N, K, A, lda, a_mn_major != 0, B, ldb,
+                        b_mn_major != 0, e, nullptr, 0, sm_count());
+  return rc == 0 ? GPT2_OK : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA);
+}
+
 int gpt2op_attention_fwd(void* stream, int precision, const void* qkv, void* out, float* lse, int B, int T, int H,
                          int head_dim) {
   if (!qkv || !out || !lse) return GPT2_ERR_ARG;

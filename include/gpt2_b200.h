@@ -160,6 +160,25 @@ int gpt2op_gemm_bf16(void* stream, int M, int N, int K, const void* A, int64_t l
                      int64_t ldb, int b_mn_major, void* C, int64_t ldc, int epilogue, const float* bias, float alpha,
                      float* workspace, int64_t ws_floats);
 
+/* The fused epilogues of the Transformer block on the same GEMM (D, layouts and alignment as
+ * for gpt2op_gemm_bf16).  "Karpathy's Zero to Hero, Lecture 9" notes, "Code you'll write"
+ * (the pre-norm Block adds each sublayer's output to the residual stream; the MLP applies
+ * the tanh GELU) and "1:48:25 – 2:00:19 torch.compile and the GPU memory hierarchy" (the
+ * elementwise work fused with the kernel that produces its input):
+ *   epilogue 3 (residual):  C(f32)[m*ldc + n] = aux(f32)[m*ld_aux + n] + alpha D + bias[n]
+ *   epilogue 4 (GELU):      u = alpha D + bias[n];  aux_out(bf16)[m*ld_aux_out + n] = u;
+ *                           C(bf16)[m*ldc + n] = gelu_tanh(u)
+ *   epilogue 5 (GELU grad): C(bf16)[m*ldc + n] = alpha D * gelu_tanh'(aux(bf16)[m*ld_aux + n])
+ * bias (f32 [N]) may be NULL for 3 and 4 and is ignored by 5.  aux / aux_out are device
+ * buffers the caller owns, 16-byte aligned, with ld_aux / ld_aux_out multiples of 8
+ * elements; aux may equal C for epilogue 3 (an in-place residual update).  GELU uses the
+ * hardware tanh approximation (results rounded to bf16).  GPT2_ERR_ARG for a null operand or
+ * an unknown epilogue; GPT2_ERR_CUDA if a launch or tensor-map encode fails. */
+int gpt2op_gemm_bf16_fused(void* stream, int M, int N, int K, const void* A, int64_t lda, int a_mn_major,
+                           const void* B, int64_t ldb, int b_mn_major, void* C, int64_t ldc, int epilogue,
+                           const float* bias, float alpha, const void* aux, int64_t ld_aux, void* aux_out,
+                           int64_t ld_aux_out);
+
 /* Causal attention forward over qkv [B*T, 3C] (q | k | v, head h at columns h*hd..):
  * out [B*T, C], lse [B, H, T] float.  precision selects fp32 or bf16 qkv/out. */
 int gpt2op_attention_fwd(void* stream, int precision, const void* qkv, void* out, float* lse, int B, int T, int H,
