@@ -54,6 +54,28 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def recorded_traffic(cls: str):
+    """DRAM bytes per call of a profiler class, from the ncu launch-list summaries under
+    profiles/: (bytes, note).  A figure counts only while the kernel sources it lists still
+    hash to the recorded SHA-256; a changed kernel gives (None, reason)."""
+    import glob
+    import hashlib
+    import re
+    pat = re.compile(r"<!-- traffic (\w+) bytes_per_call=(\d+) sources=([\w./,]+) sha256=([0-9a-f]{64}) -->")
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        for m in pat.finditer(open(path).read()):
+            if m.group(1) != cls:
+                continue
+            h = hashlib.sha256()
+            for f in m.group(3).split(","):
+                h.update(open(os.path.join(ROOT, "decoder_only_transformer_train_b200", f), "rb").read())
+            name = os.path.basename(path)
+            if h.hexdigest() != m.group(4):
+                return None, f"{name}: kernel sources changed since the capture"
+            return int(m.group(2)), f"{name}: dram__bytes_read.sum + dram__bytes_write.sum per call"
+    return None, "no capture recorded"
+
+
 # ------------------------------------------------------------------ clocks sampling
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -315,6 +337,7 @@ def run_ours(args, world, rank, local):
             roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                     "traffic": None, "kernel": dom, "launches": d["launches"],
                     "avg_launch_ms": d["ms"] / max(1, d["launches"]), "peak_kind": f"{pk['source']} HBM copy"}
+        roof["traffic"], roof["traffic_note"] = recorded_traffic(dom)
         step_ms = sum(p["ms"] for p in prof.values())
         kernels = {}
         for c, p in prof.items():
