@@ -117,7 +117,14 @@ class ClockSampler:
         smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        pw = [v for v in (num(r[3]) for r in rows) if v is not None]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_median": statistics.median(pw) if pw else None, "power_w_max": max(pw) if pw else None,
                 "reasons": reasons, "samples": len(rows)}
 
 

@@ -18,6 +18,7 @@
 // Zero to Hero, Lecture 9: Reproduce GPT-2 (124M)" notes, "Code you'll write") and of the
 // tied lm_head; the epilogues fuse the bias, the residual add, the tanh-GELU and its
 // derivative, and the softmax partials of the cross-entropy.
+#include <stdlib.h>
 #include "sm100.cuh"
 #include "gemm.h"
 #include "kernels.h"
@@ -31,16 +32,24 @@ constexpr int EPI_THREADS = 256;
 
 constexpr int BOX_BYTES = 2048;     // one epilogue staging box: 32 rows x 64 bytes
 
-template <int BN>
+// CG = 1: one CTA computes a 128 x BN tile.  CG = 2: a CTA pair (cluster of 2, tcgen05
+// cta_group::2) computes a 256 x BN tile; each CTA stages its own 128 rows of A and
+// BN / 2 rows of B, so a stage is smaller and the pipeline deeper.
+template <int BN, int CG = 1>
 struct TileCfg {
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 192 ? 4 : 6);
+  static constexpr int B_ROWS = BN / CG;                      // rows of B staged by one CTA
   static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = CG == 1 ? (BN == 256 ? 4 : (BN == 192 ? 4 : 6))
+                                        : (BN == 256 ? 6 : (BN == 192 ? 6 : 8));
   static constexpr int STG_BYTES = 8 * 2 * BOX_BYTES;   // 8 epilogue warps x 2 boxes
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES + 1024;   // +1024: manual alignment
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;   // power of two >= 2*BN
+  static_assert((2 * STAGES + 4 + 8) * 8 + 8 <= BAR_BYTES, "GEMM barriers");
+  static_assert(SMEM <= 232448, "GEMM shared memory");
+  static_assert(CG == 1 || (BN / 2) % 16 == 0, "CTA-pair tile width");
 };
 
 // Tile order: with few column tiles (n_fast) the column tiles of one row block are
@@ -196,12 +205,15 @@ struct EpiWarp {
   }
 };
 
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmIn,
                const __grid_constant__ CUtensorMap tmOut2, TileSched sched, EpiParams ep) {
-  using Cfg = TileCfg<BN>;
+  using Cfg = TileCfg<BN, CG>;
+  constexpr int BMT = BM * CG;                       // rows of an output tile
+  const uint32_t rank = (CG == 2) ? cluster_ctarank() : 0u;   // 0: the pair's leader (issues the MMAs)
+  const int cl_id = blockIdx.x / CG, n_cl = gridDim.x / CG;   // tiles are dealt per CTA group
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stg = smem + Cfg::STAGES * Cfg::STAGE_BYTES;                       // epilogue boxes
@@ -223,7 +235,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], EPI_THREADS);
+      mbar_init(&tempty_bar[a], 8 * CG);   // one arrival per epilogue warp of every CTA of the group
     }
     for (int w = 0; w < 8; ++w) mbar_init(&epi_bar[w], 1);
     *abort_flag = 0;
@@ -235,11 +247,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tma_prefetch_desc(&tmOut2);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
-    tmem_relinquish();
+    if (CG == 2) {
+      tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync();   // the peer's barriers are initialised before any cross-CTA signal
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int ntiles = sched.num_tiles();
@@ -250,45 +268,53 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      // this CTA's rows of A and of B within a tile; with a CTA pair both halves complete
+      // on the leader's full barrier, which the leader arms for the bytes of both
+      auto load = [&](void* dst, const CUtensorMap* map, int x, int y, int st) {
+        if (CG == 2) tma_load_2d_pair(dst, map, x, y, cluster_addr(&full_bar[st], 0));
+        else tma_load_2d(dst, map, x, y, &full_bar[st]);
+      };
+      for (int t = cl_id; t < ntiles && ok; t += n_cl) {
         int tm, tn, split, kb0, kb1;
         sched.decode(t, tm, tn, split, kb0, kb1);
-        const int m0 = tm * BM, n0 = tn * BN;
+        const int m0 = tm * BMT + (int)rank * BM, n0 = tn * BN + (int)rank * Cfg::B_ROWS;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           uint8_t* sA = smem + stage * Cfg::STAGE_BYTES;
           uint8_t* sB = sA + Cfg::A_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], Cfg::STAGE_BYTES);
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], CG * Cfg::STAGE_BYTES);
           const int k0 = kb * BK;
           if (!A_MN) {
-            tma_load_2d(sA, &tmA, k0, m0, &full_bar[stage]);
+            load(sA, &tmA, k0, m0, stage);
           } else {
 #pragma unroll
-            for (int j = 0; j < BM / 64; ++j) tma_load_2d(sA + j * 8192, &tmA, m0 + 64 * j, k0, &full_bar[stage]);
+            for (int j = 0; j < BM / 64; ++j) load(sA + j * 8192, &tmA, m0 + 64 * j, k0, stage);
           }
           if (!B_MN) {
-            tma_load_2d(sB, &tmB, k0, n0, &full_bar[stage]);
+            load(sB, &tmB, k0, n0, stage);
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sB + j * 8192, &tmB, n0 + 64 * j, k0, &full_bar[stage]);
+            for (int j = 0; j < Cfg::B_ROWS / 64; ++j) load(sB + j * 8192, &tmB, n0 + 64 * j, k0, stage);
           }
           if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1; }
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = make_idesc_bf16(BM, BN, A_MN, B_MN);
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------------ MMA issuer (the leader)
+      constexpr uint32_t idesc = make_idesc_bf16(BMT, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      for (int t = cl_id; t < ntiles && ok; t += n_cl) {
         int tm, tn, split, kb0, kb1;
         sched.decode(t, tm, tn, split, kb0, kb1);
-        if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag)) break;
+        if (CG == 2 ? !mbar_wait_cluster(&tempty_bar[acc], acc_phase ^ 1, abort_flag)
+                    : !mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag))
+          break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -302,13 +328,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                                      : make_sdesc_sw128(aBase + k * 32, 16, 1024);
             const uint64_t bd = B_MN ? make_sdesc_sw128(bBase + k * 2048, 8192, 1024)
                                      : make_sdesc_sw128(bBase + k * 32, 16, 1024);
-            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            if (CG == 2) tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            else tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           }
-          tc_commit(&empty_bar[stage]);
+          if (CG == 2) tc_commit_pair(&empty_bar[stage], 0x3);   // both CTAs' stage is free
+          else tc_commit(&empty_bar[stage]);
           if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        tc_commit(&tfull_bar[acc]);
+        if (CG == 2) tc_commit_pair(&tfull_bar[acc], 0x3);       // both halves of D are ready
+        else tc_commit(&tfull_bar[acc]);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
@@ -334,13 +363,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+    // the leader's TMEM-empty barrier: every epilogue warp of the CTA group arrives once per tile
+    const uint32_t tempty_leader0 = (CG == 2) ? cluster_addr(&tempty_bar[0], 0) : 0u;
+    for (int t = cl_id; t < ntiles && ok; t += n_cl) {
       int tm, tn, split, kb0, kb1;
       sched.decode(t, tm, tn, split, kb0, kb1);
       if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
-      const int m = tm * BM + row;
-      const int m_warp = tm * BM + q * 32;                      // first row of this warp's slab
+      const int row0 = tm * BMT + (int)rank * BM;               // this CTA's rows of the tile
+      const int m = row0 + row;
+      const int m_warp = row0 + q * 32;                         // first row of this warp's slab
       const int y_out = (kind == EPI_SPLITK) ? split * ep.ld_aux + m_warp : m_warp;   // ws rows per split: ld_aux
       const int n_base = tn * BN;
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0.0f, 0x7fffffff};
@@ -435,7 +467,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (y_row >= n_lo && y_row < min(n_lo + BN / 2, ep.N)) ep.zt[m] = ce.zt;
       }
       tc_fence_before();
-      mbar_arrive(&tempty_bar[acc]);
+      __syncwarp();
+      if (lane == 0) {
+        if (CG == 2) mbar_arrive_cluster(tempty_leader0 + acc * 8);
+        else mbar_arrive(&tempty_bar[acc]);
+      }
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
@@ -444,11 +480,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync();   // neither CTA leaves while its peer may still signal it
+  else __syncthreads();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    if (CG == 2) tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
+    else tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
   }
 }
 
@@ -534,20 +572,54 @@ int encode_epi_box(CUtensorMap* map, bool bf16_elems, const void* base, uint64_t
                                 CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int BN, bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN, int CG>
 int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
               const CUtensorMap& tin, const CUtensorMap& tout2, TileSched sched, const EpiParams& ep, int num_sms) {
-  using Cfg = TileCfg<BN>;
-  auto kern = gemm_tc_kernel<BN, A_MN, B_MN>;
+  using Cfg = TileCfg<BN, CG>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, CG>;
   static bool attr_set = false;
+  static int max_groups = 0;   // co-resident CTA groups of this kernel
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
       return -3;
+    max_groups = num_sms / CG;
+    if (CG == 2) {
+      cudaLaunchConfig_t cfg{};
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * max_groups);
+      cfg.blockDim = dim3(NUM_THREADS);
+      cfg.dynamicSmemBytes = Cfg::SMEM;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return -3;
+      if (n < max_groups) max_groups = n;
+    }
     attr_set = true;
   }
   const int tiles = sched.m_tiles * sched.n_tiles * sched.splits;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  kern<<<grid, NUM_THREADS, Cfg::SMEM, st>>>(ta, tb, tout, tin, tout2, sched, ep);
+  const int groups = tiles < max_groups ? tiles : max_groups;
+  if (CG == 1) {
+    kern<<<groups, NUM_THREADS, Cfg::SMEM, st>>>(ta, tb, tout, tin, tout2, sched, ep);
+  } else {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * groups);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM;
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tout, tin, tout2, sched, ep) != cudaSuccess) return -3;
+  }
   note_kernel_launches(1);
   return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }
@@ -558,42 +630,57 @@ int gemm_tc_tile_n(int N) { return N > 128 ? 256 : 128; }
 int gemm_tc_ce_tiles(int N) { return cdiv(N, gemm_tc_tile_n(N)) * 2; }
 
 namespace {
-// Picks the output tile width (128, 192 or 256 columns) and the number of K splits from a
-// small cost model in MMA clock cycles: the busiest SM's tiles x the tile's main loop
-// (narrower tiles re-read more operand bytes per FLOP, hence the efficiency factor), plus
-// for split-K the extra fp32 traffic of the partials and their reduction.
+// Picks the output tile width (128, 192 or 256 columns), the CTA group (one CTA per
+// 128-row tile, or a CTA pair per 256-row tile) and the number of K splits from a small
+// cost model in MMA clock cycles: the busiest SM's tiles x the tile's main loop (narrower
+// tiles re-read more operand bytes per FLOP, hence the efficiency factor; a pair stages half
+// the operand bytes per SM and keeps a deeper pipeline), plus for split-K the extra fp32
+// traffic of the partials and their reduction.  Pairs are left out where measurement found
+// them slower: with split-K, and for the epilogues that read inputs or evaluate GELU on short
+// K (the epilogue, not the main loop, bounds those).  GPT2_B200_GEMM_PAIRS=0 / 1 in the
+// environment forces single CTAs / pairs (where the shape allows them).
 struct TileChoice {
-  int bn, splits;
+  int bn, splits, cg;
 };
-TileChoice choose_tiles(int M, int N, int K, bool can_split, size_t ws_elems, int num_sms, bool fixed_bn) {
-  const int m_tiles = cdiv(M, BM);
+TileChoice choose_tiles(int M, int N, int K, bool can_split, size_t ws_elems, int num_sms, bool fixed_bn,
+                        bool b_mn, bool heavy_epilogue) {
   const int nk = cdiv(K, BK);
   const int bns[3] = {256, 192, 128};
   const double eff[3] = {1.0, 0.96, 0.88};
-  TileChoice best{gemm_tc_tile_n(N), 1};
+  const char* env = getenv("GPT2_B200_GEMM_PAIRS");
+  const int pairs = (env && env[0] == '0') ? 0 : ((env && env[0] == '1') ? 1 : -1);
+  TileChoice best{gemm_tc_tile_n(N), 1, 1};
   double best_cost = 1e300;
-  for (int i = 0; i < 3; ++i) {
-    const int bn = bns[i];
-    if (fixed_bn && bn != gemm_tc_tile_n(N)) continue;
-    if (bn > 128 && N <= 128) continue;
-    const int tiles = m_tiles * cdiv(N, bn);
-    for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
-      if (sp > 1 && (nk / sp < 8 || N % 4 != 0 || (size_t)sp * cdiv(M, BM) * BM * N > ws_elems)) break;
-      const int kb = cdiv(nk, sp);
-      const double per_tile = (double)bn * kb * 2.0 / eff[i] + 1500.0;   // MMA clks of a 128 x bn x 64kb tile + overhead
-      const double waves = (double)cdiv(tiles * sp, num_sms);
-      double cost = waves * per_tile;
-      if (sp > 1) cost += (double)(sp + 2) * M * N * 4.0 / 6.0e12 * 1.9e9 + 3000.0;   // partial traffic + reduce launch
-      if (cost < best_cost * 0.999) {
-        best_cost = cost;
-        best = TileChoice{bn, sp};
+  for (int cg = 1; cg <= 2; ++cg) {
+    if (cg == 2 && (pairs == 0 || M <= BM)) continue;
+    if (cg == 2 && pairs != 1 && heavy_epilogue && K < 1536) continue;
+    if (cg == 1 && pairs == 1 && M > BM) continue;
+    for (int i = 0; i < 3; ++i) {
+      const int bn = bns[i];
+      if (fixed_bn && bn != gemm_tc_tile_n(N)) continue;
+      if (bn > 128 && N <= 128) continue;
+      if (cg == 2 && b_mn && bn == 192) continue;   // MN-major B is staged in 64-column boxes
+      const int tiles = cdiv(M, BM * cg) * cdiv(N, bn);
+      if (cg == 2 && pairs != 1 && tiles < num_sms / 2) continue;   // pairs only with a full wave of tiles
+      for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
+        if (sp > 1 && (nk / sp < 8 || N % 4 != 0 || (size_t)sp * cdiv(M, BM * cg) * BM * cg * N > ws_elems)) break;
+        if (sp > 1 && cg == 2 && pairs != 1) break;
+        const int kb = cdiv(nk, sp);
+        // MMA clocks per SM of a (128 cg) x bn x 64kb tile + overhead
+        const double per_tile = ((double)bn * kb * 2.0 / eff[i] + 1500.0) / (cg == 2 ? 1.2 : 1.0);
+        const double waves = (double)cdiv(tiles * sp, num_sms / cg);
+        double cost = waves * per_tile;
+        if (sp > 1) cost += (double)(sp + 2) * M * N * 4.0 / 6.0e12 * 1.9e9 + 3000.0;   // partial traffic + reduce launch
+        if (cost < best_cost * 0.999) {
+          best_cost = cost;
+          best = TileChoice{bn, sp, cg};
+        }
       }
     }
   }
   return best;
 }
 }  // namespace
-
 int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long lda, bool a_mn, const void* B,
                  long long ldb, bool b_mn, EpiParams ep, float* ws, size_t ws_elems, int num_sms) {
   if (M <= 0 || N <= 0) return 0;
@@ -606,19 +693,22 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   const bool can_split = (ep.kind == EPI_ACCUM_F32 && ws != nullptr && (reinterpret_cast<uintptr_t>(ep.C) % 16) == 0 &&
                          (reinterpret_cast<uintptr_t>(ws) % 16) == 0);
   // the softmax partials of EPI_CE_FWD are laid out per 256/128-column tile
-  const TileChoice tc = choose_tiles(M, N, K, can_split, ws_elems, num_sms, ep.kind == EPI_CE_FWD);
+  const bool heavy = (ep.kind == EPI_RESID_F32 || ep.kind == EPI_GELU_FWD || ep.kind == EPI_GELU_BWD ||
+                     ep.kind == EPI_CE_FWD);
+  const TileChoice tc = choose_tiles(M, N, K, can_split, ws_elems, num_sms, ep.kind == EPI_CE_FWD, b_mn, heavy);
   const int BN = tc.bn;
+  const int CG = tc.cg;
   CUtensorMap ta, tb;
   int rc;
   if (!a_mn) rc = encode_bf16_2d(&ta, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda, BK, BM);
   else rc = encode_bf16_2d(&ta, A, (uint64_t)M, (uint64_t)K, (uint64_t)lda, 64, BK);
   if (rc) return rc;
-  if (!b_mn) rc = encode_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb, BK, (uint32_t)BN);
+  if (!b_mn) rc = encode_bf16_2d(&tb, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb, BK, (uint32_t)(BN / CG));
   else rc = encode_bf16_2d(&tb, B, (uint64_t)N, (uint64_t)K, (uint64_t)ldb, 64, BK);
   if (rc) return rc;
 
   TileSched sched;
-  sched.m_tiles = cdiv(M, BM);
+  sched.m_tiles = cdiv(M, BM * CG);
   sched.n_tiles = cdiv(N, BN);
   sched.nk = cdiv(K, BK);
   sched.splits = 1;
@@ -640,7 +730,7 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   // epilogue tensor maps: output, input (residual / accumulator / GELU pre-activation),
   // second output (GELU pre-activation); unused ones repeat the output map
   CUtensorMap tout, tin, tout2;
-  const int Mpad = cdiv(M, BM) * BM;
+  const int Mpad = cdiv(M, BM * CG) * BM * CG;
   if (split) {
     run.ld_aux = Mpad;   // rows per split in the workspace
     rc = encode_epi_box(&tout, false, ws, (uint64_t)N, (uint64_t)sched.splits * Mpad, (uint64_t)N);
@@ -660,15 +750,23 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   if (ep.kind == EPI_GELU_FWD)
     rc = encode_epi_box(&tout2, true, ep.aux_out, (uint64_t)N, (uint64_t)M, (uint64_t)ep.ld_aux_out);
   if (rc) return rc;
-#define LAUNCH_BN(BNV)                                                                                     \
-  do {                                                                                                     \
-    if (!a_mn && !b_mn) rc = launch_tc<BNV, false, false>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);      \
-    else if (!a_mn && b_mn) rc = launch_tc<BNV, false, true>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);   \
-    else rc = launch_tc<BNV, true, true>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);                       \
+#define LAUNCH_BN(BNV, CGV)                                                                                   \
+  do {                                                                                                        \
+    if (!a_mn && !b_mn) rc = launch_tc<BNV, false, false, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);   \
+    else if (!a_mn && b_mn) rc = launch_tc<BNV, false, true, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms); \
+    else rc = launch_tc<BNV, true, true, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);                    \
   } while (0)
-  if (BN == 256) LAUNCH_BN(256);
-  else if (BN == 192) LAUNCH_BN(192);
-  else LAUNCH_BN(128);
+  if (CG == 1) {
+    if (BN == 256) LAUNCH_BN(256, 1);
+    else if (BN == 192) LAUNCH_BN(192, 1);
+    else LAUNCH_BN(128, 1);
+  } else {
+    if (BN == 256) LAUNCH_BN(256, 2);
+    else if (BN == 192) {
+      if (b_mn) return -1;   // excluded by the tile choice
+      rc = launch_tc<192, false, false, 2>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);
+    } else LAUNCH_BN(128, 2);
+  }
 #undef LAUNCH_BN
   if (rc) return rc;
   if (split) {

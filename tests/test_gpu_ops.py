@@ -26,6 +26,14 @@ def _randn(shape, seed, scale=1.0):
 
 
 # ------------------------------------------------------------------ GEMM
+@pytest.fixture(params=["0", "1"], ids=["cta", "cta_pair"])
+def gemm_pairs(request, monkeypatch):
+    """Every GEMM test runs twice: with one CTA per 128-row tile, and with CTA pairs
+    (tcgen05 cta_group::2, 256-row tiles) wherever the shape allows them."""
+    monkeypatch.setenv("GPT2_B200_GEMM_PAIRS", request.param)
+    return request.param
+
+
 GEMM_SHAPES = [(128, 256, 64), (300, 200, 136), (1000, 768, 768), (129, 1000, 320), (64, 64, 16)]
 LAYOUTS = [(False, False), (False, True), (True, True)]
 
@@ -45,7 +53,7 @@ def _layout(X, mn_major):
 
 @pytest.mark.parametrize("a_mn,b_mn", LAYOUTS)
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-def test_gemm_bf16_all_layouts_and_epilogues(a_mn, b_mn, M, N, K):
+def test_gemm_bf16_all_layouts_and_epilogues(a_mn, b_mn, M, N, K, gemm_pairs):
     A = bf16_round(_randn((M, K), M + 3 * K))
     Bm = bf16_round(_randn((N, K), N + 5 * K))
     bias = _randn((N,), 17).float()
@@ -80,7 +88,7 @@ FUSED_SHAPES = [(300, 200, 136), (1000, 768, 768), (129, 1000, 320), (512, 3072,
 
 @pytest.mark.parametrize("b_mn", [False, True])
 @pytest.mark.parametrize("M,N,K", FUSED_SHAPES)
-def test_gemm_bf16_fused_epilogues(b_mn, M, N, K):
+def test_gemm_bf16_fused_epilogues(b_mn, M, N, K, gemm_pairs):
     """Residual add, GELU (keeping the pre-activation) and GELU' epilogues against their
     definitions on the fp64 product of the same bf16 operands."""
     A = bf16_round(_randn((M, K), 91 + M))
@@ -121,7 +129,7 @@ def test_gemm_bf16_fused_epilogues(b_mn, M, N, K):
         assert torch.all(G[:, N:] == 0) and torch.all(U[:, N:] == 0) and torch.all(DG[:, N:] == 0)
 
 
-def test_gemm_split_k_weight_gradient_shape_is_deterministic():
+def test_gemm_split_k_weight_gradient_shape_is_deterministic(gemm_pairs):
     """dW += dY^T X with K = 16384 tokens (few output tiles, long K: split-K path)."""
     M, N, K = 768, 768, 16384
     dY = bf16_round(_randn((M, K), 31))      # logical A [M, K], stored MN-major like a [tokens, out] buffer
@@ -141,7 +149,7 @@ def test_gemm_split_k_weight_gradient_shape_is_deterministic():
 
 
 @pytest.mark.parametrize("M,N,K", [(3072, 768, 4096), (2304, 768, 4096), (768, 3072, 4096), (768, 768, 8192)])
-def test_gemm_weight_gradient_shapes_tile_choices(M, N, K):
+def test_gemm_weight_gradient_shapes_tile_choices(M, N, K, gemm_pairs):
     """dW += dY^T X on the weight-gradient shapes, where the launcher picks 128/192/256-wide
     tiles and split-K by its cost model."""
     dY = bf16_round(_randn((M, K), 71 + M))
@@ -216,7 +224,7 @@ def test_layernorm_forward(prec, N, C):
 
 # ------------------------------------------------------------------ classifier head
 @pytest.mark.parametrize("N,V,C", [(256, 1000, 64), (384, 50304, 768), (130, 50257, 768)])
-def test_classifier_head_forward_backward(N, V, C):
+def test_classifier_head_forward_backward(N, V, C, gemm_pairs):
     """lm_head + softmax + cross-entropy: loss, lse, argmax, dh and dW."""
     h = bf16_round(_randn((N, C), 61))
     W = bf16_round(_randn((V, C), 62, scale=0.02))
