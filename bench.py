@@ -27,7 +27,27 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "GPT-2 124M train tokens/sec (B=16,T=1024, 1 B200); ms/step; MFU vs BF16 peak"
-FLOP_PER_TOKEN = 6 * (12 * 12 * 768 * 768 + 50304 * 768) + 6 * 12 * 1024 * 768   # 798,031,872 (causal attention)
+# the headline model and the medium one (GPT-2 350M shape: 24 layers, 1024 channels, 16 heads)
+MODELS = {"124m": dict(n_layer=12, n_embd=768, n_head=12, label="GPT-2 124M", micro_batch=16, accum=32),
+          "medium": dict(n_layer=24, n_embd=1024, n_head=16, label="GPT-2 medium (L=24, C=1024, H=16)",
+                         micro_batch=8, accum=8)}
+
+
+def flop_per_token(model: str, T: int = 1024, Vp: int = 50304) -> int:
+    """Training FLOPs per token: 6 (12 L C^2 + Vp C) for the matrix products (pad columns
+    counted) plus 6 L T C for the causal attention products."""
+    m = MODELS[model]
+    L, C = m["n_layer"], m["n_embd"]
+    return 6 * (12 * L * C * C + Vp * C) + 6 * L * T * C
+
+
+FLOP_PER_TOKEN = flop_per_token("124m")   # 798,031,872
+
+
+def metric_name(model: str) -> str:
+    if model == "124m":
+        return METRIC
+    return f"{MODELS[model]['label']} train tokens/sec (1 B200); ms/step; MFU vs BF16 peak"
 NOMINAL_BF16_TFLOPS = 2250.0
 
 
@@ -37,12 +57,20 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--micro-batch", type=int, default=16)
+    ap.add_argument("--model", default="124m", choices=sorted(MODELS),
+                    help="124m: the headline workload; medium: the 24-layer, 1024-channel model")
+    ap.add_argument("--micro-batch", type=int, default=None)
     ap.add_argument("--seq", type=int, default=1024)
-    ap.add_argument("--accum", type=int, default=32)
+    ap.add_argument("--accum", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    return ap.parse_args()
+    args = ap.parse_args()
+    m = MODELS[args.model]
+    if args.micro_batch is None:
+        args.micro_batch = m["micro_batch"]
+    if args.accum is None:
+        args.accum = m["accum"]
+    return args
 
 
 def peaks():
@@ -160,14 +188,15 @@ def barrier(world):
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
-def cpu_oracle_sample(seq: int, samples: int = 1):
+def cpu_oracle_sample(seq: int, samples: int = 1, model: str = "124m", seqs_per_step: int = 512):
     """Times the CPU oracle (fp32, as it stands) on B=1 x `seq` tokens of the same model:
-    forward + backward per sample, plus one clip + AdamW step amortised over the 32
-    micro-steps of an optimizer step."""
+    forward + backward per sample, plus one clip + AdamW step amortised over the
+    `seqs_per_step` sequences (micro-batch x accumulation steps) of an optimizer step."""
     import torch
     import oracle as O
     from decoder_only_transformer_train_b200 import synthetic as S
-    cfg = O.GPT2_124M
+    m = MODELS[model]
+    cfg = O.Config(n_layer=m["n_layer"], n_embd=m["n_embd"], n_head=m["n_head"])
     params = O.init_params(cfg, 1, dtype=torch.float32)
     x, y = S.token_batch(3, 1, seq, cfg.vocab_size)
     x, y = torch.from_numpy(x), torch.from_numpy(y)
@@ -183,46 +212,48 @@ def cpu_oracle_sample(seq: int, samples: int = 1):
     t1 = time.perf_counter()
     O.optimizer_step(params, grads, m, v, 1, cfg, lr=O.get_lr(1000))
     t_opt = time.perf_counter() - t1
-    per_micro = t_fb + t_opt / 32
+    per_micro = t_fb + t_opt / seqs_per_step
     return seq / per_micro, torch.get_num_threads(), t_fb, t_opt
 
 
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, world, rank):
     """The oracle, as it stands, on the host cores: each step is a bounded sample of the
-    workload (one B=1 x T micro-batch forward + backward, plus 1/32 of an optimizer step)."""
+    workload (one B=1 x T sequence forward + backward, plus its share of an optimizer step)."""
     if rank != 0:
         return
     import torch
     tok_s, threads, t_fb, t_opt = None, None, None, None
     rates = []
     for i in range(args.warmup + args.steps):
-        r, threads, t_fb, t_opt = cpu_oracle_sample(args.seq)
+        r, threads, t_fb, t_opt = cpu_oracle_sample(args.seq, model=args.model,
+                                                    seqs_per_step=args.micro_batch * args.accum)
         if i >= args.warmup:
             rates.append(r)
     value = statistics.mean(rates)
     ms = args.micro_batch * args.seq * args.accum / value * 1000.0
     line = {
-        "metric": METRIC, "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "metric": metric_name(args.model), "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(args),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": f"GPT-2 124M fp32 CPU oracle, B=1 x T={args.seq} forward+backward "
-                                   f"({t_fb:.2f} s) plus 1/32 of clip+AdamW ({t_opt:.2f} s) per step"},
+                         "sample": f"{MODELS[args.model]['label']} fp32 CPU oracle, B=1 x T={args.seq} forward+backward "
+                                   f"({t_fb:.2f} s) plus 1/{args.micro_batch * args.accum} of clip+AdamW "
+                                   f"({t_opt:.2f} s) per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 def workload_config(args):
-    return {"workload": f"GPT-2 124M training step: B={args.micro_batch} x T={args.seq}, "
+    return {"workload": f"{MODELS[args.model]['label']} training step: B={args.micro_batch} x T={args.seq}, "
                         f"{args.accum} accumulation micro-steps ({args.micro_batch * args.seq * args.accum} tokens), "
                         f"global-norm clip 1.0, AdamW at lr=get_lr(1000)",
             "micro_batch": args.micro_batch, "seq_len": args.seq, "grad_accum_steps": args.accum,
             "tokens_per_step": args.micro_batch * args.seq * args.accum,
             "parallelism": "replicas" if args.gpus > 1 else "single-gpu",
-            "l2": "inputs larger than L2 (0.5 GB params + ~6 GB activations per micro-step)"}
+            "l2": "inputs larger than L2 (every micro-step moves several GB of parameters and activations)"}
 
 
 # ------------------------------------------------------------------ our arm
@@ -236,7 +267,9 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local)
     dist_init(world, "nccl")
     B, T, k = args.micro_batch, args.seq, args.accum
-    cfg = BD.Config(n_layer=12, n_embd=768, n_head=12, block_size=1024, vocab_size=50257, padded_vocab_size=50304,
+    mdl = MODELS[args.model]
+    cfg = BD.Config(n_layer=mdl["n_layer"], n_embd=mdl["n_embd"], n_head=mdl["n_head"], block_size=1024,
+                    vocab_size=50257, padded_vocab_size=50304,
                     max_batch=B, grad_accum_steps=k, precision=BD.GPT2_BF16)
     stream = torch.cuda.Stream(device)
     model = BD.GPT2(cfg, seed=1, stream=stream.cuda_stream)
@@ -321,10 +354,10 @@ def run_ours(args, world, rank, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r, threads, t_fb, t_opt = cpu_oracle_sample(T)
+        r, threads, t_fb, t_opt = cpu_oracle_sample(T, model=args.model, seqs_per_step=B * k)
         cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"GPT-2 124M fp32 CPU oracle, B=1 x T={T} forward+backward ({t_fb:.2f} s) plus "
-                         f"1/32 of clip+AdamW ({t_opt:.2f} s)"}
+               "sample": f"{MODELS[args.model]['label']} fp32 CPU oracle, B=1 x T={T} forward+backward ({t_fb:.2f} s) plus "
+                         f"1/{B * k} of clip+AdamW ({t_opt:.2f} s)"}
 
     if rank == 0:
         pk = peaks()
@@ -357,14 +390,15 @@ def run_ours(args, world, rank, local):
                 ent["gbs"] = round(p["bytes"] / (p["ms"] / 1e3) / 1e9, 1)
             kernels[c] = ent
         per_gpu = value / world
+        fpt = flop_per_token(args.model, args.seq)
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "metric": metric_name(args.model), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(args),
-            "mfu": {"vs_nominal_2250": per_gpu * FLOP_PER_TOKEN / (NOMINAL_BF16_TFLOPS * 1e12),
-                    "vs_measured_sustained": per_gpu * FLOP_PER_TOKEN / (pk["bf16_tflops_sustained"] * 1e12),
-                    "flop_per_token": FLOP_PER_TOKEN},
+            "mfu": {"vs_nominal_2250": per_gpu * fpt / (NOMINAL_BF16_TFLOPS * 1e12),
+                    "vs_measured_sustained": per_gpu * fpt / (pk["bf16_tflops_sustained"] * 1e12),
+                    "flop_per_token": fpt},
             "roofline": roof, "kernels": kernels, "cpu_baseline": cpu, "e2e": e2e,
             "clocks": clk, "gpu_launches": launches,
             "loss": {"after_warmup": first_loss, "after_timed": last_loss},

@@ -124,6 +124,20 @@ def test_tiny_bf16_step_matches_oracle():
     assert torch.equal(torch.from_numpy(r["argmax_gpu"]).long()[clear], O.argmax_lowest(z).long()[clear])
 
 
+# The medium model's width (GPT-2 350M: 1024 channels, 16 heads of 64) with two layers, so
+# that the oracle stays quick: LayerNorm over 1024 columns, the 1024/3072/4096-wide GEMMs and
+# 16-head attention run the kernels of the 24-layer model.
+MEDIUM_WIDTH = O.Config(n_layer=2, n_embd=1024, n_head=16, block_size=256, vocab_size=1000,
+                        padded_vocab_size=1024)
+
+
+def test_medium_width_bf16_step_matches_oracle():
+    r = _run_step(MEDIUM_WIDTH, BD.GPT2_BF16, B=2, T=256)
+    assert abs(r["losses"][0] - r["loss_ref"]) < 2e-2
+    errs = _per_tensor(r["grads_gpu"], r["grads_ref"], MEDIUM_WIDTH)
+    assert max(errs.values()) < 2e-2, {k: v for k, v in errs.items() if v >= 2e-2}
+
+
 def test_grad_accumulation_fp32_equals_one_batch():
     cfg = TINY
     flat = O.flatten(O.init_params(cfg, 5, dtype=torch.float32), cfg).numpy()
