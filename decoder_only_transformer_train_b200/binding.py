@@ -40,6 +40,7 @@ _PROTOS = {
     "gpt2_create": (_i, [ctypes.POINTER(gpt2_config), _u64, ctypes.POINTER(_vp)]),
     "gpt2_destroy": (None, [_vp]),
     "gpt2_set_stream": (_i, [_vp, _vp]),
+    "gpt2_set_graphs": (_i, [_vp, _i]),
     "gpt2_forward": (_i, [_vp, _vp, _vp, _i, _i, _fp]),
     "gpt2_forward_host": (_i, [_vp, _vp, _vp, _i, _i, _fp]),
     "gpt2_backward": (_i, [_vp]),
@@ -164,6 +165,10 @@ class GPT2:
     @property
     def num_params(self) -> int:
         return int(lib().gpt2_num_params(self._h))
+
+    def set_graphs(self, enable: bool):
+        """Replay the forward / backward launch sequences as CUDA graphs (default on)."""
+        _check(lib().gpt2_set_graphs(self._h, int(enable)), self._h)
 
     def forward(self, tokens, targets=None, sync_loss: bool = True) -> float | None:
         """tokens/targets: int32 CUDA tensors [B, T]."""

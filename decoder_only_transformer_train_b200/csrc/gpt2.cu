@@ -1,3 +1,4 @@
+#include <stdlib.h>
 // GPT-2 training step behind the C ABI of gpt2_b200.h: owns the parameters (fp32 master
 // weights in one flat buffer, canonical order), their bf16 copies, the gradients, the
 // AdamW moments and the activation arena, and enqueues the kernels of one forward,
@@ -119,6 +120,15 @@ struct gpt2_ctx {
   int norm_nparts = 0;
 
   int lastB = 0, lastT = 0;
+  // CUDA graphs of the forward / backward launch sequences, one per (kind, B, T): the first
+  // call with a key runs eagerly, the second is captured, later ones replay the graph
+  struct GraphEntry {
+    int kind, B, T, calls;
+    cudaGraphExec_t exec;
+    long long launches;
+  };
+  std::vector<GraphEntry> graphs;
+  bool use_graphs = true;
   bool have_targets = false;
 
   // per-kernel-class CUDA-event profiling (gpt2_profile_start / gpt2_profile_stop)
@@ -538,6 +548,55 @@ int refresh_shadow(gpt2_ctx* c) {
 
 }  // namespace
 
+// Runs the launch sequence `body` (forward_impl or backward_impl) on the context stream:
+// eagerly on the first call with a key, captured into a CUDA graph on the second, replayed
+// after that.  A capture that fails turns graphs off for the context and runs `body` eagerly.
+// Profiling runs eagerly (its events are recorded per launch).
+template <class F>
+static int run_graphed(gpt2_ctx* c, int kind, int B, int T, F body) {
+  if (!c->use_graphs || c->prof_on) return body();
+  gpt2_ctx::GraphEntry* g = nullptr;
+  for (auto& e : c->graphs)
+    if (e.kind == kind && e.B == B && e.T == T) g = &e;
+  if (g == nullptr) {
+    c->graphs.push_back(gpt2_ctx::GraphEntry{kind, B, T, 0, nullptr, 0});
+    g = &c->graphs.back();
+  }
+  if (g->exec == nullptr) {
+    if (g->calls++ == 0) return body();   // modules loaded, kernel attributes set
+    if (cudaStreamBeginCapture(c->stream, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+      cudaGetLastError();
+      c->use_graphs = false;
+      return body();
+    }
+    const long long n0 = kernel_launch_count();
+    const int rc = body();
+    cudaGraph_t graph = nullptr;
+    cudaError_t e = cudaStreamEndCapture(c->stream, &graph);
+    const long long n = kernel_launch_count() - n0;
+    note_kernel_launches((int)-n);   // nothing ran while capturing
+    if (rc != 0 || e != cudaSuccess || graph == nullptr) {
+      if (graph) cudaGraphDestroy(graph);
+      cudaGetLastError();
+      c->use_graphs = false;
+      return rc ? rc : body();
+    }
+    e = cudaGraphInstantiate(&g->exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) {
+      g->exec = nullptr;
+      cudaGetLastError();
+      c->use_graphs = false;
+      return body();
+    }
+    g->launches = n;
+  }
+  cudaError_t e = cudaGraphLaunch(g->exec, c->stream);
+  if (e != cudaSuccess) return cuda_fail(c, e, "graph launch");
+  note_kernel_launches((int)g->launches);
+  return GPT2_OK;
+}
+
 // ====================================================================== C ABI
 extern "C" {
 
@@ -564,6 +623,10 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
       delete c;
       return GPT2_ERR_ARG;   // the tcgen05 path needs sm_100
     }
+  }
+  {
+    const char* ge = getenv("GPT2_B200_GRAPHS");
+    c->use_graphs = !(ge && ge[0] == '0');
   }
   if (cudaStreamCreateWithFlags(&c->own_stream, cudaStreamNonBlocking) != cudaSuccess) {
     delete c;
@@ -675,6 +738,8 @@ fail_out:
 void gpt2_destroy(gpt2_ctx* c) {
   if (c == nullptr) return;
   if (c->stream) cudaStreamSynchronize(c->stream);
+  for (auto& g : c->graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
   for (cudaEvent_t e : c->prof_events) cudaEventDestroy(e);
   for (void* p : c->allocs) cudaFree(p);
   if (c->own_stream) cudaStreamDestroy(c->own_stream);
@@ -684,6 +749,12 @@ void gpt2_destroy(gpt2_ctx* c) {
 int gpt2_set_stream(gpt2_ctx* c, void* s) {
   if (c == nullptr) return GPT2_ERR_ARG;
   c->stream = s ? reinterpret_cast<cudaStream_t>(s) : c->own_stream;
+  return GPT2_OK;
+}
+
+int gpt2_set_graphs(gpt2_ctx* c, int enable) {
+  if (c == nullptr) return GPT2_ERR_ARG;
+  c->use_graphs = enable != 0;
   return GPT2_OK;
 }
 
@@ -702,9 +773,10 @@ static int forward_common(gpt2_ctx* c, const int32_t* tokens, const int32_t* tar
   c->lastB = B;
   c->lastT = T;
   c->have_targets = false;
-  int rc = forward_impl(c, B, T, targets != nullptr);
+  const bool with_t = targets != nullptr;
+  int rc = run_graphed(c, with_t ? 1 : 0, B, T, [&] { return forward_impl(c, B, T, with_t); });
   if (rc) return rc;
-  c->have_targets = targets != nullptr;
+  c->have_targets = with_t;
   if (loss_out) {
     rc = check_device(c);
     if (rc) return rc;
@@ -726,7 +798,7 @@ int gpt2_forward_host(gpt2_ctx* c, const int32_t* tokens, const int32_t* targets
 int gpt2_backward(gpt2_ctx* c) {
   if (c == nullptr) return GPT2_ERR_ARG;
   if (!c->have_targets) return fail(c, GPT2_ERR_STATE, "backward needs a preceding forward with targets");
-  int rc = backward_impl(c);
+  int rc = run_graphed(c, 2, c->lastB, c->lastT, [&] { return backward_impl(c); });
   c->have_targets = false;   // the logits buffer now holds their gradient
   return rc;
 }

@@ -77,6 +77,15 @@ void gpt2_destroy(gpt2_ctx* ctx);
  * selects the library's own stream. */
 int gpt2_set_stream(gpt2_ctx* ctx, void* cuda_stream);
 
+/* Launch the forward and backward passes as CUDA graphs (default: on, unless the
+ * environment variable GPT2_B200_GRAPHS is "0" when the context is created).  For each
+ * (pass, B, T) the first call runs its kernels directly, the second captures them into a
+ * graph on the context stream, and later calls replay that graph, which removes the
+ * per-kernel launch gaps.  The graph holds the context's buffers and the launch decisions
+ * of that shape; results are identical to direct launches.  If a capture fails the context
+ * falls back to direct launches.  Calls made while profiling run directly. */
+int gpt2_set_graphs(gpt2_ctx* ctx, int enable);
+
 /* Forward pass and mean cross-entropy (L9 "Code you'll write": GPT.forward; "52:38 –
  * 1:06:18": F.cross_entropy on flattened logits).
  * tokens, targets: DEVICE int32 [B, T] row-major, caller-owned, read during the call's

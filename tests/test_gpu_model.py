@@ -138,6 +138,34 @@ def test_medium_width_bf16_step_matches_oracle():
     assert max(errs.values()) < 2e-2, {k: v for k, v in errs.items() if v >= 2e-2}
 
 
+def test_graph_replay_matches_direct_launches():
+    """Two optimizer steps of three micro-steps each: with graphs on, the first call of a
+    shape runs directly, the second is captured and the rest replay the graph.  Every loss
+    and every updated weight must equal the direct-launch run bit for bit, and the library's
+    launch counter must count the same kernels."""
+    B, T, k = 2, 64, 3
+    batches = [S.token_batch(5, B, T, TINY.vocab_size, micro_step=i) for i in range(k)]
+    runs = []
+    for graphs in (False, True):
+        model = BD.GPT2(_bd_config(TINY, B, k, BD.GPT2_BF16), seed=1)
+        model.set_graphs(graphs)
+        n0 = BD.lib().gpt2_kernel_launches()
+        losses = []
+        for _ in range(2):
+            model.zero_grad()
+            for x, y in batches:
+                losses.append(model.forward(cuda_i32(x), cuda_i32(y)))
+                model.backward()
+            model.adamw_step(6e-4)
+        model.synchronize()
+        launches = BD.lib().gpt2_kernel_launches() - n0
+        runs.append((losses, model.get_params(), launches))
+        model.close()
+    assert runs[0][0] == runs[1][0]
+    assert np.array_equal(runs[0][1], runs[1][1])
+    assert runs[0][2] == runs[1][2]
+
+
 def test_grad_accumulation_fp32_equals_one_batch():
     cfg = TINY
     flat = O.flatten(O.init_params(cfg, 5, dtype=torch.float32), cfg).numpy()
