@@ -42,12 +42,15 @@ struct TileCfg {
   static constexpr int B_BYTES = B_ROWS * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = CG == 1 ? (BN == 256 ? 4 : (BN == 192 ? 4 : 6))
-                                        : (BN == 256 ? 6 : (BN == 192 ? 6 : 8));
-  static constexpr int STG_BYTES = 8 * 2 * BOX_BYTES;   // 8 epilogue warps x 2 boxes
-  static constexpr int BAR_BYTES = 256;
+                                        : (BN == 256 ? 5 : (BN == 192 ? 5 : 6));
+  // epilogue staging boxes per warp: a pair's smaller stages leave room for a ring of 4, so
+  // epilogue inputs can be loaded ahead
+  static constexpr int NBOX = CG == 2 ? 4 : 2;
+  static constexpr int STG_BYTES = 8 * NBOX * BOX_BYTES;
+  static constexpr int BAR_BYTES = 512;
   static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + BAR_BYTES + 1024;   // +1024: manual alignment
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;   // power of two >= 2*BN
-  static_assert((2 * STAGES + 4 + 8) * 8 + 8 <= BAR_BYTES, "GEMM barriers");
+  static_assert((2 * STAGES + 4 + 8 * NBOX) * 8 + 8 <= BAR_BYTES, "GEMM barriers");
   static_assert(SMEM <= 232448, "GEMM shared memory");
   static_assert(CG == 1 || (BN / 2) % 16 == 0, "CTA-pair tile width");
 };
@@ -169,39 +172,51 @@ __device__ __forceinline__ bool kind_out_bf16(int kind) {
   return kind == EPI_STORE_ACT || kind == EPI_GELU_FWD || kind == EPI_GELU_BWD || kind == EPI_CE_FWD;
 }
 
-// Per-warp epilogue state: two staging boxes used alternately, and the warp's mbarrier for
-// TMA loads of epilogue inputs.
-struct EpiWarp {
-  uint8_t* box0;
-  uint8_t* box1;
-  uint64_t* bar;
-  uint32_t bar_phase;
-  int cur;
+// Per-warp epilogue state: a ring of NB staging boxes, each with an mbarrier for TMA loads of
+// epilogue inputs.  Boxes are handed out in ring order and every box handed out ends in
+// exactly one TMA store (one bulk group), so allocation a is store group a: before
+// allocation a reuses its box, the store of allocation a - NB must have read it.
+template <int NB>
+struct EpiRing {
+  uint8_t* boxes;
+  uint64_t* bars;
+  uint32_t phases;          // bit i: parity of the next completion of bars[i]
+  int alloc;                // boxes handed out so far
+  int stores;               // store groups committed so far
   volatile int* abort_flag;
   int lane;
-  // wait until the box about to be reused is no longer read by an earlier TMA store
-  __device__ __forceinline__ uint8_t* acquire() {
-    if (lane == 0) bulk_wait_group_read<1>();
-    __syncwarp();
-    return cur ? box1 : box0;
-  }
-  __device__ __forceinline__ bool load(uint8_t* b, const CUtensorMap* map, int x, int y) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar, BOX_BYTES);
-      tma_load_2d(b, map, x, y, bar);
+  __device__ __forceinline__ uint8_t* box(int i) const { return boxes + i * BOX_BYTES; }
+  __device__ __forceinline__ int take() {
+    const int a = alloc++;
+    const int pend = stores - 1 - (a - NB);   // store groups that may stay in flight
+    if (a >= NB && lane == 0) {
+      if (pend <= 0) bulk_wait_group_read<0>();
+      else if (pend == 1 || NB == 2) bulk_wait_group_read<1>();
+      else if (pend == 2) bulk_wait_group_read<2>();
+      else bulk_wait_group_read<3>();
     }
-    const bool ok = mbar_wait(bar, bar_phase, abort_flag);
-    bar_phase ^= 1;
+    __syncwarp();
+    return a % NB;
+  }
+  __device__ __forceinline__ void issue_load(int i, const CUtensorMap* map, int x, int y) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars[i], BOX_BYTES);
+      tma_load_2d(box(i), map, x, y, &bars[i]);
+    }
+  }
+  __device__ __forceinline__ bool wait_load(int i) {
+    const bool ok = mbar_wait(&bars[i], (phases >> i) & 1u, abort_flag);
+    phases ^= 1u << i;
     return ok;
   }
-  __device__ __forceinline__ void store(uint8_t* b, const CUtensorMap* map, int x, int y) {
+  __device__ __forceinline__ void store(int i, const CUtensorMap* map, int x, int y) {
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      tma_store_2d(map, x, y, b);
+      tma_store_2d(map, x, y, box(i));
       bulk_commit_group();
     }
-    cur ^= 1;
+    ++stores;
   }
 };
 
@@ -221,8 +236,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* empty_bar = full_bar + Cfg::STAGES;
   uint64_t* tfull_bar = empty_bar + Cfg::STAGES;
   uint64_t* tempty_bar = tfull_bar + 2;
-  uint64_t* epi_bar = tempty_bar + 2;             // [8] one per epilogue warp
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + 8);
+  uint64_t* epi_bar = tempty_bar + 2;             // [8][NBOX] per epilogue warp and box
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + 8 * Cfg::NBOX);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -237,7 +252,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       mbar_init(&tfull_bar[a], 1);
       mbar_init(&tempty_bar[a], 8 * CG);   // one arrival per epilogue warp of every CTA of the group
     }
-    for (int w = 0; w < 8; ++w) mbar_init(&epi_bar[w], 1);
+    for (int w = 0; w < 8 * Cfg::NBOX; ++w) mbar_init(&epi_bar[w], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -344,22 +359,30 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     }
   } else {
     // -------------------------------------------------------------- epilogue
+    constexpr int NB = Cfg::NBOX;
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 2) >> 2;        // which half of the tile's columns
     const int row = q * 32 + lane;
     const int ew = warp - 2;
-    EpiWarp E;
-    E.box0 = stg + (ew * 2) * BOX_BYTES;
-    E.box1 = stg + (ew * 2 + 1) * BOX_BYTES;
-    E.bar = &epi_bar[ew];
-    E.bar_phase = 0;
-    E.cur = 0;
+    EpiRing<NB> E;
+    E.boxes = stg + ew * NB * BOX_BYTES;
+    E.bars = &epi_bar[ew * NB];
+    E.phases = 0;
+    E.alloc = 0;
+    E.stores = 0;
     E.abort_flag = abort_flag;
     E.lane = lane;
     const int kind = ep.kind;
     const bool out_bf16 = kind_out_bf16(kind);
     const bool use_bias = ep.bias != nullptr && kind_has_bias(kind);
     const float alpha = ep.alpha;
+    // inputs read into the staging boxes and overwritten there by the result: residual or
+    // accumulator (fp32, two 16-column boxes per 32-column chunk) or the GELU pre-activation
+    // (bf16, one box per chunk).  The first NB boxes of them are requested before the
+    // accumulator is ready; later ones as boxes retire.
+    const bool has_in = (kind == EPI_RESID_F32 || kind == EPI_ACCUM_F32 || kind == EPI_GELU_BWD);
+    const CUtensorMap* in_map = (kind == EPI_ACCUM_F32) ? &tmOut : &tmIn;
+    const int depth = out_bf16 ? NB : NB / 2;   // chunks loaded ahead
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
@@ -368,22 +391,37 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int t = cl_id; t < ntiles && ok; t += n_cl) {
       int tm, tn, split, kb0, kb1;
       sched.decode(t, tm, tn, split, kb0, kb1);
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
-      tc_fence_after();
       const int row0 = tm * BMT + (int)rank * BM;               // this CTA's rows of the tile
       const int m = row0 + row;
       const int m_warp = row0 + q * 32;                         // first row of this warp's slab
       const int y_out = (kind == EPI_SPLITK) ? split * ep.ld_aux + m_warp : m_warp;   // ws rows per split: ld_aux
-      const int n_base = tn * BN;
+      const int c_begin = tn * BN + half * (BN / 2);            // first column of this warp's half tile
+      // 32-column chunks of the half tile that start inside the matrix (warp-uniform)
+      int nch = 0;
+      if (m_warp < ep.M && c_begin < ep.N) nch = min(BN / 64, (ep.N - c_begin + 31) / 32);
+      // fp32 boxes of chunk c: two, or one when its second 16 columns lie past N
+      auto nbox_of = [&](int c) -> int { return out_bf16 ? 1 : ((c_begin + 32 * c + 16 < ep.N) ? 2 : 1); };
+      auto load_chunk = [&](int c) {
+        const int nb = nbox_of(c);
+        for (int i = 0; i < nb; ++i) {
+          const int bi = E.take();
+          E.issue_load(bi, in_map, c_begin + 32 * c + 16 * i, m_warp);
+        }
+      };
+      const int in_first = E.alloc;                             // allocation index of chunk 0's first input box
+      if (has_in)
+        for (int c = 0; c < min(depth, nch); ++c) load_chunk(c);
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0.0f, 0x7fffffff};
       const int y_row = (kind == EPI_CE_FWD && m < ep.M) ? ep.targets[m] : -1;
+      if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
 #pragma unroll 1
-      for (int c = half * (BN / 2); c < (half + 1) * (BN / 2) && ok; c += 32) {
+      for (int c = 0; c < nch && ok; ++c) {
+        const int col = half * (BN / 2) + 32 * c;               // column within the tile
+        const int n0 = c_begin + 32 * c;
         uint32_t r[32];
-        tmem_ld32(tmem_base + acc * BN + c + (static_cast<uint32_t>(q * 32) << 16), r);
+        tmem_ld32(tmem_base + acc * BN + col + (static_cast<uint32_t>(q * 32) << 16), r);
         tmem_wait_ld();
-        const int n0 = n_base + c;
-        if (n0 >= ep.N || m_warp >= ep.M) continue;            // warp-uniform
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
@@ -407,31 +445,33 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               u[j] = alpha * v[j] + b[j];
               g[j] = gelu_tanh_fast(u[j]);
             }
-            uint8_t* bx = E.acquire();
-            box_put_bf16(bx, lane, u);
+            int bx = E.take();
+            box_put_bf16(E.box(bx), lane, u);
             E.store(bx, &tmOut2, n0, m_warp);
-            bx = E.acquire();
-            box_put_bf16(bx, lane, g);
+            bx = E.take();
+            box_put_bf16(E.box(bx), lane, g);
             E.store(bx, &tmOut, n0, m_warp);
           } else if (kind == EPI_GELU_BWD) {
-            uint8_t* bx = E.acquire();
-            if (!E.load(bx, &tmIn, n0, m_warp)) { ok = false; break; }
+            const int bx = (in_first + c) % NB;
+            if (!E.wait_load(bx)) { ok = false; break; }
             float u[32];
-            box_get_bf16(bx, lane, u);
+            box_get_bf16(E.box(bx), lane, u);
             __syncwarp();
 #pragma unroll
             for (int j = 0; j < 32; ++j) u[j] = alpha * v[j] * gelu_tanh_grad_fast(u[j]);
-            box_put_bf16(bx, lane, u);
+            box_put_bf16(E.box(bx), lane, u);
             E.store(bx, &tmOut, n0, m_warp);
+            if (c + depth < nch) load_chunk(c + depth);
           } else {   // EPI_STORE_ACT, EPI_CE_FWD
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] + b[j];
-            uint8_t* bx = E.acquire();
-            box_put_bf16(bx, lane, v);
+            const int bx = E.take();
+            box_put_bf16(E.box(bx), lane, v);
             E.store(bx, &tmOut, n0, m_warp);
           }
         } else {
           // fp32 output: two 16-column boxes
+          const int ib = in_first + 2 * c;                      // allocation index of chunk c's first input box
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int n1 = n0 + hh * 16;
@@ -442,18 +482,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               const float bj = (use_bias && n1 + j < ep.N) ? ep.bias[n1 + j] : 0.f;
               o[j] = (kind == EPI_SPLITK) ? v[hh * 16 + j] : alpha * v[hh * 16 + j] + bj;
             }
-            uint8_t* bx = E.acquire();
-            if (kind == EPI_RESID_F32 || kind == EPI_ACCUM_F32) {
-              if (!E.load(bx, (kind == EPI_RESID_F32) ? &tmIn : &tmOut, n1, m_warp)) { ok = false; continue; }
+            int bx;
+            if (has_in) {
+              bx = (ib + hh) % NB;
+              if (!E.wait_load(bx)) { ok = false; continue; }
               float in[16];
-              box_get_f32(bx, lane, in);
+              box_get_f32(E.box(bx), lane, in);
               __syncwarp();
 #pragma unroll
               for (int j = 0; j < 16; ++j) o[j] += in[j];
+            } else {
+              bx = E.take();
             }
-            box_put_f32(bx, lane, o);
+            box_put_f32(E.box(bx), lane, o);
             E.store(bx, &tmOut, n1, y_out);
           }
+          if (ok && has_in && c + depth < nch) load_chunk(c + depth);
         }
       }
       if (kind == EPI_CE_FWD && m < ep.M) {
@@ -463,8 +507,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         p.amax = ce.amax;
         p.aidx = ce.aidx;
         ep.ce_part[(long long)m * ep.n_ctiles + tn * 2 + half] = p;
-        const int n_lo = n_base + half * (BN / 2);
-        if (y_row >= n_lo && y_row < min(n_lo + BN / 2, ep.N)) ep.zt[m] = ce.zt;
+        if (y_row >= c_begin && y_row < min(c_begin + BN / 2, ep.N)) ep.zt[m] = ce.zt;
       }
       tc_fence_before();
       __syncwarp();
