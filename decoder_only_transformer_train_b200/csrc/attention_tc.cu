@@ -42,47 +42,37 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 // Row max of a 128-column S tile in TMEM (64 columns per round trip); on the diagonal
-// tile the keys after query row r are left out.
+// tile the keys after query row r are left out.  Four independent max chains.
 template <bool DIAG>
 __device__ __forceinline__ float s_row_max(uint32_t taddr, int r) {
-  float mx = -INFINITY;
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int c0 = 0; c0 < 128; c0 += 64) {
-    uint32_t v0[32], v1[32];
-    tmem_ld32(taddr + c0, v0);
-    tmem_ld32(taddr + c0 + 32, v1);
-    tmem_wait_ld();
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      if (DIAG) {
-        const float a = (c0 + e > r) ? -INFINITY : __uint_as_float(v0[e]);
-        const float b = (c0 + e + 1 > r) ? -INFINITY : __uint_as_float(v0[e + 1]);
-        const float c = (c0 + 32 + e > r) ? -INFINITY : __uint_as_float(v1[e]);
-        const float d = (c0 + 33 + e > r) ? -INFINITY : __uint_as_float(v1[e + 1]);
-        mx = max3f(mx, a, b);
-        mx = max3f(mx, c, d);
-      } else {
-        mx = max3f(mx, __uint_as_float(v0[e]), __uint_as_float(v0[e + 1]));
-        mx = max3f(mx, __uint_as_float(v1[e]), __uint_as_float(v1[e + 1]));
-      }
-    }
-  }
-  return mx;
-}
-
-// P = 2^(s * scale_log2 - m_ref) for a 128-column S row, written as bf16 into row r of a
-// 128 x 128 K-major SW128 operand; returns the row sum of P.
-template <bool DIAG>
-__device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint8_t* prow) {
-  float2 sum = make_float2(0.f, 0.f);
-  const float2 sc = make_float2(scale_log2, scale_log2);
-  const float2 nm = make_float2(-m_ref, -m_ref);
-#pragma unroll 1
   for (int c0 = 0; c0 < 128; c0 += 64) {
     uint32_t v[64];
     tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
     tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
     tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 64; e += 2) {
+      float a = __uint_as_float(v[e]), b = __uint_as_float(v[e + 1]);
+      if (DIAG) {
+        if (c0 + e > r) a = -INFINITY;
+        if (c0 + e + 1 > r) b = -INFINITY;
+      }
+      m4[(e >> 1) & 3] = max3f(m4[(e >> 1) & 3], a, b);
+    }
+  }
+  return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+}
+
+// P = 2^(s * scale_log2 - m_ref) for a 128-column S row, written as bf16 into row r of a
+// 128 x 128 K-major SW128 operand; returns the row sum of P (four independent partial sums).
+template <bool DIAG>
+__device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint8_t* prow) {
+  float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  const float2 sc = make_float2(scale_log2, scale_log2);
+  const float2 nm = make_float2(-m_ref, -m_ref);
+  auto half = [&](int c0, const uint32_t* v) {
 #pragma unroll
     for (int g8 = 0; g8 < 8; ++g8) {
       float p[8];
@@ -96,7 +86,7 @@ __device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_
           if (col > r) p[e] = 0.f;
           if (col + 1 > r) p[e + 1] = 0.f;
         }
-        sum = fadd2(sum, make_float2(p[e], p[e + 1]));
+        sum[e >> 1] = fadd2(sum[e >> 1], make_float2(p[e], p[e + 1]));
       }
       uint4 w;
       w.x = pack_bf16x2(p[0], p[1]);
@@ -105,8 +95,17 @@ __device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_
       w.w = pack_bf16x2(p[6], p[7]);
       *reinterpret_cast<uint4*>(prow + (c0 >> 6) * 16384 + ((g8 ^ (r & 7)) << 4)) = w;
     }
+  };
+#pragma unroll 1
+  for (int c0 = 0; c0 < 128; c0 += 64) {
+    uint32_t v[64];
+    tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
+    tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+    tmem_wait_ld();
+    half(c0, v);
   }
-  return sum.x + sum.y;
+  const float2 s01 = fadd2(sum[0], sum[1]), s23 = fadd2(sum[2], sum[3]);
+  return (s01.x + s01.y) + (s23.x + s23.y);
 }
 
 // Item order shared by all roles: item t -> (query tile, batch*head), heaviest first.
@@ -464,9 +463,9 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
 // Gradients of the causal attention with the probabilities recomputed from the saved
 // log-sum-exp (scaled scores z = q.k / sqrt(hd), P = softmax(z), D = rowsum(dO * O)):
 //   dV = P^T dO,   dZ = P * (dO V^T - D),   dQ = dZ K / sqrt(hd),   dK = dZ^T Q / sqrt(hd).
-// Two kernels keep every sum in a fixed order (no atomics): one CTA per 128-key tile
-// accumulates dK and dV over the query tiles at or after it, one CTA per 128-query tile
-// accumulates dQ over the key tiles at or before it.
+// Two kernels keep every sum in a fixed order (no atomics): the dK/dV kernel accumulates
+// each 128-key tile over the query tiles at or after it, the dQ kernel each 128-query tile
+// over the key tiles at or before it.
 namespace {
 
 constexpr int BWD_THREADS = 576;   // producer, MMA, 16 elementwise warps (4 per TMEM lane quarter)
