@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(32 * LNP_GROUPS) ln_param_reduce_kernel(const 
 // ================================================================ bias gradients
 // out[n] += sum_m x[m, n]: partial sums over COLSUM_CHUNKS row chunks, each in a fixed
 // order, then the chunks summed in order.
-constexpr int COLSUM_CHUNKS = 8;   // row chunks (partials per column)
+constexpr int COLSUM_CHUNKS = 16;  // row chunks (partials per column): 2-4 blocks of 256 threads per SM
 // Block: 8 column groups of 8 columns x 32 row lanes.  Thread (cx, ry) sums rows
 // ry, ry+32, ... of its chunk for columns c0..c0+7 with 16-byte loads; the 32 row lanes are
 // then added in order through shared memory.
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
 #pragma unroll
   for (int i = 0; i < 8; ++i) s[i] = 0.f;
   if (c0 + 8 <= N) {
-#pragma unroll 4
+#pragma unroll 8
     for (int m = m0 + ry; m < m1; m += 32) {
       const T* p = x + (long long)m * ldx + c0;
       if (sizeof(T) == 2) {
@@ -636,10 +636,83 @@ inline int grid_for(long long n, int threads, int cap = 148 * 16) {
 }
 inline int ok() { return cudaGetLastError() == cudaSuccess ? 0 : -3; }
 
+// Same with 16-byte accesses (C a multiple of 128): lane l holds float4 groups l, l + 32, ...;
+// gamma and beta stay in registers across the rows a warp takes (rows warp, warp + stride,
+// ... of a grid sized to the SM count).
+template <typename OutT, int V4>
+__global__ void __launch_bounds__(256) ln_fwd_vec_kernel(const float* __restrict__ x, const float* __restrict__ w,
+                                                         const float* __restrict__ b, OutT* __restrict__ y,
+                                                         float* __restrict__ mean, float* __restrict__ rstd, int N) {
+  constexpr int C = V4 * 128;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4 wv[V4], bv[V4];
+#pragma unroll
+  for (int k = 0; k < V4; ++k) {
+    wv[k] = reinterpret_cast<const float4*>(w)[lane + 32 * k];
+    bv[k] = reinterpret_cast<const float4*>(b)[lane + 32 * k];
+  }
+  for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
+    const float4* xr = reinterpret_cast<const float4*>(x + (long long)row * C);
+    float4 v[V4];
+#pragma unroll
+    for (int k = 0; k < V4; ++k) v[k] = __ldcs(xr + lane + 32 * k);
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < V4; ++k) s += (v[k].x + v[k].y) + (v[k].z + v[k].w);
+    const float mu = warp_sum(s) * (1.0f / C);
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < V4; ++k) {
+      const float a = v[k].x - mu, bq = v[k].y - mu, c = v[k].z - mu, d = v[k].w - mu;
+      ss += (a * a + bq * bq) + (c * c + d * d);
+    }
+    const float r = rsqrtf(warp_sum(ss) * (1.0f / C) + 1e-5f);
+    OutT* yr = y + (long long)row * C;
+#pragma unroll
+    for (int k = 0; k < V4; ++k) {
+      const float o0 = (v[k].x - mu) * r * wv[k].x + bv[k].x, o1 = (v[k].y - mu) * r * wv[k].y + bv[k].y;
+      const float o2 = (v[k].z - mu) * r * wv[k].z + bv[k].z, o3 = (v[k].w - mu) * r * wv[k].w + bv[k].w;
+      const int c = 4 * (lane + 32 * k);
+      if (sizeof(OutT) == 2) {
+        uint2 pk;
+        pk.x = pack_bf16x2(o0, o1);
+        pk.y = pack_bf16x2(o2, o3);
+        *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(yr) + c) = pk;
+      } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(yr) + c) = make_float4(o0, o1, o2, o3);
+      }
+    }
+    if (lane == 0) {
+      mean[row] = mu;
+      rstd[row] = r;
+    }
+  }
+}
+
 template <typename OutT>
 int ln_fwd_dispatch(cudaStream_t st, const float* x, const float* w, const float* b, OutT* y, float* mean,
                     float* rstd, int N, int C) {
   const int grid = cdiv(N, 8);
+  // 16-byte path: x, w, b, y 16-byte aligned and C a multiple of 128
+  const bool vec = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(b) |
+                     reinterpret_cast<uintptr_t>(y)) % 16) == 0;
+  static int nsm = 0;
+  if (nsm == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (nsm <= 0) nsm = 148;
+  }
+  const int vgrid = grid < nsm * 2 ? grid : nsm * 2;   // 2 resident blocks per SM (registers), rows strided
+  if (vec && (C == 768 || C == 1024 || C == 512 || C == 384 || C == 256 || C == 128)) {
+    switch (C) {
+#define LNV(V4) case V4 * 128: ln_fwd_vec_kernel<OutT, V4><<<vgrid, 256, 0, st>>>(x, w, b, y, mean, rstd, N); break;
+      LNV(1) LNV(2) LNV(3) LNV(4) LNV(6) LNV(8)
+#undef LNV
+    }
+    note_kernel_launches(1);
+    return ok();
+  }
   switch (C) {
 #define LNF(CPL) case CPL * 32: ln_fwd_kernel<OutT, CPL><<<grid, 256, 0, st>>>(x, w, b, y, mean, rstd, N); break;
     LNF(1) LNF(2) LNF(4) LNF(8) LNF(12) LNF(16) LNF(24) LNF(32)
