@@ -403,25 +403,43 @@ __global__ void ce_dz_kernel(T* __restrict__ z, long long ld, const float* __res
     st_f(zr + v, (p - (v == y ? 1.f : 0.f)) * sc);
   }
 }
-__global__ void ce_dz_bf16x8_kernel(uint4* __restrict__ z, long long ld8, const float* __restrict__ lse,
-                                    const int* __restrict__ targets, const float* __restrict__ dz_scale, int Vp8) {
-  const int row = blockIdx.y;
-  const int y = targets[row];
-  const float l = lse[row];
-  const float sc = (y >= 0) ? *dz_scale : 0.f;
-  uint4* zr = z + (long long)row * ld8;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < Vp8; i += gridDim.x * blockDim.x) {
-    uint4 q = zr[i];
-    uint32_t* w = reinterpret_cast<uint32_t*>(&q);
+// Persistent over rows (a grid sized to the SM count; block b takes rows b, b + grid, ...):
+// each thread keeps four 16-byte streaming loads in flight.  exp(z - lse) is computed as
+// 2^(z log2e - lse log2e) with the hardware ex2 (the result is rounded to bf16).
+__global__ void __launch_bounds__(512) ce_dz_bf16x8_kernel(uint4* __restrict__ z, long long ld8,
+                                                           const float* __restrict__ lse,
+                                                           const int* __restrict__ targets,
+                                                           const float* __restrict__ dz_scale, int Vp8, int N) {
+  const float LOG2E = 1.4426950408889634f;
+  const float scale = *dz_scale;
+  for (int row = blockIdx.x; row < N; row += gridDim.x) {
+    const int y = targets[row];
+    const float nl = -lse[row] * LOG2E;
+    const float sc = (y >= 0) ? scale : 0.f;
+    uint4* zr = z + (long long)row * ld8;
+    for (int i0 = threadIdx.x; i0 < Vp8; i0 += 4 * blockDim.x) {
+      uint4 q[4];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 f = unpack_bf16x2(w[k]);
-      const int v0 = i * 8 + 2 * k;
-      const float a = (expf(f.x - l) - (v0 == y ? 1.f : 0.f)) * sc;
-      const float b = (expf(f.y - l) - (v0 + 1 == y ? 1.f : 0.f)) * sc;
-      w[k] = pack_bf16x2(a, b);
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < Vp8) q[u] = __ldcs(zr + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i >= Vp8) continue;
+        uint32_t* w = reinterpret_cast<uint32_t*>(&q[u]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 f = unpack_bf16x2(w[k]);
+          const int v0 = i * 8 + 2 * k;
+          const float a = (ex2(fmaf(f.x, LOG2E, nl)) - (v0 == y ? 1.f : 0.f)) * sc;
+          const float bq = (ex2(fmaf(f.y, LOG2E, nl)) - (v0 + 1 == y ? 1.f : 0.f)) * sc;
+          w[k] = pack_bf16x2(a, bq);
+        }
+        __stcs(zr + i, q[u]);
+      }
     }
-    zr[i] = q;
   }
 }
 
@@ -817,8 +835,16 @@ int launch_ce_dz(cudaStream_t st, bool is_bf16, void* logits, long long ld, cons
                  const float* dz_scale, int N, int Vp) {
   if (is_bf16 && Vp % 8 == 0 && ld % 8 == 0) {
     const int v8 = Vp / 8;
-    dim3 grid(cdiv(v8, 256), N);
-    ce_dz_bf16x8_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<uint4*>(logits), ld / 8, lse, targets, dz_scale, v8);
+    static int nsm = 0;
+    if (nsm == 0) {
+      int dev = 0;
+      cudaGetDevice(&dev);
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+      if (nsm <= 0) nsm = 148;
+    }
+    const int grid = N < nsm * 4 ? N : nsm * 4;   // 4 blocks of 512 threads per SM
+    ce_dz_bf16x8_kernel<<<grid, 512, 0, st>>>(reinterpret_cast<uint4*>(logits), ld / 8, lse, targets, dz_scale, v8,
+                                              N);
   } else {
     dim3 grid(cdiv(Vp, 256), N);
     if (is_bf16) ce_dz_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<bf16*>(logits), ld, lse, targets, dz_scale, Vp);
