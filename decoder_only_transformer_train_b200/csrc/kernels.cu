@@ -196,29 +196,25 @@ __global__ void __launch_bounds__(32 * LNP_GROUPS) ln_param_reduce_kernel(const 
 }
 
 // ================================================================ bias gradients
-// out[n] += sum_m x[m, n]: partial sums over COLSUM_CHUNKS row chunks, each in a fixed
-// order, then the chunks summed in order.
-constexpr int COLSUM_CHUNKS = 16;  // row chunks (partials per column): 2-4 blocks of 256 threads per SM
-// Block: 8 column groups of 8 columns x 32 row lanes.  Thread (cx, ry) sums rows
-// ry, ry+32, ... of its chunk for columns c0..c0+7 with 16-byte loads; the 32 row lanes are
-// then added in order through shared memory.
+// out[n] += sum_m x[m, n] (bias gradients), in a fixed order: partial sums over row chunks,
+// then the chunks added in order.
+// Row-contiguous partial column sums: block b sums rows [b rpc, (b + 1) rpc) of every column.
+// A thread owns one 16-byte group of columns (8 bf16 or 4 fp32), reads it down the rows with
+// 8 loads in flight and adds the rows in order; whole rows are read by the block, so DRAM
+// sees contiguous lines.
 template <typename T>
-__global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict__ x, long long ldx, int M, int N,
-                                                             float* __restrict__ part) {
-  __shared__ float red[32][65];
-  const int cx = threadIdx.x & 7, ry = threadIdx.x >> 3;
-  const int c0 = blockIdx.x * 64 + cx * 8;
-  const int rows = cdiv(M, COLSUM_CHUNKS);
-  const int m0 = blockIdx.y * rows, m1 = min(M, m0 + rows);
-  float s[8];
+__global__ void __launch_bounds__(1024) colsum_rows_kernel(const T* __restrict__ x, long long ldx, int M, int N,
+                                                           int rpc, float* __restrict__ part) {
+  constexpr int VEC = 16 / (int)sizeof(T);
+  const int G = N / VEC;
+  const int m0 = blockIdx.x * rpc, m1 = min(M, m0 + rpc);
+  for (int g = threadIdx.x; g < G; g += blockDim.x) {
+    float s[VEC];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) s[i] = 0.f;
-  if (c0 + 8 <= N) {
-#pragma unroll 8
-    for (int m = m0 + ry; m < m1; m += 32) {
-      const T* p = x + (long long)m * ldx + c0;
+    for (int i = 0; i < VEC; ++i) s[i] = 0.f;
+    const T* p = x + (long long)m0 * ldx + g * VEC;
+    auto add = [&](const uint4& q) {
       if (sizeof(T) == 2) {
-        const uint4 q = *reinterpret_cast<const uint4*>(p);
         const uint32_t* u = reinterpret_cast<const uint32_t*>(&q);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -227,41 +223,53 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
           s[2 * i + 1] += f.y;
         }
       } else {
-        const float4 a = *reinterpret_cast<const float4*>(p);
-        const float4 b = *reinterpret_cast<const float4*>(p + 4);
-        s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
-        s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
-      }
-    }
-  } else {
-    for (int m = m0 + ry; m < m1; m += 32)
-      for (int i = 0; i < 8 && c0 + i < N; ++i) s[i] += ld_f(x + (long long)m * ldx + c0 + i);
-  }
+        const float* f = reinterpret_cast<const float*>(&q);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) red[ry][cx * 8 + i] = s[i];
-  __syncthreads();
-  if (threadIdx.x < 64) {
-    const int c = blockIdx.x * 64 + threadIdx.x;
-    float t = 0.f;
-#pragma unroll 8
-    for (int r = 0; r < 32; ++r) t += red[r][threadIdx.x];
-    if (c < N) part[(long long)blockIdx.y * N + c] = t;
+        for (int i = 0; i < 4; ++i) s[i] += f[i];
+      }
+    };
+    int m = m0;
+    for (; m + 8 <= m1; m += 8) {
+      uint4 q[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) q[u] = __ldcs(reinterpret_cast<const uint4*>(p + (long long)(m - m0 + u) * ldx));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) add(q[u]);
+    }
+    for (; m < m1; ++m) add(__ldcs(reinterpret_cast<const uint4*>(p + (long long)(m - m0) * ldx)));
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) part[(long long)blockIdx.x * N + g * VEC + i] = s[i];
   }
 }
-__global__ void colsum_reduce_kernel(const float* __restrict__ part, int nchunks, int N, float* __restrict__ out) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+// out[n] += sum_k part[k][n] in a fixed order.  Block: 32 columns x 16 chunk groups; group g
+// adds chunks g, g + 16, ... in order (8 loads in flight), then the 16 group sums are added
+// in group order.
+__global__ void __launch_bounds__(512) colsum_reduce_kernel(const float* __restrict__ part, int nchunks, int N,
+                                                            float* __restrict__ out) {
+  __shared__ float red[16][33];
+  const int lane = threadIdx.x & 31, gr = threadIdx.x >> 5;
+  const int n = blockIdx.x * 32 + lane;
   float s = 0.f;
-  int k = 0;
-  for (; k + 8 <= nchunks; k += 8) {
-    float v[8];
+  if (n < N) {
+    for (int k0 = gr; k0 < nchunks; k0 += 16 * 8) {
+      float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = part[(long long)(k + i) * N + n];
+      for (int i = 0; i < 8; ++i) {
+        const int k = k0 + 16 * i;
+        v[i] = (k < nchunks) ? part[(long long)k * N + n] : 0.f;
+      }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s += v[i];
+      for (int i = 0; i < 8; ++i) s += v[i];
+    }
   }
-  for (; k < nchunks; ++k) s += part[(long long)k * N + n];
-  out[n] += s;
+  red[gr][lane] = s;
+  __syncthreads();
+  if (gr == 0 && n < N) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t += red[i][lane];
+    out[n] += t;
+  }
 }
 
 // ================================================================ cross-entropy
@@ -797,15 +805,22 @@ int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const float* dy, const f
   return ok();
 }
 
-int colsum_chunks(int M) { return COLSUM_CHUNKS; }
+// Row chunks of the column sums (a function of M only, so the partial buffer sized with it
+// matches every launch): up to 256 chunks of at least 32 rows.
+int colsum_chunks(int M) { return M < 32 ? 1 : (cdiv(M, 32) < 256 ? cdiv(M, 32) : 256); }
 
 int launch_colsum(cudaStream_t st, bool is_bf16, const void* x, long long ldx, int M, int N, float* part,
                   int nchunks, float* out) {
-  if (N % 8 != 0 || ldx % 8 != 0 || nchunks != COLSUM_CHUNKS) return -4;
-  dim3 grid(cdiv(N, 64), nchunks);
-  if (is_bf16) colsum_partial_kernel<bf16><<<grid, 256, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, part);
-  else colsum_partial_kernel<float><<<grid, 256, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, part);
-  colsum_reduce_kernel<<<cdiv(N, 256), 256, 0, st>>>(part, nchunks, N, out);
+  if (N % 8 != 0 || ldx % 8 != 0 || nchunks != colsum_chunks(M) || (reinterpret_cast<uintptr_t>(x) % 16) != 0)
+    return -4;
+  const int rpc = cdiv(M, nchunks);
+  const int used = cdiv(M, rpc);
+  const int groups = N / (is_bf16 ? 8 : 4);
+  int threads = (groups + 31) / 32 * 32;
+  if (threads > 1024) threads = 1024;
+  if (is_bf16) colsum_rows_kernel<bf16><<<used, threads, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, rpc, part);
+  else colsum_rows_kernel<float><<<used, threads, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, rpc, part);
+  colsum_reduce_kernel<<<cdiv(N, 32), 512, 0, st>>>(part, used, N, out);
   note_kernel_launches(2);
   return ok();
 }
