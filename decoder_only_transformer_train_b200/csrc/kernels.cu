@@ -749,10 +749,119 @@ int ln_fwd_dispatch(cudaStream_t st, const float* x, const float* w, const float
   return ok();
 }
 
+// Same with 16-byte accesses (C a multiple of 128): lane l holds float4 column groups
+// l, l + 32, ...; gamma stays in registers and the per-warp accumulators are updated four
+// columns at a time.
+template <typename ActT, int V4>
+__global__ void __launch_bounds__(256, 2) ln_bwd_vec_kernel(const float* __restrict__ dy, const float* __restrict__ x,
+                                                            const float* __restrict__ mean,
+                                                            const float* __restrict__ rstd, const float* __restrict__ w,
+                                                            float* __restrict__ dres, ActT* __restrict__ dres_act,
+                                                            int accumulate, float* __restrict__ part, int N) {
+  constexpr int C = V4 * 128, C4 = C / 4;
+  extern __shared__ float red[];   // [8][3C]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float4* mine = reinterpret_cast<float4*>(red + warp * 3 * C);
+  const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr bool HOIST_W = V4 <= 6;   // wider rows load gamma per row (registers)
+  float4 wv[HOIST_W ? V4 : 1];
+#pragma unroll
+  for (int k = 0; k < V4; ++k) {
+    mine[lane + 32 * k] = z4;
+    mine[C4 + lane + 32 * k] = z4;
+    mine[2 * C4 + lane + 32 * k] = z4;
+    if (HOIST_W) wv[HOIST_W ? k : 0] = __ldg(reinterpret_cast<const float4*>(w) + lane + 32 * k);
+  }
+  for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
+    const float4* dyr = reinterpret_cast<const float4*>(dy + (long long)row * C);
+    const float4* xr = reinterpret_cast<const float4*>(x + (long long)row * C);
+    float4* dr = reinterpret_cast<float4*>(dres + (long long)row * C);
+    const float mu = mean[row], r = rstd[row];
+    float4 g[V4], xh[V4], prev[V4];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < V4; ++k) prev[k] = accumulate ? dr[lane + 32 * k] : z4;   // issued early
+#pragma unroll
+    for (int k = 0; k < V4; ++k) {
+      const int c = lane + 32 * k;
+      const float4 d = __ldcs(dyr + c), xv = __ldcs(xr + c);
+      xh[k] = make_float4((xv.x - mu) * r, (xv.y - mu) * r, (xv.z - mu) * r, (xv.w - mu) * r);
+      const float4 wk = HOIST_W ? wv[HOIST_W ? k : 0] : __ldg(reinterpret_cast<const float4*>(w) + c);
+      g[k] = make_float4(d.x * wk.x, d.y * wk.y, d.z * wk.z, d.w * wk.w);
+      s1 += (g[k].x + g[k].y) + (g[k].z + g[k].w);
+      s2 += (g[k].x * xh[k].x + g[k].y * xh[k].y) + (g[k].z * xh[k].z + g[k].w * xh[k].w);
+      float4 a = mine[c];
+      a.x += d.x * xh[k].x; a.y += d.y * xh[k].y; a.z += d.z * xh[k].z; a.w += d.w * xh[k].w;
+      mine[c] = a;
+      float4 bb = mine[C4 + c];
+      bb.x += d.x; bb.y += d.y; bb.z += d.z; bb.w += d.w;
+      mine[C4 + c] = bb;
+    }
+    s1 = warp_sum(s1) * (1.0f / C);
+    s2 = warp_sum(s2) * (1.0f / C);
+    ActT* da = dres_act + (long long)row * C;
+#pragma unroll
+    for (int k = 0; k < V4; ++k) {
+      const int c = lane + 32 * k;
+      float4 o;
+      o.x = r * (g[k].x - s1 - xh[k].x * s2) + prev[k].x;
+      o.y = r * (g[k].y - s1 - xh[k].y * s2) + prev[k].y;
+      o.z = r * (g[k].z - s1 - xh[k].z * s2) + prev[k].z;
+      o.w = r * (g[k].w - s1 - xh[k].w * s2) + prev[k].w;
+      dr[c] = o;
+      if (sizeof(ActT) == 2) {
+        uint2 pk;
+        pk.x = pack_bf16x2(o.x, o.y);
+        pk.y = pack_bf16x2(o.z, o.w);
+        *reinterpret_cast<uint2*>(reinterpret_cast<bf16*>(da) + 4 * c) = pk;
+      } else {
+        reinterpret_cast<float4*>(da)[c] = o;
+      }
+      float4 t = mine[2 * C4 + c];
+      t.x += o.x; t.y += o.y; t.z += o.z; t.w += o.w;
+      mine[2 * C4 + c] = t;
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < 3 * C; c += blockDim.x) {
+    float sum = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) sum += red[wi * 3 * C + c];
+    part[(long long)blockIdx.x * 3 * C + c] = sum;
+  }
+}
+
 template <typename ActT>
 int ln_bwd_dispatch(cudaStream_t st, const float* dy, const float* x, const float* mean, const float* rstd,
                     const float* w, float* dres, ActT* dres_act, int acc, float* part, int nblocks, int N, int C) {
   const int smem = 8 * 3 * C * (int)sizeof(float);
+  const bool vec = ((reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(x) |
+                     reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(dres) |
+                     reinterpret_cast<uintptr_t>(dres_act)) % 16) == 0;
+  // (fp32 activations at 1024 columns stay on the scalar path: the vector form would spill)
+  const bool vec_c = C == 768 || C == 512 || C == 384 || C == 256 || C == 128 || (C == 1024 && sizeof(ActT) == 2);
+  if (vec && vec_c) {
+    switch (C) {
+#define LNBV(V4)                                                                                                 \
+  case V4 * 128: {                                                                                               \
+    auto k = ln_bwd_vec_kernel<ActT, V4>;                                                                        \
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) return -3; \
+    k<<<nblocks, 256, smem, st>>>(dy, x, mean, rstd, w, dres, dres_act, acc, part, N);                           \
+    break;                                                                                                       \
+  }
+      LNBV(1) LNBV(2) LNBV(3) LNBV(4) LNBV(6)
+      case 8 * 128:
+        if constexpr (sizeof(ActT) == 2) {
+          auto k = ln_bwd_vec_kernel<ActT, 8>;
+          if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) return -3;
+          k<<<nblocks, 256, smem, st>>>(dy, x, mean, rstd, w, dres, dres_act, acc, part, N);
+        }
+        break;
+#undef LNBV
+    }
+    note_kernel_launches(1);
+    return ok();
+  }
   switch (C) {
 #define LNB(CPL)                                                                                               \
   case CPL * 32: {                                                                                             \
