@@ -255,6 +255,13 @@ def argmax_lowest(logits):
 
 
 # ----------------------------------------------------------------------------- model
+def encoder_forward(wte, wpe, tokens):
+    """x0[b, t] = wte[tokens[b, t]] + wpe[t] ([L9] "Code you'll write", forward pass:
+    token embedding plus position embedding).  tokens: int [B, T]."""
+    tok = torch.as_tensor(tokens).long()
+    return wte[tok] + wpe[: tok.shape[1]].unsqueeze(0)
+
+
 def forward(params, cfg: Config, tokens, targets=None):
     """GPT.forward ([L9] "Code you'll write", forward pass with loss): token + position
     embedding, n_layer pre-LayerNorm blocks x = x + attn(ln_1(x)); x = x + mlp(ln_2(x)),
@@ -264,7 +271,7 @@ def forward(params, cfg: Config, tokens, targets=None):
     assert T <= cfg.block_size
     C, H, hd = cfg.n_embd, cfg.n_head, cfg.head_dim
     tok = torch.as_tensor(tokens).long()
-    x = params["wte"][tok] + params["wpe"][:T].unsqueeze(0)          # [B, T, C]
+    x = encoder_forward(params["wte"], params["wpe"], tok)            # [B, T, C]
     cache = {"tokens": tok, "layers": [], "B": B, "T": T}
     for l in range(cfg.n_layer):
         P = lambda n: params[f"h.{l}.{n}"]

@@ -347,6 +347,31 @@ def test_encoder_backward_invariant():
     assert torch.allclose(grads["wte"][v], dx0[where].sum(0), atol=1e-12)
 
 
+def test_encoder_forward_is_adjoint_of_backward():
+    """The embedding is linear in (wte, wpe), so <x0, dx0> = <wte, dwte> + <wpe, dwpe>
+    for the backward's dwte, dwpe; with wte the identity and wpe zero, x0's rows are the
+    one-hot codes of the ids."""
+    g = torch.Generator().manual_seed(8)
+    V, Tmax, C = 11, 9, 11
+    tok = torch.tensor([[3, 3, 0, 10, 7], [1, 3, 9, 9, 2]])
+    wte = torch.randn(V, C, generator=g, dtype=D)
+    wpe = torch.randn(Tmax, C, generator=g, dtype=D)
+    dx0 = torch.randn(2, 5, C, generator=g, dtype=D)
+    x0 = O.encoder_forward(wte, wpe, tok)
+    grads = {"wte": torch.zeros_like(wte), "wpe": torch.zeros_like(wpe)}
+    O.encoder_backward(grads, tok, dx0)
+    lhs = float((x0 * dx0).sum())
+    rhs = float((wte * grads["wte"]).sum() + (wpe * grads["wpe"]).sum())
+    assert abs(lhs - rhs) < 1e-12 * max(1.0, abs(lhs))
+    assert float(grads["wpe"][5:].abs().sum()) == 0.0
+    onehot = O.encoder_forward(torch.eye(V, dtype=D), torch.zeros(Tmax, V, dtype=D), tok)
+    for b in range(2):
+        for t in range(5):
+            row = [0.0] * V
+            row[int(tok[b, t])] = 1.0
+            assert onehot[b, t].tolist() == row
+
+
 def test_grad_accumulation_equals_one_big_batch():
     """[L9] 2:34:49 – 2:46:43: k micro-steps with loss/k give the full-batch gradient."""
     cfg = SMALL
