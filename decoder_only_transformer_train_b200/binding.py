@@ -64,6 +64,9 @@ _PROTOS = {
     "gpt2op_attention_bwd": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
     "gpt2op_attention_bwd_noalloc": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
     "gpt2op_layernorm_fwd": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i]),
+    "gpt2op_embedding_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
+    "gpt2op_embedding_bwd_ws_bytes": (_i64, [_i, _i]),
+    "gpt2op_embedding_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
     "gpt2op_classifier_aux_floats": (_i64, [_i, _i]),
     "gpt2op_classifier_fwd_bwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "gpt2op_device_error": (_i, []),
@@ -300,6 +303,21 @@ def attention_bwd_noalloc(qkv, out, dout, lse, dqkv, B, T, H, head_dim, precisio
 def layernorm_fwd(x, w, b, y, mean, rstd, N, C, precision, stream=None):
     _check(lib().gpt2op_layernorm_fwd(_stream(stream), precision, _ptr(x), _ptr(w), _ptr(b), _ptr(y), _ptr(mean),
                                       _ptr(rstd), N, C))
+
+
+def embedding_fwd(tokens, wte, wpe, x, B, T, C, V, stream=None):
+    _check(lib().gpt2op_embedding_fwd(_stream(stream), _ptr(tokens), _ptr(wte), _ptr(wpe), _ptr(x), B, T, C, V))
+
+
+def embedding_bwd_ws_bytes(N: int, C: int) -> int:
+    return int(lib().gpt2op_embedding_bwd_ws_bytes(N, C))
+
+
+def embedding_bwd(tokens, dx0, dwte, dwpe, B, T, C, V, ws, stream=None):
+    """dwte, dwpe += the embedding gradients of dx0; ws (embedding_bwd_ws_bytes bytes)
+    holds the ascending sort keys token << 15 | position in its first B*T uint32 words."""
+    _check(lib().gpt2op_embedding_bwd(_stream(stream), _ptr(tokens), _ptr(dx0), _ptr(dwte), _ptr(dwpe), B, T, C, V,
+                                      _ptr(ws)))
 
 
 def classifier_aux_floats(N: int, V: int) -> int:

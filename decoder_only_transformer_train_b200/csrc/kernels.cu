@@ -32,24 +32,39 @@ namespace {
 // ================================================================ encoder forward
 // x[n, :] = wte[tok[n], :] + wpe[n mod T, :]   (L9, "Code you'll write": forward pass).
 // Out-of-range ids are reported and embed as zeros.
-__global__ void encoder_fwd_kernel(const int* __restrict__ tok, const float4* __restrict__ wte,
-                                   const float4* __restrict__ wpe, float4* __restrict__ x, int N, int T, int C4,
-                                   int V) {
-  const long long total = (long long)N * C4;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int n = (int)(i / C4), c = (int)(i % C4);
-    const int t = n % T;
-    const int id = tok[n];
-    float4 o;
-    if (id < 0 || id >= V) {
-      if (c == 0) raise_device_error(DEVERR_TOKEN);
-      o = make_float4(0.f, 0.f, 0.f, 0.f);
-    } else {
-      const float4 a = wte[(long long)id * C4 + c], b = wpe[(long long)t * C4 + c];
-      o = make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+// Thread x of a block copies channels 4x .. 4x+3 of four rows per pass, the rows of a
+// block's passes strided by the grid, so that four wte and four wpe loads are in flight.
+__global__ void __launch_bounds__(256) encoder_fwd_kernel(const int* __restrict__ tok,
+                                                          const float4* __restrict__ wte,
+                                                          const float4* __restrict__ wpe, float4* __restrict__ x,
+                                                          int N, int T, int C4, int V) {
+  const int c = blockIdx.y * blockDim.x + threadIdx.x;
+  if (c >= C4) return;
+  for (int n0 = blockIdx.x * 4; n0 < N; n0 += gridDim.x * 4) {
+    float4 a[4], p[4];
+    int id[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int n = n0 + u;
+      id[u] = n < N ? tok[n] : 0;
+      const bool valid = n < N && id[u] >= 0 && id[u] < V;
+      if (valid) {
+        a[u] = __ldg(wte + (long long)id[u] * C4 + c);
+        p[u] = __ldg(wpe + (long long)(n % T) * C4 + c);
+      }
     }
-    x[i] = o;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int n = n0 + u;
+      if (n >= N) break;
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (id[u] < 0 || id[u] >= V) {
+        if (c == 0) raise_device_error(DEVERR_TOKEN);
+      } else {
+        o = make_float4(a[u].x + p[u].x, a[u].y + p[u].y, a[u].z + p[u].z, a[u].w + p[u].w);
+      }
+      x[(long long)n * C4 + c] = o;
+    }
   }
 }
 
@@ -452,95 +467,211 @@ __global__ void __launch_bounds__(512) ce_dz_bf16x8_kernel(uint4* __restrict__ z
 }
 
 // ================================================================ encoder backward
-// dwte[v] += sum of dx0 rows at positions holding token v; dwpe[t] += sum_b dx0[b, t].
-// Deterministic: (token, position) keys are sorted in one CTA (bitonic), runs of equal
-// tokens are summed in position order by fixed 32-entry chunks; a run that crosses chunk
-// boundaries is finished by the chunk where it starts, adding the later chunks' partial
-// sums in chunk order.
+// dwte[v] += sum of dx0 rows at positions holding token v; dwpe[t] += sum_b dx0[b, t]
+// (L9, "Code you'll write": wte and wpe receive the gradient of the residual stream at
+// the first block's input; wte's share adds to the lm_head's, the weight being tied).
+// Deterministic, with no atomics: the (token, position) keys are sorted in one CTA; runs of
+// equal tokens are summed in position order inside fixed ENC_CHUNK-entry chunks; a run that
+// crosses chunk boundaries is finished by the chunk where it starts, which adds the later
+// chunks' partial sums through eight interleaved accumulators combined in a fixed order.
 constexpr int ENC_CHUNK = 32;
 constexpr int ENC_POS_BITS = 15;   // positions < 32768
+constexpr int ENC_SORT_THREADS = 1024;
 
-__global__ void __launch_bounds__(1024) enc_sort_kernel(const int* __restrict__ tok, int N, int V, int P,
-                                                        uint32_t* __restrict__ sorted) {
-  extern __shared__ uint32_t keys[];
-  for (int i = threadIdx.x; i < P; i += 1024) {
-    uint32_t k = 0xFFFFFFFFu;
+__device__ __forceinline__ int key_tok(uint32_t k) { return static_cast<int>(k >> ENC_POS_BITS); }
+__device__ __forceinline__ int key_pos(uint32_t k) { return static_cast<int>(k & ((1u << ENC_POS_BITS) - 1)); }
+// one spare word after every 32, so that a warp reading E consecutive keys per lane
+// (E a power of two up to 32) hits 32 distinct banks
+__device__ __forceinline__ int enc_pad(int i) { return i + (i >> 5); }
+
+// Compare-exchange at register distance J inside one thread's E keys; base is the
+// thread's first key index, k the size of the bitonic sequences being merged.
+template <int J, int E>
+__device__ __forceinline__ void enc_reg_stage(uint32_t (&r)[E], int base, int k) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if ((e & J) == 0) {
+      const uint32_t a = r[e], b = r[e | J];
+      const uint32_t lo = min(a, b), hi = max(a, b);
+      const bool asc = ((base + e) & k) == 0;
+      r[e] = asc ? lo : hi;
+      r[e | J] = asc ? hi : lo;
+    }
+  }
+}
+template <int E>
+__device__ __forceinline__ void enc_reg_stages(uint32_t (&r)[E], int base, int j, int k) {
+  if constexpr (E > 16) if (j == 16) enc_reg_stage<16>(r, base, k);
+  if constexpr (E > 8) if (j == 8) enc_reg_stage<8>(r, base, k);
+  if constexpr (E > 4) if (j == 4) enc_reg_stage<4>(r, base, k);
+  if constexpr (E > 2) if (j == 2) enc_reg_stage<2>(r, base, k);
+  if constexpr (E > 1) if (j == 1) enc_reg_stage<1>(r, base, k);
+}
+
+// Bitonic sort of P = 1024 E keys (tokens clamped to [0, V), key = token << 15 | position;
+// 0xFFFFFFFF past N).  Thread t keeps keys tE .. tE + E-1 in registers: a compare-exchange
+// at distance j < E stays in the thread, E <= j < 32E is one warp shuffle per key, and only
+// the longer distances go through shared memory (15 of the 105 stages for P = 16384).
+template <int E>
+__global__ void __launch_bounds__(ENC_SORT_THREADS) enc_sort_kernel(const int* __restrict__ tok, int N, int V,
+                                                                     uint32_t* __restrict__ sorted) {
+  constexpr int P = ENC_SORT_THREADS * E;
+  extern __shared__ uint32_t s[];   // enc_pad(P) words
+  const int tid = threadIdx.x;
+  for (int i = tid; i < P; i += ENC_SORT_THREADS) {
+    uint32_t key = 0xFFFFFFFFu;
     if (i < N) {
       int t = tok[i];
       t = t < 0 ? 0 : (t >= V ? V - 1 : t);
-      k = (static_cast<uint32_t>(t) << ENC_POS_BITS) | static_cast<uint32_t>(i);
+      key = (static_cast<uint32_t>(t) << ENC_POS_BITS) | static_cast<uint32_t>(i);
     }
-    keys[i] = k;
+    s[enc_pad(i)] = key;
   }
+  __syncthreads();
+  const int base = tid * E;
+  uint32_t r[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) r[e] = s[enc_pad(base + e)];
   for (int k = 2; k <= P; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      __syncthreads();
-      for (int i = threadIdx.x; i < P; i += 1024) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint32_t a = keys[i], b = keys[ixj];
-          const bool asc = (i & k) == 0;
-          if ((a > b) == asc) {
-            keys[i] = b;
-            keys[ixj] = a;
-          }
+      if (j < E) {
+        enc_reg_stages<E>(r, base, j, k);
+        continue;
+      }
+      // the partner of key i is i ^ j, in the same register slot of thread tid ^ (j / E);
+      // key i keeps the smaller of the two when it is the lower index of an ascending pair
+      // or the upper index of a descending one
+      const bool keep_min = ((base & j) == 0) == ((base & k) == 0);
+      if (j < 32 * E) {
+        const int lane_dist = j / E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint32_t b = __shfl_xor_sync(0xffffffffu, r[e], lane_dist);
+          r[e] = keep_min ? min(r[e], b) : max(r[e], b);
+        }
+      } else {
+        __syncthreads();   // every read of the previous shared-memory stage is done
+#pragma unroll
+        for (int e = 0; e < E; ++e) s[enc_pad(base + e)] = r[e];
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const uint32_t b = s[enc_pad((base + e) ^ j)];
+          r[e] = keep_min ? min(r[e], b) : max(r[e], b);
         }
       }
     }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < N; i += 1024) sorted[i] = keys[i];
+#pragma unroll
+  for (int e = 0; e < E; ++e) s[enc_pad(base + e)] = r[e];
+  __syncthreads();
+  for (int i = tid; i < N; i += ENC_SORT_THREADS) sorted[i] = s[enc_pad(i)];
 }
 
-__device__ __forceinline__ int key_tok(uint32_t k) { return static_cast<int>(k >> ENC_POS_BITS); }
-
-__global__ void enc_chunk_kernel(const uint32_t* __restrict__ sorted, const float* __restrict__ dx0,
-                                 float* __restrict__ dwte, float* __restrict__ part, int N, int C) {
+// One block per chunk of ENC_CHUNK sorted keys; thread x sums channels 4x .. 4x+3 of the
+// chunk's rows, eight rows in flight.  A segment (the part of a run inside the chunk) that
+// is a whole run goes straight into dwte; otherwise it is stored as the chunk's partial:
+// slot 0 for the segment at the chunk's start, slot 1 for a run that starts later and
+// leaves through the chunk's end.
+__global__ void __launch_bounds__(256) enc_chunk_kernel(const uint32_t* __restrict__ sorted,
+                                                        const float* __restrict__ dx0, float* __restrict__ dwte,
+                                                        float* __restrict__ part, int N, int C) {
+  __shared__ int tk[ENC_CHUNK + 2];   // tk[1 + i]: token of the chunk's i-th key; tk[0], tk[n + 1]: neighbours or -1
+  __shared__ int ps[ENC_CHUNK];
   const int c = blockIdx.x;
-  const int ch = blockIdx.y * 128 + threadIdx.x * 4;
+  const int i0 = c * ENC_CHUNK, n = min(N - i0, ENC_CHUNK);
+  for (int x = threadIdx.x; x < ENC_CHUNK + 2; x += blockDim.x) {   // blocks may have only 32 threads
+    const int i = i0 - 1 + x;
+    int t = -1;
+    if (i >= 0 && i < N && x <= n + 1) {
+      const uint32_t key = sorted[i];
+      t = key_tok(key);
+      if (x >= 1 && x <= n) ps[x - 1] = key_pos(key);
+    }
+    tk[x] = t;
+  }
+  __syncthreads();
+  const int ch = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
   if (ch >= C) return;
-  const int i0 = c * ENC_CHUNK, i1 = min(N, i0 + ENC_CHUNK);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  int seg_start = i0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = sorted[i];
-    const int t = key_tok(key);
-    const int pos = static_cast<int>(key & ((1u << ENC_POS_BITS) - 1));
-    const float4 d = *reinterpret_cast<const float4*>(dx0 + (long long)pos * C + ch);
-    acc.x += d.x; acc.y += d.y; acc.z += d.z; acc.w += d.w;
-    const bool run_end = (i + 1 == N) || key_tok(sorted[i + 1]) != t;
-    if (run_end || i + 1 == i1) {
-      const bool starts_here = (seg_start > i0) || (i0 == 0) || key_tok(sorted[i0 - 1]) != t;
-      if (starts_here && run_end) {
-        float4* o = reinterpret_cast<float4*>(dwte + (long long)t * C + ch);
-        float4 w = *o;
-        w.x += acc.x; w.y += acc.y; w.z += acc.z; w.w += acc.w;
-        *o = w;
-      } else {
-        const int slot = (seg_start == i0) ? 0 : 1;
-        *reinterpret_cast<float4*>(part + ((long long)c * 2 + slot) * C + ch) = acc;
+  int seg_start = 0;
+  for (int g = 0; g < n; g += 8) {
+    float4 d[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (g + u < n) d[u] = __ldg(reinterpret_cast<const float4*>(dx0 + (long long)ps[g + u] * C + ch));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = g + u;
+      if (i >= n) break;
+      acc.x += d[u].x; acc.y += d[u].y; acc.z += d[u].z; acc.w += d[u].w;
+      const int t = tk[i + 1];
+      const bool run_end = tk[i + 2] != t;
+      if (run_end || i + 1 == n) {
+        const bool starts_here = seg_start > 0 || tk[0] != t;
+        if (starts_here && run_end) {
+          float4* o = reinterpret_cast<float4*>(dwte + (long long)t * C + ch);
+          float4 w = *o;
+          w.x += acc.x; w.y += acc.y; w.z += acc.z; w.w += acc.w;
+          *o = w;
+        } else {
+          const int slot = seg_start == 0 ? 0 : 1;
+          *reinterpret_cast<float4*>(part + ((long long)c * 2 + slot) * C + ch) = acc;
+        }
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        seg_start = i + 1;
       }
-      acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      seg_start = i + 1;
     }
   }
 }
 
-__global__ void enc_fixup_kernel(const uint32_t* __restrict__ sorted, float* __restrict__ dwte,
-                                 const float* __restrict__ part, int N, int C, int nchunks) {
+// The chunk where a boundary-crossing run starts adds its own partial and, over eight
+// interleaved accumulators (chunk c + 1 + q goes to accumulator q mod 8, each in chunk
+// order, then accumulators 0..7 in turn), slot 0 of every later chunk the run covers.
+__global__ void __launch_bounds__(256) enc_fixup_kernel(const uint32_t* __restrict__ sorted,
+                                                        float* __restrict__ dwte, const float* __restrict__ part,
+                                                        int N, int C, int nchunks) {
+  __shared__ int last_chunk;
   const int c = blockIdx.x;
-  const int ch = blockIdx.y * 128 + threadIdx.x * 4;
-  if (ch >= C) return;
   const int i0 = c * ENC_CHUNK, i1 = min(N, i0 + ENC_CHUNK);
   const int t = key_tok(sorted[i1 - 1]);
   const bool crosses_out = (i1 < N) && key_tok(sorted[i1]) == t;
   const bool crosses_in = (i0 > 0) && key_tok(sorted[i0 - 1]) == t && key_tok(sorted[i0]) == t;
   if (!crosses_out || crosses_in) return;
-  const int slot = (key_tok(sorted[i0]) == t) ? 0 : 1;
+  if (threadIdx.x < 32) {
+    // the run's last chunk: one before the first later chunk that starts with another
+    // token (or the end), looked up 32 chunk heads per ballot; chunk c + 1 starts with t
+    int c_last = -1;
+    for (int cb = c + 1; c_last < 0; cb += 32) {
+      const int cc = cb + static_cast<int>(threadIdx.x);
+      const bool other = cc >= nchunks || key_tok(sorted[(long long)cc * ENC_CHUNK]) != t;
+      const unsigned m = __ballot_sync(0xffffffffu, other);
+      if (m) c_last = cb + __ffs(m) - 2;
+    }
+    if (threadIdx.x == 0) last_chunk = c_last;
+  }
+  __syncthreads();
+  const int ch = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  if (ch >= C) return;
+  const int slot = key_tok(sorted[i0]) == t ? 0 : 1;
+  const int cnt = last_chunk - c;
+  float4 a[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q0 = 0; q0 < cnt; q0 += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (q0 + u < cnt) {
+        const float4 p = __ldg(reinterpret_cast<const float4*>(part + (long long)(c + 1 + q0 + u) * 2 * C + ch));
+        a[u].x += p.x; a[u].y += p.y; a[u].z += p.z; a[u].w += p.w;
+      }
+    }
+  }
   float4 tot = *reinterpret_cast<const float4*>(part + ((long long)c * 2 + slot) * C + ch);
-  for (int c2 = c + 1; c2 < nchunks && key_tok(sorted[c2 * ENC_CHUNK]) == t; ++c2) {
-    const float4 p = *reinterpret_cast<const float4*>(part + ((long long)c2 * 2) * C + ch);
-    tot.x += p.x; tot.y += p.y; tot.z += p.z; tot.w += p.w;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    tot.x += a[u].x; tot.y += a[u].y; tot.z += a[u].z; tot.w += a[u].w;
   }
   float4* o = reinterpret_cast<float4*>(dwte + (long long)t * C + ch);
   float4 w = *o;
@@ -548,13 +679,26 @@ __global__ void enc_fixup_kernel(const uint32_t* __restrict__ sorted, float* __r
   *o = w;
 }
 
-__global__ void dwpe_kernel(const float* __restrict__ dx0, float* __restrict__ dwpe, int B, int T, int C) {
-  const long long total = (long long)T * C;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    float s = 0.f;
-    for (int b = 0; b < B; ++b) s += dx0[(long long)b * total + i];
-    dwpe[i] += s;
+// dwpe[t] += sum over b in order of dx0[b, t]: four channels per thread, eight rows in flight.
+__global__ void __launch_bounds__(256) dwpe_kernel(const float4* __restrict__ dx0, float4* __restrict__ dwpe, int B,
+                                                   int TC4) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < TC4; i += gridDim.x * blockDim.x) {
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int b0 = 0; b0 < B; b0 += 8) {
+      float4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (b0 + u < B) v[u] = __ldg(dx0 + (long long)(b0 + u) * TC4 + i);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (b0 + u < B) {
+          s.x += v[u].x; s.y += v[u].y; s.z += v[u].z; s.w += v[u].w;
+        }
+      }
+    }
+    float4 w = dwpe[i];
+    w.x += s.x; w.y += s.y; w.z += s.z; w.w += s.w;
+    dwpe[i] = w;
   }
 }
 
@@ -883,11 +1027,13 @@ int ln_bwd_dispatch(cudaStream_t st, const float* dy, const float* x, const floa
 // ==================================================================== launchers
 int launch_encoder_fwd(cudaStream_t st, const int* tok, const float* wte, const float* wpe, float* x, int N, int T,
                        int C, int V) {
-  if (C % 4) return -4;
-  const long long total = (long long)N * (C / 4);
-  encoder_fwd_kernel<<<grid_for(total, 256), 256, 0, st>>>(tok, reinterpret_cast<const float4*>(wte),
-                                                           reinterpret_cast<const float4*>(wpe),
-                                                           reinterpret_cast<float4*>(x), N, T, C / 4, V);
+  if (N <= 0 || T <= 0 || C <= 0 || C % 4) return -4;
+  const int c4 = C / 4;
+  const int threads = c4 <= 256 ? (c4 + 31) / 32 * 32 : 256;
+  dim3 grid(grid_for(cdiv(N, 4), 1, 148 * 8), cdiv(c4, threads));
+  encoder_fwd_kernel<<<grid, threads, 0, st>>>(tok, reinterpret_cast<const float4*>(wte),
+                                               reinterpret_cast<const float4*>(wpe), reinterpret_cast<float4*>(x),
+                                               N, T, c4, V);
   note_kernel_launches(1);
   return ok();
 }
@@ -980,22 +1126,44 @@ int launch_ce_dz(cudaStream_t st, bool is_bf16, void* logits, long long ld, cons
 
 size_t encoder_bwd_part_floats(int N, int C) { return (size_t)cdiv(N, ENC_CHUNK) * 2 * (size_t)C; }
 
+template <int E>
+static int enc_sort_launch(cudaStream_t st, const int* tok, int N, int V, uint32_t* sorted) {
+  const int smem = (ENC_SORT_THREADS * E + ENC_SORT_THREADS * E / 32) * (int)sizeof(uint32_t);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(enc_sort_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return -3;
+  enc_sort_kernel<E><<<1, ENC_SORT_THREADS, smem, st>>>(tok, N, V, sorted);
+  return 0;
+}
+
 int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float* dwte, float* dwpe, int B, int T,
                        int C, uint32_t* sorted_keys, float* chunk_part, int V) {
-  const int N = B * T;
-  if (N > (1 << ENC_POS_BITS) || V > (1 << (32 - ENC_POS_BITS)) || C % 4) return -4;
-  int P = 1;
+  const long long Nll = (long long)B * T;
+  if (B <= 0 || T <= 0 || Nll > (1 << ENC_POS_BITS) || V <= 0 || V > (1 << (32 - ENC_POS_BITS)) || C <= 0 ||
+      C % 4)
+    return -4;
+  const int N = (int)Nll;
+  int P = ENC_SORT_THREADS;
   while (P < N) P <<= 1;
-  const int smem = P * (int)sizeof(uint32_t);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(enc_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return -3;
-  enc_sort_kernel<<<1, 1024, smem, st>>>(tok, N, V, P, sorted_keys);
+  int rc;
+  switch (P / ENC_SORT_THREADS) {
+    case 1: rc = enc_sort_launch<1>(st, tok, N, V, sorted_keys); break;
+    case 2: rc = enc_sort_launch<2>(st, tok, N, V, sorted_keys); break;
+    case 4: rc = enc_sort_launch<4>(st, tok, N, V, sorted_keys); break;
+    case 8: rc = enc_sort_launch<8>(st, tok, N, V, sorted_keys); break;
+    case 16: rc = enc_sort_launch<16>(st, tok, N, V, sorted_keys); break;
+    default: rc = enc_sort_launch<32>(st, tok, N, V, sorted_keys); break;
+  }
+  if (rc) return rc;
   const int nchunks = cdiv(N, ENC_CHUNK);
-  dim3 grid(nchunks, cdiv(C, 128));
-  enc_chunk_kernel<<<grid, 32, 0, st>>>(sorted_keys, dx0, dwte, chunk_part, N, C);
-  enc_fixup_kernel<<<grid, 32, 0, st>>>(sorted_keys, dwte, chunk_part, N, C, nchunks);
-  dwpe_kernel<<<grid_for((long long)T * C, 256), 256, 0, st>>>(dx0, dwpe, B, T, C);
+  const int c4 = C / 4;
+  const int threads = c4 <= 256 ? (c4 + 31) / 32 * 32 : 256;
+  dim3 grid(nchunks, cdiv(c4, threads));
+  enc_chunk_kernel<<<grid, threads, 0, st>>>(sorted_keys, dx0, dwte, chunk_part, N, C);
+  enc_fixup_kernel<<<grid, threads, 0, st>>>(sorted_keys, dwte, chunk_part, N, C, nchunks);
+  const int tc4 = T * c4;
+  dwpe_kernel<<<grid_for(tc4, 256), 256, 0, st>>>(reinterpret_cast<const float4*>(dx0),
+                                                  reinterpret_cast<float4*>(dwpe), B, tc4);
   note_kernel_launches(4);
   return ok();
 }

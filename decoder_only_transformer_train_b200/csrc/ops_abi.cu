@@ -88,6 +88,32 @@ int gpt2op_layernorm_fwd(void* stream, int precision, const float* x, const floa
   return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
 }
 
+int gpt2op_embedding_fwd(void* stream, const int32_t* tokens, const float* wte, const float* wpe, float* x, int B,
+                         int T, int C, int V) {
+  if (!tokens || !wte || !wpe || !x) return GPT2_ERR_ARG;
+  if (B <= 0 || T <= 0 || C <= 0 || V <= 0 || C % 4 || (long long)B * T > INT32_MAX) return GPT2_ERR_SHAPE;
+  const int rc = launch_encoder_fwd(reinterpret_cast<cudaStream_t>(stream), tokens, wte, wpe, x, B * T, T, C, V);
+  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+}
+
+static int64_t embedding_keys_bytes(int N) { return ((int64_t)N * 4 + 255) / 256 * 256; }
+
+int64_t gpt2op_embedding_bwd_ws_bytes(int N, int C) {
+  if (N <= 0 || C <= 0) return 0;
+  return embedding_keys_bytes(N) + (int64_t)encoder_bwd_part_floats(N, C) * 4;
+}
+
+int gpt2op_embedding_bwd(void* stream, const int32_t* tokens, const float* dx0, float* dwte, float* dwpe, int B,
+                         int T, int C, int V, void* ws) {
+  if (!tokens || !dx0 || !dwte || !dwpe || !ws) return GPT2_ERR_ARG;
+  if (B <= 0 || T <= 0 || C <= 0 || V <= 0 || C % 4 || (long long)B * T > 32768) return GPT2_ERR_SHAPE;
+  char* w = static_cast<char*>(ws);
+  const int rc = launch_encoder_bwd(reinterpret_cast<cudaStream_t>(stream), tokens, dx0, dwte, dwpe, B, T, C,
+                                    reinterpret_cast<uint32_t*>(w),
+                                    reinterpret_cast<float*>(w + embedding_keys_bytes(B * T)), V);
+  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+}
+
 int64_t gpt2op_classifier_aux_floats(int N, int V) {
   const int ntiles = gemm_tc_ce_tiles(V);
   // partials (4 floats each), zt, loss_row, and 8 scalars

@@ -6,7 +6,7 @@ GPT-2 124M training step with B micro-batch rows of T tokens (default B=16, T=10
 
 Each case is timed with CUDA events on the current stream over N launches after W warm-up
 launches and printed as one line: microseconds per launch and TFLOP/s (GEMM, attention) or
-GB/s of algorithmic bytes (LayerNorm).  With --flush-l2 every launch is timed on its own
+GB/s of algorithmic bytes (LayerNorm, embedding).  With --flush-l2 every launch is timed on its own
 after a 256 MiB write that evicts L2; otherwise the N launches run back to back.  Inputs are
 seeded normal values made on the device; the numbers measure speed only.  Device memory
 stays under about 5 GB, so one case can run under a profiler."""
@@ -17,6 +17,7 @@ import re
 import torch
 
 from decoder_only_transformer_train_b200 import binding as BD
+from decoder_only_transformer_train_b200 import synthetic as S
 
 
 def gemm_cases(ntok, C, V):
@@ -159,6 +160,32 @@ def main(argv=None):
         ms = timer(fn, args.iters, args.warmup)
         nbytes = ntok * C * (4 + 2) + ntok * 8
         report("ln_fwd", ms, N=ntok, C=C, gbs=round(nbytes / (ms * 1e-3) / 1e9, 1))
+
+    if sel.search("embed_fwd") or sel.search("embed_bwd"):
+        # Zipf ids over the real vocabulary, as in the training step's synthetic batches
+        ids = S.zipf_tokens(7, ntok, 50257)
+        tok = torch.from_numpy(ids).cuda()
+        distinct = int(len(set(ids.tolist())))
+        if sel.search("embed_fwd"):
+            wte, wpe = rnd(50257, C, dt=torch.float32), rnd(T, C, dt=torch.float32)
+            x = torch.empty(ntok, C, dtype=torch.float32, device=dev)
+            fn = lambda: BD.embedding_fwd(tok, wte, wpe, x, B, T, C, 50257)
+            ms = timer(fn, args.iters, args.warmup)
+            # x written once; each distinct wte row and each wpe row read once
+            nbytes = ntok * C * 4 + (distinct + T) * C * 4
+            report("embed_fwd", ms, N=ntok, C=C, gbs=round(nbytes / (ms * 1e-3) / 1e9, 1))
+            del wte, wpe, x
+        if sel.search("embed_bwd"):
+            dx0 = rnd(ntok, C, dt=torch.float32)
+            dwte = torch.zeros(50257, C, dtype=torch.float32, device=dev)
+            dwpe = torch.zeros(T, C, dtype=torch.float32, device=dev)
+            ws = torch.empty(BD.embedding_bwd_ws_bytes(ntok, C), dtype=torch.uint8, device=dev)
+            fn = lambda: BD.embedding_bwd(tok, dx0, dwte, dwpe, B, T, C, 50257, ws)
+            ms = timer(fn, args.iters, args.warmup)
+            # dx0 read once; the distinct dwte rows and every dwpe row read and written
+            nbytes = ntok * C * 4 + 2 * (distinct + T) * C * 4
+            report("embed_bwd", ms, N=ntok, C=C, distinct=distinct, gbs=round(nbytes / (ms * 1e-3) / 1e9, 1))
+            del dx0, dwte, dwpe, ws
 
     for Vc, name in ((V, "classifier"), (50257, "classifier_50257")):
         if not sel.search(name):

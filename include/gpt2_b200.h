@@ -220,6 +220,24 @@ int gpt2op_attention_bwd_noalloc(void* stream, int precision, const void* qkv, c
 int gpt2op_layernorm_fwd(void* stream, int precision, const float* x, const float* w, const float* b, void* y,
                          float* mean, float* rstd, int N, int C);
 
+/* Token and position embedding ("Karpathy's Zero to Hero, Lecture 9: Reproduce GPT-2
+ * (124M)" notes, "Code you'll write": the forward pass adds wte[token] and wpe[position]).
+ * Forward: x f32 [B*T, C] = wte[tokens[n]] + wpe[n mod T] from f32 tables wte [V, C] and
+ * wpe [>= T, C]; tokens int32 [B*T].  An id outside [0, V) embeds as zeros and sets the
+ * device error word to GPT2_ERR_TOKEN (read with gpt2op_device_error).
+ * Backward: dwte[v] += the sum of the rows of dx0 (f32 [B*T, C]) at positions holding
+ * token v, dwpe[t] += sum over b of dx0[b*T + t]; ids are clamped into [0, V).  The sums
+ * are deterministic (no atomics; a fixed order that depends only on the ids).  ws is
+ * device scratch of gpt2op_embedding_bwd_ws_bytes(B*T, C) bytes, 256-byte aligned; after
+ * the call its first B*T uint32 words hold the sort keys token << 15 | position in
+ * ascending order.  Both: GPT2_ERR_ARG for a null pointer; GPT2_ERR_SHAPE unless B, T,
+ * C, V > 0, C % 4 == 0, and for the backward B*T <= 32768 and V <= 131072. */
+int gpt2op_embedding_fwd(void* stream, const int32_t* tokens, const float* wte, const float* wpe, float* x, int B,
+                         int T, int C, int V);
+int64_t gpt2op_embedding_bwd_ws_bytes(int N, int C);
+int gpt2op_embedding_bwd(void* stream, const int32_t* tokens, const float* dx0, float* dwte, float* dwpe, int B,
+                         int T, int C, int V, void* ws);
+
 /* Fused classifier head (lm_head + softmax + cross-entropy), forward and backward, on
  * caller buffers: h bf16 [N, C] (the final LayerNorm output), W bf16 [V, C] (the tied
  * weight), targets int32 [N] in [0, V) or -1.  Writes loss (f32 scalar, mean over
