@@ -67,9 +67,13 @@ __device__ __forceinline__ float s_row_max(uint32_t taddr, int r) {
 
 // P = 2^(s * scale_log2 - m_ref) for a 128-column S row, written as bf16 into row r of a
 // 128 x 128 K-major SW128 operand; returns the row sum of P (four independent partial sums).
-template <bool DIAG>
-__device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint8_t* prow) {
+// With MAX, the same pass also returns the row's raw max in *mx (masked keys left out), so
+// that a tile whose max stays within the rescale threshold of m_ref is read from TMEM once.
+template <bool DIAG, bool MAX = false>
+__device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint8_t* prow,
+                                             float* mx = nullptr) {
   float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   const float2 sc = make_float2(scale_log2, scale_log2);
   const float2 nm = make_float2(-m_ref, -m_ref);
   auto half = [&](int c0, const uint32_t* v) {
@@ -78,13 +82,20 @@ __device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_
       float p[8];
 #pragma unroll
       for (int e = 0; e < 8; e += 2) {
-        const float2 x = ffma2(make_float2(__uint_as_float(v[g8 * 8 + e]), __uint_as_float(v[g8 * 8 + e + 1])), sc, nm);
+        const float sa = __uint_as_float(v[g8 * 8 + e]), sb = __uint_as_float(v[g8 * 8 + e + 1]);
+        const float2 x = ffma2(make_float2(sa, sb), sc, nm);
         p[e] = ex2(x.x);
         p[e + 1] = ex2(x.y);
         if (DIAG) {
           const int col = c0 + g8 * 8 + e;
           if (col > r) p[e] = 0.f;
           if (col + 1 > r) p[e + 1] = 0.f;
+        }
+        if (MAX) {
+          const int col = c0 + g8 * 8 + e;
+          const float ma = (DIAG && col > r) ? -INFINITY : sa;
+          const float mb = (DIAG && col + 1 > r) ? -INFINITY : sb;
+          m4[e >> 1] = max3f(m4[e >> 1], ma, mb);
         }
         sum[e >> 1] = fadd2(sum[e >> 1], make_float2(p[e], p[e + 1]));
       }
@@ -104,6 +115,7 @@ __device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_
     tmem_wait_ld();
     half(c0, v);
   }
+  if (MAX) *mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
   const float2 s01 = fadd2(sum[0], sum[1]), s23 = fadd2(sum[2], sum[3]);
   return (s01.x + s01.y) + (s23.x + s23.y);
 }
@@ -293,31 +305,46 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         tc_fence_after();
         const bool diag = (j == qt);
         const uint32_t srow = tmem + lane_off + s_col;
-        const float mx = diag ? s_row_max<true>(srow, r) : s_row_max<false>(srow, r);
-        const float m_new = mx * scale_log2;
-        // the group's previous P.V MMA must be done: P buffer free, O stable
-        if (!mbar_wait(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
+        float sum;
         if (!has) {
-          m_ref = m_new;
-        } else if (m_new > m_ref + RESCALE_THRESHOLD) {
-          const float f = ex2(m_ref - m_new);
-          tc_fence_after();
+          // the group's first tile of the item: its row max sets m_ref (two TMEM passes)
+          const float mx = diag ? s_row_max<true>(srow, r) : s_row_max<false>(srow, r);
+          // the group's previous P.V MMA must be done: P buffer free, O stable
+          if (!mbar_wait(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
+          m_ref = mx * scale_log2;
+          sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, prow)
+                     : p_row_store<false>(srow, r, scale_log2, m_ref, prow);
+        } else {
+          // one pass: P against the current m_ref, and the tile's row max alongside
+          if (!mbar_wait(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
+          float mx;
+          sum = diag ? p_row_store<true, true>(srow, r, scale_log2, m_ref, prow, &mx)
+                     : p_row_store<false, true>(srow, r, scale_log2, m_ref, prow, &mx);
+          const float m_new = mx * scale_log2;
+          const bool grow = m_new > m_ref + RESCALE_THRESHOLD;
+          // tcgen05.ld / st are warp-collective, so the whole warp takes this branch when
+          // any of its rows' max grew past the threshold: those rows rescale O and l and
+          // write P again against the new max; the others scale by exactly 1 and write the
+          // same P again.
+          if (__any_sync(0xffffffffu, grow)) {
+            const float f = grow ? ex2(m_ref - m_new) : 1.0f;
+            tc_fence_after();
 #pragma unroll
-          for (int c0 = 0; c0 < HD; c0 += 16) {
-            uint32_t v[16];
-            tmem_ld16(tmem + lane_off + O_COL + grp * HD + c0, v);
-            tmem_wait_ld();
+            for (int c0 = 0; c0 < HD; c0 += 16) {
+              uint32_t v[16];
+              tmem_ld16(tmem + lane_off + O_COL + grp * HD + c0, v);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-            tmem_st16(tmem + lane_off + O_COL + grp * HD + c0, v);
+              for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+              tmem_st16(tmem + lane_off + O_COL + grp * HD + c0, v);
+            }
+            tmem_wait_st();
+            l *= f;
+            if (grow) m_ref = m_new;
+            sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, prow)
+                       : p_row_store<false>(srow, r, scale_log2, m_ref, prow);
           }
-          tmem_wait_st();
-          l *= f;
-          m_ref = m_new;
         }
-        // pass 2: P = 2^(s*scale*log2e - m_ref) to shared memory, row sum
-        const float sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, prow)
-                               : p_row_store<false>(srow, r, scale_log2, m_ref, prow);
         l += sum;
         tc_fence_before();
         mbar_arrive(&s_empty[grp]);

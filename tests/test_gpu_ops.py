@@ -203,6 +203,37 @@ def test_attention_forward_backward(prec, B, T, H, hd):
     assert rel_l2(g[:, 2 * C:], merge(dv)) < tol_g
 
 
+@pytest.mark.parametrize("prec", [BD.GPT2_FP32, BD.GPT2_BF16])
+@pytest.mark.parametrize("B,T,H", [(2, 1024, 3), (1, 700, 2)])
+def test_attention_forward_when_the_row_max_keeps_growing(prec, B, T, H):
+    """Keys scaled up along the sequence (and queries by 3) make a row's max grow by more
+    than the kernel's rescale threshold from one key tile to the next, so the accumulated
+    output is rescaled and the tile's probabilities recomputed many times per row."""
+    hd = 64
+    C = H * hd
+    qkv = _randn((B * T, 3 * C), 97 + T)
+    pos = torch.arange(B * T, dtype=torch.float64) % T
+    qkv[:, :C] *= 3.0
+    qkv[:, C:2 * C] *= (1.0 + pos / 64.0)[:, None]
+    if prec == BD.GPT2_BF16:
+        qkv = bf16_round(qkv)
+    heads = lambda t: t.reshape(B, T, H, hd).transpose(1, 2)
+    q, k, v = (heads(t) for t in qkv.split(C, dim=1))
+    o_ref, _ = O.causal_attention_forward(q, k, v)
+    lse_ref = torch.logsumexp(
+        (q @ k.transpose(-1, -2) / math.sqrt(hd)).masked_fill(torch.ones(T, T, dtype=torch.bool).triu(1),
+                                                              float("-inf")), dim=-1)
+    dt = torch.bfloat16 if prec == BD.GPT2_BF16 else torch.float32
+    out_d = torch.zeros(B * T, C, dtype=dt, device="cuda")
+    lse_d = torch.zeros(B * H * T, dtype=torch.float32, device="cuda")
+    BD.attention_fwd(qkv.to(dt).cuda(), out_d, lse_d, B, T, H, hd, prec)
+    torch.cuda.synchronize()
+    assert BD.device_error() == 0
+    merge = lambda t: t.transpose(1, 2).reshape(B * T, C)
+    assert rel_l2(out_d.cpu(), merge(o_ref)) < (1e-5 if prec == BD.GPT2_FP32 else 5e-3)
+    assert torch.allclose(lse_d.cpu().double(), lse_ref.reshape(-1), rtol=1e-5, atol=1e-4)
+
+
 # ------------------------------------------------------------------ LayerNorm
 @pytest.mark.parametrize("prec", [BD.GPT2_FP32, BD.GPT2_BF16])
 @pytest.mark.parametrize("N,C", [(77, 64), (1000, 768), (33, 1024)])
