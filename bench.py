@@ -44,10 +44,10 @@ def flop_per_token(model: str, T: int = 1024, Vp: int = 50304) -> int:
 FLOP_PER_TOKEN = flop_per_token("124m")   # 798,031,872
 
 
-def metric_name(model: str) -> str:
-    if model == "124m":
+def metric_name(model: str, B: int = 16, T: int = 1024) -> str:
+    if model == "124m" and (B, T) == (16, 1024):
         return METRIC
-    return f"{MODELS[model]['label']} train tokens/sec (1 B200); ms/step; MFU vs BF16 peak"
+    return f"{MODELS[model]['label']} train tokens/sec (B={B},T={T}, 1 B200); ms/step; MFU vs BF16 peak"
 NOMINAL_BF16_TFLOPS = 2250.0
 
 
@@ -66,10 +66,12 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     m = MODELS[args.model]
+    # a longer context keeps the model's tokens per micro-step (the embedding backward sorts
+    # at most 32768 positions) and per step (e.g. T=2048: B=16, 16 micro-steps for the 124M model)
     if args.micro_batch is None:
-        args.micro_batch = m["micro_batch"]
+        args.micro_batch = max(1, min(m["micro_batch"], 32768 // args.seq))
     if args.accum is None:
-        args.accum = m["accum"]
+        args.accum = max(1, m["micro_batch"] * m["accum"] * 1024 // (args.micro_batch * args.seq))
     return args
 
 
@@ -196,7 +198,7 @@ def cpu_oracle_sample(seq: int, samples: int = 1, model: str = "124m", seqs_per_
     import oracle as O
     from decoder_only_transformer_train_b200 import synthetic as S
     m = MODELS[model]
-    cfg = O.Config(n_layer=m["n_layer"], n_embd=m["n_embd"], n_head=m["n_head"])
+    cfg = O.Config(n_layer=m["n_layer"], n_embd=m["n_embd"], n_head=m["n_head"], block_size=max(1024, seq))
     params = O.init_params(cfg, 1, dtype=torch.float32)
     x, y = S.token_batch(3, 1, seq, cfg.vocab_size)
     x, y = torch.from_numpy(x), torch.from_numpy(y)
@@ -233,7 +235,7 @@ def run_reference(args, world, rank):
     value = statistics.mean(rates)
     ms = args.micro_batch * args.seq * args.accum / value * 1000.0
     line = {
-        "metric": metric_name(args.model), "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "metric": metric_name(args.model, args.micro_batch, args.seq), "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(args),
@@ -268,7 +270,7 @@ def run_ours(args, world, rank, local):
     dist_init(world, "nccl")
     B, T, k = args.micro_batch, args.seq, args.accum
     mdl = MODELS[args.model]
-    cfg = BD.Config(n_layer=mdl["n_layer"], n_embd=mdl["n_embd"], n_head=mdl["n_head"], block_size=1024,
+    cfg = BD.Config(n_layer=mdl["n_layer"], n_embd=mdl["n_embd"], n_head=mdl["n_head"], block_size=max(1024, T),
                     vocab_size=50257, padded_vocab_size=50304,
                     max_batch=B, grad_accum_steps=k, precision=BD.GPT2_BF16)
     stream = torch.cuda.Stream(device)
@@ -392,7 +394,7 @@ def run_ours(args, world, rank, local):
         per_gpu = value / world
         fpt = flop_per_token(args.model, args.seq)
         line = {
-            "metric": metric_name(args.model), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "metric": metric_name(args.model, args.micro_batch, args.seq), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(args),

@@ -138,6 +138,62 @@ def test_medium_width_bf16_step_matches_oracle():
     assert max(errs.values()) < 2e-2, {k: v for k, v in errs.items() if v >= 2e-2}
 
 
+# The GPT-3 context length with the 124M model's head size ("Karpathy's Zero to Hero, Lecture 9"
+# notes, "3:41:50 – 3:53:37 Results: one epoch and an overnight run": T = 2048 to match GPT-3):
+# 16 key tiles per query row in the attention kernels, a 2048-row position table.
+LONG_CONTEXT = O.Config(n_layer=2, n_embd=128, n_head=2, block_size=2048, vocab_size=1000, padded_vocab_size=1024)
+
+
+def test_context_2048_bf16_step_matches_oracle():
+    r = _run_step(LONG_CONTEXT, BD.GPT2_BF16, B=1, T=2048)
+    assert abs(r["losses"][0] - r["loss_ref"]) < 2e-2
+    errs = _per_tensor(r["grads_gpu"], r["grads_ref"], LONG_CONTEXT)
+    assert max(errs.values()) < 2e-2, {k: v for k, v in errs.items() if v >= 2e-2}
+
+
+def test_resume_from_saved_state_continues_bit_for_bit():
+    """Exact resume ("Karpathy's Zero to Hero, Lecture 9" notes, "3:53:37 – 3:59:21
+    Checkpoints, fine-tuning and llm.c": the weights alone are not enough, AdamW's m and v
+    and the random state are needed too).  Three steps straight through must equal two
+    steps, a save of (params, m, v, t), a fresh context restored from it, and the third
+    step, bit for bit.  The token stream is a counter-based generator, so the data position
+    is the micro-step index; the model itself draws no random numbers after init."""
+    B, T, k = 2, 64, 2
+    batches = lambda step: [S.token_batch(21, B, T, TINY.vocab_size, micro_step=step * k + i) for i in range(k)]
+
+    def train(model, step):
+        model.zero_grad()
+        losses = []
+        for x, y in batches(step):
+            losses.append(model.forward(cuda_i32(x), cuda_i32(y)))
+            model.backward()
+        norm = model.adamw_step(O.get_lr(step + 1))
+        return losses, norm
+
+    straight = BD.GPT2(_bd_config(TINY, B, k, BD.GPT2_BF16), seed=3)
+    log_a = [train(straight, s) for s in range(3)]
+    final_a = straight.get_params()
+    m_a, v_a, t_a = straight.get_optimizer_state()
+    straight.close()
+
+    first = BD.GPT2(_bd_config(TINY, B, k, BD.GPT2_BF16), seed=3)
+    log_b = [train(first, s) for s in range(2)]
+    saved = (first.get_params(), *first.get_optimizer_state())
+    first.close()
+    assert saved[3] == 2
+    resumed = BD.GPT2(_bd_config(TINY, B, k, BD.GPT2_BF16), seed=77)   # other init: all of it is overwritten
+    resumed.set_params(saved[0])
+    resumed.set_optimizer_state(saved[1], saved[2], saved[3])
+    log_b.append(train(resumed, 2))
+    final_b = resumed.get_params()
+    m_b, v_b, t_b = resumed.get_optimizer_state()
+    resumed.close()
+
+    assert log_a == log_b
+    assert np.array_equal(final_a, final_b)
+    assert np.array_equal(m_a, m_b) and np.array_equal(v_a, v_b) and t_a == t_b == 3
+
+
 def test_graph_replay_matches_direct_launches():
     """Two optimizer steps of three micro-steps each: with graphs on, the first call of a
     shape runs directly, the second is captured and the rest replay the graph.  Every loss
