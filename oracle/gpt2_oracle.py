@@ -254,6 +254,29 @@ def argmax_lowest(logits):
     return torch.where(logits == m, idx, logits.shape[-1]).min(dim=-1).values.to(torch.int32)
 
 
+def sample_top_k(logits_row, k: int, u: float):
+    """Next-token sampling from one row of logits ([L9] "28:07 – 41:44 Loading the weights
+    and generating text": softmax, keep the 50 most probable tokens, renormalise, draw one;
+    "3:22:33 – 3:28:16 Validation loss and sampling during training": the draw uses its own
+    seeded generator).  READINGS: the kept tokens are the k largest logits, ties to the
+    lower index, in descending order (the top-k of the softmax is the top-k of the logits);
+    the draw is the inverse CDF of the renormalised probabilities in that order at the
+    uniform u in [0, 1): the first j whose cumulative probability exceeds u.
+    Returns (token, kept token ids in order)."""
+    z = [float(v) for v in logits_row]
+    k = min(k, len(z))
+    order = sorted(range(len(z)), key=lambda i: (-z[i], i))[:k]
+    w = [math.exp(z[i] - z[order[0]]) for i in order]
+    total = math.fsum(w)
+    target = u * total
+    cum = 0.0
+    for j, wj in enumerate(w):
+        cum += wj
+        if cum > target:
+            return order[j], order
+    return order[-1], order
+
+
 # ----------------------------------------------------------------------------- model
 def encoder_forward(wte, wpe, tokens):
     """x0[b, t] = wte[tokens[b, t]] + wpe[t] ([L9] "Code you'll write", forward pass:

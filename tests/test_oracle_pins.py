@@ -372,6 +372,42 @@ def test_encoder_forward_is_adjoint_of_backward():
             assert onehot[b, t].tolist() == row
 
 
+def test_sample_top_k_with_k_one_is_the_argmax():
+    g = torch.Generator().manual_seed(31)
+    z = torch.randn(3, 40, generator=g, dtype=D)
+    z[1, 7] = z[1, 30] = z[1].max() + 1.0          # a tie: the lower index wins
+    amax = O.argmax_lowest(z)
+    for r in range(3):
+        for u in (0.0, 0.37, 0.999999):
+            tok, kept = O.sample_top_k(z[r], 1, u)
+            assert tok == int(amax[r]) and kept == [tok]
+    assert O.sample_top_k(z[1], 1, 0.5)[0] == 7
+
+
+def test_sample_top_k_frequencies_follow_the_renormalised_softmax():
+    """Over a uniform grid of u, each kept token is drawn with the probability
+    exp(z_i) / sum over the kept exp(z_j); tokens outside the top k never appear."""
+    z = torch.tensor([0.3, 2.0, -1.0, 1.1, 2.0, 0.9, -3.0], dtype=D)
+    k = 4
+    kept_want = [1, 4, 3, 5]                        # 2.0 (index 1), 2.0 (index 4), 1.1, 0.9
+    n = 20000
+    counts = {}
+    for i in range(n):
+        tok, kept = O.sample_top_k(z, k, (i + 0.5) / n)
+        assert kept == kept_want
+        counts[tok] = counts.get(tok, 0) + 1
+    assert set(counts) == set(kept_want)
+    e = torch.exp(z[kept_want])
+    p = e / e.sum()
+    for j, t in enumerate(kept_want):
+        assert abs(counts[t] / n - float(p[j])) <= 1.0 / n
+    # k >= V keeps every token: the full softmax
+    tok_all = [O.sample_top_k(z, 100, (i + 0.5) / n)[0] for i in range(0, n, 10)]
+    full = torch.softmax(z, 0)
+    for t in range(7):
+        assert abs(tok_all.count(t) / len(tok_all) - float(full[t])) <= 10.0 / n + 1e-12
+
+
 def test_grad_accumulation_equals_one_big_batch():
     """[L9] 2:34:49 – 2:46:43: k micro-steps with loss/k give the full-batch gradient."""
     cfg = SMALL
