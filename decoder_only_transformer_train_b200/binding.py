@@ -56,6 +56,7 @@ _PROTOS = {
     "gpt2_get_lse": (_i, [_vp, _vp]),
     "gpt2_get_loss": (_i, [_vp, _fp]),
     "gpt2_synchronize": (_i, [_vp]),
+    "gpt2_sample_top_k": (_i, [_vp, _vp, _vp, _i, _i, _vp, _vp]),
     "gpt2_last_error": (ctypes.c_char_p, [_vp]),
     "gpt2op_gemm_bf16": (_i, [_vp, _i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _f, _vp, _i64]),
     "gpt2op_gemm_bf16_fused": (_i, [_vp, _i, _i, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, _i64, _i, _vp, ctypes.c_float,
@@ -67,6 +68,7 @@ _PROTOS = {
     "gpt2op_embedding_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i]),
     "gpt2op_embedding_bwd_ws_bytes": (_i64, [_i, _i]),
     "gpt2op_embedding_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp]),
+    "gpt2op_sample_top_k": (_i, [_vp, _i, _vp, _i64, _i, _vp, _vp, _i, _i, _i, _vp, _vp]),
     "gpt2op_classifier_aux_floats": (_i64, [_i, _i]),
     "gpt2op_classifier_fwd_bwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "gpt2op_device_error": (_i, []),
@@ -229,6 +231,12 @@ class GPT2:
         v = np.ascontiguousarray(v, dtype=np.float32)
         _check(lib().gpt2_set_optimizer_state(self._h, m.ctypes.data, v.ctypes.data, t), self._h)
 
+    def sample_top_k(self, rows, u, k: int, out, out_topk=None):
+        """Top-k sampling from the last forward's logits: rows (int32), u (f32) and out
+        (int32, and out_topk [n, min(k, vocab)]) are device tensors; asynchronous."""
+        _check(lib().gpt2_sample_top_k(self._h, _ptr(rows), _ptr(u), int(rows.numel()), k, _ptr(out),
+                                       _ptr(out_topk)), self._h)
+
     def get_argmax(self, n: int) -> np.ndarray:
         out = np.empty(n, dtype=np.int32)
         _check(lib().gpt2_get_argmax(self._h, out.ctypes.data), self._h)
@@ -318,6 +326,15 @@ def embedding_bwd(tokens, dx0, dwte, dwpe, B, T, C, V, ws, stream=None):
     holds the ascending sort keys token << 15 | position in its first B*T uint32 words."""
     _check(lib().gpt2op_embedding_bwd(_stream(stream), _ptr(tokens), _ptr(dx0), _ptr(dwte), _ptr(dwpe), B, T, C, V,
                                       _ptr(ws)))
+
+
+SAMPLE_MAX_K = 1024
+
+
+def sample_top_k(logits, ld, n_rows, rows, u, n, V, k, precision, out, out_topk=None, stream=None):
+    """gpt2op_sample_top_k on caller logits [n_rows, ld] (bf16 or f32 by precision)."""
+    _check(lib().gpt2op_sample_top_k(_stream(stream), precision, _ptr(logits), ld, n_rows, _ptr(rows), _ptr(u), n, V,
+                                     k, _ptr(out), _ptr(out_topk)))
 
 
 def classifier_aux_floats(N: int, V: int) -> int:

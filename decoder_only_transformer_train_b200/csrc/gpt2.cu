@@ -130,6 +130,7 @@ struct gpt2_ctx {
   std::vector<GraphEntry> graphs;
   bool use_graphs = true;
   bool have_targets = false;
+  bool have_logits = false;   // the last forward's logits are intact (no backward since)
 
   // per-kernel-class CUDA-event profiling (gpt2_profile_start / gpt2_profile_stop)
   bool prof_on = false;
@@ -247,6 +248,7 @@ int check_device(gpt2_ctx* c) {
     case DEVERR_TOKEN: return fail(c, GPT2_ERR_TOKEN, "input token id outside [0, vocab_size)");
     case DEVERR_TARGET: return fail(c, GPT2_ERR_TARGET, "target outside [0, vocab_size) and not -1");
     case DEVERR_TIMEOUT: return fail(c, GPT2_ERR_TIMEOUT, "a bounded device wait timed out");
+    case DEVERR_ROW: return fail(c, GPT2_ERR_ARG, "a sampled row outside the last forward's B*T rows");
     default: return fail(c, GPT2_ERR_CUDA, "device reported an internal error");
   }
 }
@@ -773,10 +775,12 @@ static int forward_common(gpt2_ctx* c, const int32_t* tokens, const int32_t* tar
   c->lastB = B;
   c->lastT = T;
   c->have_targets = false;
+  c->have_logits = false;
   const bool with_t = targets != nullptr;
   int rc = run_graphed(c, with_t ? 1 : 0, B, T, [&] { return forward_impl(c, B, T, with_t); });
   if (rc) return rc;
   c->have_targets = with_t;
+  c->have_logits = true;
   if (loss_out) {
     rc = check_device(c);
     if (rc) return rc;
@@ -800,7 +804,19 @@ int gpt2_backward(gpt2_ctx* c) {
   if (!c->have_targets) return fail(c, GPT2_ERR_STATE, "backward needs a preceding forward with targets");
   int rc = run_graphed(c, 2, c->lastB, c->lastT, [&] { return backward_impl(c); });
   c->have_targets = false;   // the logits buffer now holds their gradient
+  c->have_logits = false;
   return rc;
+}
+
+int gpt2_sample_top_k(gpt2_ctx* c, const int32_t* rows, const float* u, int n, int k, int32_t* out,
+                      int32_t* out_topk) {
+  if (c == nullptr || rows == nullptr || u == nullptr || out == nullptr) return fail(c, GPT2_ERR_ARG, "null argument");
+  if (!c->have_logits) return fail(c, GPT2_ERR_STATE, "sampling needs the logits of a forward with no backward since");
+  if (n <= 0 || k <= 0 || k > GPT2_SAMPLE_MAX_K) return fail(c, GPT2_ERR_SHAPE, "n <= 0 or k outside [1, 1024]");
+  const int rc = launch_topk_sample(c->stream, c->bf16, c->logits, c->ldl, c->lastB * c->lastT, rows, u, n,
+                                    c->cfg.vocab_size, k, out, out_topk);
+  if (rc == -4) return fail(c, GPT2_ERR_SHAPE, "sampling shape");
+  return rc ? fail(c, GPT2_ERR_CUDA, "sampling launch") : GPT2_OK;
 }
 
 int gpt2_zero_grad(gpt2_ctx* c) {

@@ -679,6 +679,101 @@ __global__ void __launch_bounds__(256) enc_fixup_kernel(const uint32_t* __restri
   *o = w;
 }
 
+// ================================================================ top-k sampling
+// Next-token sampling from rows of logits (L9, "28:07 – 41:44 Loading the weights and
+// generating text"): the k largest logits, ties to the lower id, in descending order, their
+// softmax, and the inverse CDF at the caller's uniform.  One CTA per sampled row.  Round r
+// takes the block-wide maximum of the composite keys (order-preserving logit bits, then the
+// complemented id) below round r-1's winner, so the kept list comes out already ordered,
+// with nothing marked and nothing sorted.  Not on the training step's path.
+constexpr int TOPK_THREADS = 1024;
+constexpr int TOPK_MAX = 1024;
+
+// a < b  <=>  topk_order_bits(a) < topk_order_bits(b) for every non-NaN float
+__device__ __forceinline__ uint32_t topk_order_bits(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float topk_load(const float* p) { return __ldg(p); }
+__device__ __forceinline__ float topk_load(const bf16* p) { return __bfloat162float(*p); }
+
+template <typename T>
+__global__ void __launch_bounds__(TOPK_THREADS) topk_sample_kernel(const T* __restrict__ logits, long long ld,
+                                                                   int n_rows, const int* __restrict__ rows,
+                                                                   const float* __restrict__ u, int V, int k,
+                                                                   int* __restrict__ out, int* __restrict__ out_topk) {
+  __shared__ unsigned long long warp_best[TOPK_THREADS / 32];
+  __shared__ unsigned long long best;
+  __shared__ int sel[TOPK_MAX];
+  __shared__ float selv[TOPK_MAX];
+  const int s = blockIdx.x;
+  const int row = rows[s];
+  if (row < 0 || row >= n_rows) {   // the same for the whole block
+    if (threadIdx.x == 0) {
+      out[s] = -1;
+      raise_device_error(DEVERR_ROW);
+    }
+    if (out_topk)
+      for (int j = threadIdx.x; j < k; j += TOPK_THREADS) out_topk[(long long)s * k + j] = -1;
+    return;
+  }
+  const T* z = logits + (long long)row * ld;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  unsigned long long limit = ~0ull;
+  for (int r = 0; r < k; ++r) {
+    unsigned long long mine = 0;
+    for (int i = threadIdx.x; i < V; i += TOPK_THREADS) {
+      const unsigned long long key = (static_cast<unsigned long long>(topk_order_bits(topk_load(z + i))) << 32) |
+                                     static_cast<unsigned long long>(0xFFFFFFFFu - static_cast<uint32_t>(i));
+      if ((r == 0 || key < limit) && key > mine) mine = key;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, mine, o);
+      mine = other > mine ? other : mine;
+    }
+    if (lane == 0) warp_best[warp] = mine;
+    __syncthreads();
+    if (warp == 0) {
+      mine = warp_best[lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, mine, o);
+        mine = other > mine ? other : mine;
+      }
+      if (lane == 0) {
+        best = mine;
+        const int id = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(mine & 0xFFFFFFFFull));
+        sel[r] = id;
+        selv[r] = topk_load(z + id);
+      }
+    }
+    __syncthreads();
+    limit = best;
+  }
+  if (out_topk)
+    for (int j = threadIdx.x; j < k; j += TOPK_THREADS) out_topk[(long long)s * k + j] = sel[j];
+  if (threadIdx.x == 0) {
+    // softmax over the kept logits relative to the largest, summed in the kept order
+    float total = 0.f;
+    for (int j = 0; j < k; ++j) total += expf(selv[j] - selv[0]);
+    float uu = u[s];
+    uu = (uu >= 0.f) ? uu : 0.f;
+    uu = (uu < 1.f) ? uu : 0.99999994f;
+    const float target = uu * total;
+    float cum = 0.f;
+    int pick = sel[k - 1];
+    for (int j = 0; j < k; ++j) {
+      cum += expf(selv[j] - selv[0]);
+      if (cum > target) {
+        pick = sel[j];
+        break;
+      }
+    }
+    out[s] = pick;
+  }
+}
+
 // dwpe[t] += sum over b in order of dx0[b, t]: four channels per thread, eight rows in flight.
 __global__ void __launch_bounds__(256) dwpe_kernel(const float4* __restrict__ dx0, float4* __restrict__ dwpe, int B,
                                                    int TC4) {
@@ -1165,6 +1260,20 @@ int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float*
   dwpe_kernel<<<grid_for(tc4, 256), 256, 0, st>>>(reinterpret_cast<const float4*>(dx0),
                                                   reinterpret_cast<float4*>(dwpe), B, tc4);
   note_kernel_launches(4);
+  return ok();
+}
+
+int launch_topk_sample(cudaStream_t st, bool is_bf16, const void* logits, long long ld, int n_rows, const int* rows,
+                       const float* u, int n, int V, int k, int* out, int* out_topk) {
+  if (n <= 0 || n_rows <= 0 || V <= 0 || k <= 0 || k > TOPK_MAX || ld < V) return -4;
+  if (k > V) k = V;
+  if (is_bf16)
+    topk_sample_kernel<bf16><<<n, TOPK_THREADS, 0, st>>>(static_cast<const bf16*>(logits), ld, n_rows, rows, u, V, k,
+                                                         out, out_topk);
+  else
+    topk_sample_kernel<float><<<n, TOPK_THREADS, 0, st>>>(static_cast<const float*>(logits), ld, n_rows, rows, u, V,
+                                                          k, out, out_topk);
+  note_kernel_launches(1);
   return ok();
 }
 

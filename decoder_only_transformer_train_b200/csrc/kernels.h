@@ -34,6 +34,8 @@ int launch_ce_dz(cudaStream_t st, bool bf16, void* logits, long long ld, const f
 int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float* dwte, float* dwpe, int B, int T,
                        int C, uint32_t* sorted_keys, float* chunk_part, int V);
 size_t encoder_bwd_part_floats(int N, int C);
+int launch_topk_sample(cudaStream_t st, bool is_bf16, const void* logits, long long ld, int n_rows, const int* rows,
+                       const float* u, int n, int V, int k, int* out, int* out_topk);
 int launch_global_norm(cudaStream_t st, const float* g, long long n, double* part, int nparts, float clip,
                        float* out2);
 int launch_adamw(cudaStream_t st, float* p, const float* g, float* m, float* v, uint16_t* shadow,

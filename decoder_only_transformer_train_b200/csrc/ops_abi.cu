@@ -114,6 +114,16 @@ int gpt2op_embedding_bwd(void* stream, const int32_t* tokens, const float* dx0, 
   return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
 }
 
+int gpt2op_sample_top_k(void* stream, int precision, const void* logits, int64_t ld, int n_rows,
+                        const int32_t* rows, const float* u, int n, int V, int k, int32_t* out, int32_t* out_topk) {
+  if (!logits || !rows || !u || !out) return GPT2_ERR_ARG;
+  if (precision != GPT2_FP32 && precision != GPT2_BF16) return GPT2_ERR_ARG;
+  if (n <= 0 || n_rows <= 0 || V <= 0 || k <= 0 || k > GPT2_SAMPLE_MAX_K || ld < V) return GPT2_ERR_SHAPE;
+  const int rc = launch_topk_sample(reinterpret_cast<cudaStream_t>(stream), precision == GPT2_BF16, logits, ld,
+                                    n_rows, rows, u, n, V, k, out, out_topk);
+  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+}
+
 int64_t gpt2op_classifier_aux_floats(int N, int V) {
   const int ntiles = gemm_tc_ce_tiles(V);
   // partials (4 floats each), zt, loss_row, and 8 scalars
@@ -156,6 +166,7 @@ int gpt2op_device_error(void) {
     case DEVERR_TOKEN: return GPT2_ERR_TOKEN;
     case DEVERR_TARGET: return GPT2_ERR_TARGET;
     case DEVERR_TIMEOUT: return GPT2_ERR_TIMEOUT;
+    case DEVERR_ROW: return GPT2_ERR_ARG;
     default: return GPT2_ERR_CUDA;
   }
 }

@@ -128,6 +128,26 @@ int gpt2_adamw_step(gpt2_ctx* ctx, float lr, float beta1, float beta2, float eps
  * r = (it - warmup_steps) / (max_steps - warmup_steps).  Host function, double math. */
 double gpt2_lr_cosine(int64_t it, double max_lr, int64_t warmup_steps, int64_t max_steps, double min_ratio);
 
+/* Next-token sampling ("Karpathy's Zero to Hero, Lecture 9: Reproduce GPT-2 (124M)" notes,
+ * "28:07 – 41:44 Loading the weights and generating text": the last position's logits,
+ * softmax, the 50 most probable tokens kept and renormalised, one token drawn; "3:22:33 –
+ * 3:28:16 Validation loss and sampling during training": the draw has its own seeded
+ * generator, so the uniforms are the caller's).  For each i < n, row rows[i] of the last
+ * forward's logits (token positions b*T + t, columns [0, vocab_size)): the k largest
+ * logits, ties to the lower id, in descending order; their softmax; out[i] = the first of
+ * them whose cumulative probability exceeds u[i] (u[i] clamped into [0, 1)).  If out_topk
+ * is non-NULL it receives the n x min(k, vocab_size) kept ids in that order.
+ * rows (int32 [n]), u (f32 [n]), out, out_topk: DEVICE buffers, caller-owned; the call is
+ * asynchronous on the context stream.  A forward without targets is the inference and
+ * validation path (validation loss: a forward with targets and no backward).
+ * Errors: GPT2_ERR_STATE unless the last call that touched the logits was a forward (a
+ * backward overwrites them with their gradient); GPT2_ERR_SHAPE for n <= 0 or k outside
+ * [1, GPT2_SAMPLE_MAX_K].  A row outside [0, B*T) of the last forward gives out[i] = -1 and
+ * GPT2_ERR_ARG at the next synchronising call. */
+#define GPT2_SAMPLE_MAX_K 1024
+int gpt2_sample_top_k(gpt2_ctx* ctx, const int32_t* rows, const float* u, int n, int k, int32_t* out,
+                      int32_t* out_topk);
+
 /* Number of CUDA kernels this library has launched in this process so far. */
 int64_t gpt2_kernel_launches(void);
 
@@ -237,6 +257,14 @@ int gpt2op_embedding_fwd(void* stream, const int32_t* tokens, const float* wte, 
 int64_t gpt2op_embedding_bwd_ws_bytes(int N, int C);
 int gpt2op_embedding_bwd(void* stream, const int32_t* tokens, const float* dx0, float* dwte, float* dwpe, int B,
                          int T, int C, int V, void* ws);
+
+/* The sampling of gpt2_sample_top_k on caller logits: DEVICE logits [n_rows, ld] (bf16 or
+ * f32 by precision), columns [0, V) sampled, ld >= V.  Same rows / u / out / out_topk
+ * contract; a row outside [0, n_rows) gives out[i] = -1 and sets the device error word to
+ * GPT2_ERR_ARG (read with gpt2op_device_error).  GPT2_ERR_SHAPE for n, n_rows or V <= 0,
+ * ld < V or k outside [1, GPT2_SAMPLE_MAX_K]; GPT2_ERR_ARG for a null pointer. */
+int gpt2op_sample_top_k(void* stream, int precision, const void* logits, int64_t ld, int n_rows,
+                        const int32_t* rows, const float* u, int n, int V, int k, int32_t* out, int32_t* out_topk);
 
 /* Fused classifier head (lm_head + softmax + cross-entropy), forward and backward, on
  * caller buffers: h bf16 [N, C] (the final LayerNorm output), W bf16 [V, C] (the tied
