@@ -172,10 +172,10 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict_
   }
 }
 
-// Block: 32 columns x 16 row groups.  Row group r sums partial rows r, r+16, r+32, ... in
-// that order (8 loads in flight), then the 16 group sums are added in group order, so the
-// result does not depend on timing.
-constexpr int LNP_GROUPS = 16;
+// Block: 32 columns x 32 row groups.  Row group r sums partial rows r, r+32, r+64, ... in
+// that order (8 loads in flight: one batch for the 2-per-SM partial rows of a B200), then the
+// 32 group sums are added in group order, so the result does not depend on timing.
+constexpr int LNP_GROUPS = 32;
 __global__ void __launch_bounds__(32 * LNP_GROUPS) ln_param_reduce_kernel(const float* __restrict__ part, int nblocks,
                                                                          int C, float* __restrict__ dw,
                                                                          float* __restrict__ db,
@@ -256,21 +256,22 @@ __global__ void __launch_bounds__(1024) colsum_rows_kernel(const T* __restrict__
     for (int i = 0; i < VEC; ++i) part[(long long)blockIdx.x * N + g * VEC + i] = s[i];
   }
 }
-// out[n] += sum_k part[k][n] in a fixed order.  Block: 32 columns x 16 chunk groups; group g
-// adds chunks g, g + 16, ... in order (8 loads in flight), then the 16 group sums are added
-// in group order.
-__global__ void __launch_bounds__(512) colsum_reduce_kernel(const float* __restrict__ part, int nchunks, int N,
-                                                            float* __restrict__ out) {
-  __shared__ float red[16][33];
+// out[n] += sum_k part[k][n] in a fixed order.  Block: 32 columns x 32 chunk groups; group g
+// adds chunks g, g + 32, ... in order (8 loads in flight: one batch for up to 256 chunks),
+// then the 32 group sums are added in group order.
+constexpr int CSR_GROUPS = 32;
+__global__ void __launch_bounds__(32 * CSR_GROUPS) colsum_reduce_kernel(const float* __restrict__ part, int nchunks,
+                                                                       int N, float* __restrict__ out) {
+  __shared__ float red[CSR_GROUPS][33];
   const int lane = threadIdx.x & 31, gr = threadIdx.x >> 5;
   const int n = blockIdx.x * 32 + lane;
   float s = 0.f;
   if (n < N) {
-    for (int k0 = gr; k0 < nchunks; k0 += 16 * 8) {
+    for (int k0 = gr; k0 < nchunks; k0 += CSR_GROUPS * 8) {
       float v[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int k = k0 + 16 * i;
+        const int k = k0 + CSR_GROUPS * i;
         v[i] = (k < nchunks) ? part[(long long)k * N + n] : 0.f;
       }
 #pragma unroll
@@ -282,7 +283,7 @@ __global__ void __launch_bounds__(512) colsum_reduce_kernel(const float* __restr
   if (gr == 0 && n < N) {
     float t = 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) t += red[i][lane];
+    for (int i = 0; i < CSR_GROUPS; ++i) t += red[i][lane];
     out[n] += t;
   }
 }
@@ -1170,7 +1171,7 @@ int launch_colsum(cudaStream_t st, bool is_bf16, const void* x, long long ldx, i
   if (threads > 1024) threads = 1024;
   if (is_bf16) colsum_rows_kernel<bf16><<<used, threads, 0, st>>>(reinterpret_cast<const bf16*>(x), ldx, M, N, rpc, part);
   else colsum_rows_kernel<float><<<used, threads, 0, st>>>(reinterpret_cast<const float*>(x), ldx, M, N, rpc, part);
-  colsum_reduce_kernel<<<cdiv(N, 32), 512, 0, st>>>(part, used, N, out);
+  colsum_reduce_kernel<<<cdiv(N, 32), 32 * CSR_GROUPS, 0, st>>>(part, used, N, out);
   note_kernel_launches(2);
   return ok();
 }
