@@ -1124,6 +1124,9 @@ int ln_bwd_dispatch(cudaStream_t st, const float* dy, const float* x, const floa
 int launch_encoder_fwd(cudaStream_t st, const int* tok, const float* wte, const float* wpe, float* x, int N, int T,
                        int C, int V) {
   if (N <= 0 || T <= 0 || C <= 0 || C % 4) return -4;
+  // 16-byte accesses: the tables and the output must be 16-byte aligned
+  if ((reinterpret_cast<uintptr_t>(wte) | reinterpret_cast<uintptr_t>(wpe) | reinterpret_cast<uintptr_t>(x)) % 16)
+    return -1;
   const int c4 = C / 4;
   const int threads = c4 <= 256 ? (c4 + 31) / 32 * 32 : 256;
   dim3 grid(grid_for(cdiv(N, 4), 1, 148 * 8), cdiv(c4, threads));
@@ -1238,6 +1241,10 @@ int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float*
   if (B <= 0 || T <= 0 || Nll > (1 << ENC_POS_BITS) || V <= 0 || V > (1 << (32 - ENC_POS_BITS)) || C <= 0 ||
       C % 4)
     return -4;
+  // 16-byte accesses to dx0, the gradients and the chunk partials
+  if ((reinterpret_cast<uintptr_t>(dx0) | reinterpret_cast<uintptr_t>(dwte) | reinterpret_cast<uintptr_t>(dwpe) |
+       reinterpret_cast<uintptr_t>(chunk_part)) % 16)
+    return -1;
   const int N = (int)Nll;
   int P = ENC_SORT_THREADS;
   while (P < N) P <<= 1;

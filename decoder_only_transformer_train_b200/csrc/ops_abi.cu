@@ -93,7 +93,7 @@ int gpt2op_embedding_fwd(void* stream, const int32_t* tokens, const float* wte, 
   if (!tokens || !wte || !wpe || !x) return GPT2_ERR_ARG;
   if (B <= 0 || T <= 0 || C <= 0 || V <= 0 || C % 4 || (long long)B * T > INT32_MAX) return GPT2_ERR_SHAPE;
   const int rc = launch_encoder_fwd(reinterpret_cast<cudaStream_t>(stream), tokens, wte, wpe, x, B * T, T, C, V);
-  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA));
 }
 
 static int64_t embedding_keys_bytes(int N) { return ((int64_t)N * 4 + 255) / 256 * 256; }
@@ -111,7 +111,7 @@ int gpt2op_embedding_bwd(void* stream, const int32_t* tokens, const float* dx0, 
   const int rc = launch_encoder_bwd(reinterpret_cast<cudaStream_t>(stream), tokens, dx0, dwte, dwpe, B, T, C,
                                     reinterpret_cast<uint32_t*>(w),
                                     reinterpret_cast<float*>(w + embedding_keys_bytes(B * T)), V);
-  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA));
 }
 
 int gpt2op_sample_top_k(void* stream, int precision, const void* logits, int64_t ld, int n_rows,

@@ -250,7 +250,8 @@ int gpt2op_layernorm_fwd(void* stream, int precision, const float* x, const floa
  * are deterministic (no atomics; a fixed order that depends only on the ids).  ws is
  * device scratch of gpt2op_embedding_bwd_ws_bytes(B*T, C) bytes, 256-byte aligned; after
  * the call its first B*T uint32 words hold the sort keys token << 15 | position in
- * ascending order.  Both: GPT2_ERR_ARG for a null pointer; GPT2_ERR_SHAPE unless B, T,
+ * ascending order.  The f32 tables, x, dx0, dwte, dwpe and ws must be 16-byte aligned.
+ * Both: GPT2_ERR_ARG for a null or misaligned pointer; GPT2_ERR_SHAPE unless B, T,
  * C, V > 0, C % 4 == 0, and for the backward B*T <= 32768 and V <= 131072. */
 int gpt2op_embedding_fwd(void* stream, const int32_t* tokens, const float* wte, const float* wpe, float* x, int B,
                          int T, int C, int V);

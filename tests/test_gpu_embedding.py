@@ -132,7 +132,7 @@ def test_embedding_fwd_reports_bad_ids_and_writes_zero_rows():
 def test_embedding_entry_points_reject_bad_shapes_before_any_cuda_call():
     lib = BD.lib()
     buf = np.zeros(64, dtype=np.float32)
-    p = buf.ctypes.data
+    p = (buf.ctypes.data + 15) // 16 * 16
     err_shape, err_arg = -4, -1
     assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 32, 1025, 64, V, p) == err_shape   # > 32768 positions
     assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 2, 8, 66, V, p) == err_shape       # C % 4
@@ -141,3 +141,9 @@ def test_embedding_entry_points_reject_bad_shapes_before_any_cuda_call():
     assert lib.gpt2op_embedding_fwd(None, p, p, p, p, 2, 8, 62, V) == err_shape
     assert lib.gpt2op_embedding_fwd(None, None, p, p, p, 2, 8, 64, V) == err_arg
     assert BD.embedding_bwd_ws_bytes(16384, 768) == 16384 * 4 + 512 * 2 * 768 * 4
+    # 16-byte accesses: a misaligned table, output or gradient is refused before any launch
+    q = p + 4
+    assert lib.gpt2op_embedding_fwd(None, p, q, p, p, 2, 8, 64, V) == err_arg
+    assert lib.gpt2op_embedding_fwd(None, p, p, p, q, 2, 8, 64, V) == err_arg
+    assert lib.gpt2op_embedding_bwd(None, p, q, p, p, 2, 8, 64, V, p) == err_arg
+    assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 2, 8, 64, V, q) == err_arg
