@@ -457,7 +457,8 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
   const int C = H * HD;
   PFN_encode fn = encode_fn();
   if (fn == nullptr) return -3;
-  if ((reinterpret_cast<uintptr_t>(qkv) & 15) != 0) return -1;
+  // TMA reads qkv; the epilogue writes out with 16-byte stores
+  if (((reinterpret_cast<uintptr_t>(qkv) | reinterpret_cast<uintptr_t>(out)) & 15) != 0) return -1;
   CUtensorMap tm;
   cuuint64_t dims[2] = {(cuuint64_t)(3 * C), (cuuint64_t)B * T};
   cuuint64_t strides[1] = {(cuuint64_t)(3 * C) * 2};
@@ -870,6 +871,7 @@ int encode_rows64(CUtensorMap* tm, const void* base, int cols, long long rows) {
 int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const float* lse, const float* Dbuf,
                        void* dqkv, int B, int T, int H, int hd) {
   if (hd != HD) return -4;
+  if ((reinterpret_cast<uintptr_t>(dqkv) & 15) != 0) return -1;   // 16-byte stores of dQ, dK, dV
   const int C = H * HD;
   CUtensorMap tq, td;
   int rc = encode_rows64(&tq, qkv, 3 * C, (long long)B * T);

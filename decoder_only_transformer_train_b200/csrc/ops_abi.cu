@@ -28,6 +28,7 @@ int gpt2op_gemm_bf16(void* stream, int M, int N, int K, const void* A, int64_t l
     case 2: kind = EPI_ACCUM_F32; break;
     default: return GPT2_ERR_ARG;
   }
+  if (reinterpret_cast<uintptr_t>(bias) % 16) return GPT2_ERR_ARG;   // 16-byte bias reads in the epilogue
   EpiParams e = epi_make(kind, C, ldc);
   e.bias = bias;
   e.alpha = alpha;
@@ -52,6 +53,10 @@ int gpt2op_gemm_bf16_fused(void* stream, int M, int N, int K, const void* A, int
   if ((kind == EPI_RESID_F32 || kind == EPI_GELU_BWD) && aux == nullptr) return GPT2_ERR_ARG;
   if (kind == EPI_GELU_FWD && aux_out == nullptr) return GPT2_ERR_ARG;
   if ((aux && ld_aux % 8) || (aux_out && ld_aux_out % 8)) return GPT2_ERR_ARG;
+  // the epilogue reads bias and aux and writes aux_out with 16-byte accesses
+  if ((reinterpret_cast<uintptr_t>(bias) | reinterpret_cast<uintptr_t>(aux) | reinterpret_cast<uintptr_t>(aux_out)) %
+      16)
+    return GPT2_ERR_ARG;
   EpiParams e = epi_make(kind, C, ldc);
   e.bias = (kind == EPI_GELU_BWD) ? nullptr : bias;
   e.alpha = alpha;
@@ -69,7 +74,7 @@ int gpt2op_attention_fwd(void* stream, int precision, const void* qkv, void* out
   if (!qkv || !out || !lse) return GPT2_ERR_ARG;
   int rc = launch_attn_fwd(reinterpret_cast<cudaStream_t>(stream), precision == GPT2_BF16, qkv, out, lse, B, T, H,
                            head_dim);
-  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA));
 }
 
 int gpt2op_attention_bwd(void* stream, int precision, const void* qkv, const void* out, const void* dout,
@@ -77,7 +82,7 @@ int gpt2op_attention_bwd(void* stream, int precision, const void* qkv, const voi
   if (!qkv || !out || !dout || !lse || !Dbuf || !dqkv) return GPT2_ERR_ARG;
   int rc = launch_attn_bwd(reinterpret_cast<cudaStream_t>(stream), precision == GPT2_BF16, qkv, out, dout, lse, Dbuf,
                            dqkv, B, T, H, head_dim);
-  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+  return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA));
 }
 
 int gpt2op_layernorm_fwd(void* stream, int precision, const float* x, const float* w, const float* b, void* y,

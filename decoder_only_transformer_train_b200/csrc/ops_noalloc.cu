@@ -61,5 +61,5 @@ extern "C" int gpt2op_attention_bwd_noalloc(void* stream, int precision, const v
   if (rc != GPT2_OK) return rc;
   const int lrc = launch_attn_bwd(reinterpret_cast<cudaStream_t>(stream), precision == GPT2_BF16, qkv, out, dout,
                                   lse, Dbuf, dqkv, B, T, H, head_dim);
-  return lrc == 0 ? GPT2_OK : (lrc == -4 ? GPT2_ERR_SHAPE : GPT2_ERR_CUDA);
+  return lrc == 0 ? GPT2_OK : (lrc == -4 ? GPT2_ERR_SHAPE : (lrc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA));
 }

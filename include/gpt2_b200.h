@@ -201,8 +201,9 @@ int gpt2op_gemm_bf16(void* stream, int M, int N, int K, const void* A, int64_t l
  * bias (f32 [N]) may be NULL for 3 and 4 and is ignored by 5.  aux / aux_out are device
  * buffers the caller owns, 16-byte aligned, with ld_aux / ld_aux_out multiples of 8
  * elements; aux may equal C for epilogue 3 (an in-place residual update).  GELU uses the
- * hardware tanh approximation (results rounded to bf16).  GPT2_ERR_ARG for a null operand or
- * an unknown epilogue; GPT2_ERR_CUDA if a launch or tensor-map encode fails. */
+ * hardware tanh approximation (results rounded to bf16).  GPT2_ERR_ARG for a null operand,
+ * an unknown epilogue or a bias / aux / aux_out that is not 16-byte aligned; GPT2_ERR_CUDA if
+ * a launch or tensor-map encode fails. */
 int gpt2op_gemm_bf16_fused(void* stream, int M, int N, int K, const void* A, int64_t lda, int a_mn_major,
                            const void* B, int64_t ldb, int b_mn_major, void* C, int64_t ldc, int epilogue,
                            const float* bias, float alpha, const void* aux, int64_t ld_aux, void* aux_out,
@@ -212,7 +213,9 @@ int gpt2op_gemm_bf16_fused(void* stream, int M, int N, int K, const void* A, int
  * out [B*T, C], lse [B, H, T] float.  precision selects fp32 or bf16 qkv/out. */
 int gpt2op_attention_fwd(void* stream, int precision, const void* qkv, void* out, float* lse, int B, int T, int H,
                          int head_dim);
-/* Its backward: dqkv [B*T, 3C] from dout [B*T, C]; Dbuf float [B, H, T] is scratch. */
+/* Its backward: dqkv [B*T, 3C] from dout [B*T, C]; Dbuf float [B, H, T] is scratch.
+ * Both: the bf16 tensor-core path (head_dim 64) needs qkv, out, dout and dqkv 16-byte
+ * aligned and returns GPT2_ERR_ARG otherwise; GPT2_ERR_SHAPE for an unsupported head_dim. */
 int gpt2op_attention_bwd(void* stream, int precision, const void* qkv, const void* out, const void* dout,
                          const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int head_dim);
 

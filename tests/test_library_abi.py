@@ -74,6 +74,21 @@ def test_no_host_api_rejects_bad_config_without_gpu(libpath):
     assert lib.gpt2_create(None, 1, ctypes.byref(h)) == -1
 
 
+def test_gemm_entry_points_refuse_misaligned_epilogue_operands_without_gpu(libpath):
+    """The GEMM epilogues read bias and aux and write aux_out with 16-byte accesses: a
+    pointer off a 16-byte boundary is refused (GPT2_ERR_ARG) before any CUDA call."""
+    import numpy as np
+    from decoder_only_transformer_train_b200 import binding
+    lib = binding.load(libpath)
+    buf = np.zeros(256, dtype=np.float32)
+    p = (buf.ctypes.data + 15) // 16 * 16
+    q = p + 4
+    assert lib.gpt2op_gemm_bf16(None, 128, 128, 64, p, 64, 0, p, 64, 0, p, 128, 0, q, 1.0, None, 0) == -1
+    for bias, aux, aux_out in ((q, p, p), (p, q, p), (p, p, q)):
+        assert lib.gpt2op_gemm_bf16_fused(None, 128, 128, 64, p, 64, 0, p, 64, 0, p, 128, 4, bias, 1.0, aux, 128,
+                                          aux_out, 128) == -1
+
+
 def test_lr_schedule_host_function_matches_oracle(libpath):
     import oracle as O
     from decoder_only_transformer_train_b200 import binding
