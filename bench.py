@@ -64,6 +64,9 @@ def parse():
     ap.add_argument("--accum", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ddp", action="store_true",
+                    help="data-parallel instead of independent replicas: the ranks split each optimizer step's "
+                         "micro-steps and average the gradients with one all-reduce before AdamW")
     args = ap.parse_args()
     m = MODELS[args.model]
     # a longer context keeps the model's tokens per micro-step (the embedding backward sorts
@@ -159,6 +162,18 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ distributed plumbing
+def ddp_shape(args, world: int):
+    """Data-parallel runs keep the optimizer step's tokens: the accumulation micro-steps are
+    split across the ranks ("2:59:25 – 3:10:20 Synchronizing gradients and losses" of the
+    Lecture 9 notes: each rank's gradients are averaged once, after its last micro-step)."""
+    args.ddp_world = world if (args.ddp and world > 1) else 1
+    if args.ddp_world > 1:
+        if args.accum % world:
+            raise SystemExit(f"--ddp: {args.accum} accumulation micro-steps do not split over {world} ranks")
+        args.accum //= world
+    return args
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -173,13 +188,14 @@ def dist_init(world, backend):
         dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
 
 
-def dist_max(x: float, world: int, device) -> float:
+def dist_max(x: float, world: int, device, op: str = "max") -> float:
+    """The maximum (or, with op="sum", the sum) of x over the ranks."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
     t = torch.tensor([x], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
 
 
@@ -249,12 +265,14 @@ def run_reference(args, world, rank):
 
 
 def workload_config(args):
+    dw = getattr(args, "ddp_world", 1)
+    tokens = args.micro_batch * args.seq * args.accum * dw
+    steps_txt = f"{args.accum} accumulation micro-steps" + (f" on each of {dw} data-parallel ranks" if dw > 1 else "")
     return {"workload": f"{MODELS[args.model]['label']} training step: B={args.micro_batch} x T={args.seq}, "
-                        f"{args.accum} accumulation micro-steps ({args.micro_batch * args.seq * args.accum} tokens), "
-                        f"global-norm clip 1.0, AdamW at lr=get_lr(1000)",
+                        f"{steps_txt} ({tokens} tokens), global-norm clip 1.0, AdamW at lr=get_lr(1000)",
             "micro_batch": args.micro_batch, "seq_len": args.seq, "grad_accum_steps": args.accum,
-            "tokens_per_step": args.micro_batch * args.seq * args.accum,
-            "parallelism": "replicas" if args.gpus > 1 else "single-gpu",
+            "tokens_per_step": tokens,
+            "parallelism": f"ddp{dw}" if dw > 1 else ("replicas" if args.gpus > 1 else "single-gpu"),
             "l2": "inputs larger than L2 (every micro-step moves several GB of parameters and activations)"}
 
 
@@ -282,12 +300,22 @@ def run_ours(args, world, rank, local):
     y_host = run[1:].reshape(k, B, T).astype(np.int32)
     x_dev = torch.from_numpy(x_host).to(device)
     y_dev = torch.from_numpy(y_host).to(device)
+    ddp = getattr(args, "ddp_world", 1) > 1
+    grads = model.grad_tensor() if ddp else None
+
+    def grad_sync():
+        # data-parallel: every rank's gradient (of its loss / k) averaged across ranks, once
+        # per optimizer step, on the model's stream before the clip and AdamW
+        if ddp:
+            import torch.distributed as dist
+            dist.all_reduce(grads, op=dist.ReduceOp.AVG)
 
     def step():
         model.zero_grad()
         for i in range(k):
             model.forward(x_dev[i], y_dev[i], sync_loss=False)
             model.backward()
+        grad_sync()
         model.adamw_step(lr, sync_norm=False)
 
     with torch.cuda.stream(stream):
@@ -316,6 +344,9 @@ def run_ours(args, world, rank, local):
     tokens = world * args.steps * k * B * T
     value = tokens / (ms_max / 1000.0)
     last_loss = model.get_loss()
+    if ddp:   # the logged loss is the mean over the ranks, like the gradients
+        first_loss = dist_max(first_loss / world, world, device, op="sum")
+        last_loss = dist_max(last_loss / world, world, device, op="sum")
 
     # per-kernel-class event timing of one more step (roofline of the dominant kernel)
     with torch.cuda.stream(stream):
@@ -337,6 +368,7 @@ def run_ours(args, world, rank, local):
                 model.forward_host(xp[i], yp[i], sync_loss=False)
                 model.backward()
             model.get_loss()
+            grad_sync()
             return model.adamw_step(lr, sync_norm=True)
 
         barrier(world)
@@ -395,7 +427,8 @@ def run_ours(args, world, rank, local):
         fpt = flop_per_token(args.model, args.seq)
         line = {
             "metric": metric_name(args.model, args.micro_batch, args.seq), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "strong" if ddp else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": workload_config(args),
             "mfu": {"vs_nominal_2250": per_gpu * fpt / (NOMINAL_BF16_TFLOPS * 1e12),
@@ -406,6 +439,7 @@ def run_ours(args, world, rank, local):
             "loss": {"after_warmup": first_loss, "after_timed": last_loss},
         }
         print(json.dumps(line), flush=True)
+    del grads
     model.close()
     if world > 1:
         import torch.distributed as dist
@@ -417,6 +451,7 @@ def main():
     world, rank, local = dist_setup()
     if world > 1:
         args.gpus = world
+    ddp_shape(args, world)
     if args.impl == "reference":
         run_reference(args, world, rank)
         return

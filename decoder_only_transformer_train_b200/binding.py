@@ -45,6 +45,7 @@ _PROTOS = {
     "gpt2_forward_host": (_i, [_vp, _vp, _vp, _i, _i, _fp]),
     "gpt2_backward": (_i, [_vp]),
     "gpt2_zero_grad": (_i, [_vp]),
+    "gpt2_get_grad_buffer": (_i, [_vp, ctypes.POINTER(_vp), ctypes.POINTER(_i64)]),
     "gpt2_adamw_step": (_i, [_vp, _f, _f, _f, _f, _f, _f, _fp]),
     "gpt2_num_params": (_i64, [_vp]),
     "gpt2_get_params": (_i, [_vp, _vp]),
@@ -213,6 +214,20 @@ class GPT2:
         flat = np.ascontiguousarray(flat, dtype=np.float32)
         assert flat.size == self.num_params
         _check(lib().gpt2_set_params(self._h, flat.ctypes.data), self._h)
+
+    def grad_tensor(self):
+        """The library's flat f32 gradient buffer as a torch CUDA tensor that aliases it
+        (zero-copy, through __cuda_array_interface__), e.g. for a data-parallel all-reduce
+        between the last backward of a step and adamw_step.  It must not outlive the model."""
+        import torch
+        p, n = ctypes.c_void_p(), ctypes.c_int64()
+        _check(lib().gpt2_get_grad_buffer(self._h, ctypes.byref(p), ctypes.byref(n)), self._h)
+
+        class _DeviceBuffer:
+            __cuda_array_interface__ = {"shape": (int(n.value),), "typestr": "<f4", "data": (int(p.value), False),
+                                        "version": 3, "strides": None, "stream": None}
+
+        return torch.as_tensor(_DeviceBuffer(), device="cuda")
 
     def get_grads(self) -> np.ndarray:
         out = np.empty(self.num_params, dtype=np.float32)

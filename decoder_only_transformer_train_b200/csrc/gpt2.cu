@@ -819,6 +819,13 @@ int gpt2_sample_top_k(gpt2_ctx* c, const int32_t* rows, const float* u, int n, i
   return rc ? fail(c, GPT2_ERR_CUDA, "sampling launch") : GPT2_OK;
 }
 
+int gpt2_get_grad_buffer(gpt2_ctx* c, float** device_ptr, int64_t* n) {
+  if (c == nullptr || device_ptr == nullptr || n == nullptr) return GPT2_ERR_ARG;
+  *device_ptr = c->grads;
+  *n = (int64_t)c->nparams;
+  return GPT2_OK;
+}
+
 int gpt2_zero_grad(gpt2_ctx* c) {
   if (c == nullptr) return GPT2_ERR_ARG;
   cudaError_t e = cudaMemsetAsync(c->grads, 0, c->nparams * sizeof(float), c->stream);

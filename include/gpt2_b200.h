@@ -109,6 +109,15 @@ int gpt2_forward_host(gpt2_ctx* ctx, const int32_t* tokens, const int32_t* targe
  * preceding forward with targets. */
 int gpt2_backward(gpt2_ctx* ctx);
 
+/* The flat f32 gradient buffer on the device (gpt2_num_params floats in the canonical
+ * order below), owned by the context and valid until gpt2_destroy.  A caller may read or
+ * rewrite it on the context stream between the last gpt2_backward of a step and
+ * gpt2_adamw_step: data-parallel training averages it across ranks there, once per
+ * optimizer step (L9 "2:59:25 – 3:10:20 Synchronizing gradients and losses": the
+ * all-reduce averages every gradient, and only on the last micro-step).  Fills
+ * *device_ptr and *n; GPT2_ERR_ARG for a null argument. */
+int gpt2_get_grad_buffer(gpt2_ctx* ctx, float** device_ptr, int64_t* n);
+
 /* Sets every gradient to zero (optimizer.zero_grad(), L9 "52:38 – 1:06:18"). */
 int gpt2_zero_grad(gpt2_ctx* ctx);
 

@@ -46,3 +46,20 @@ def test_flop_model():
     assert bench.flop_per_token("124m") == 6 * (12 * L * C * C + Vp * C) + 6 * L * 1024 * C == 798031872
     assert bench.flop_per_token("124m", 2048) - bench.flop_per_token("124m", 1024) == 6 * L * 1024 * C
     assert bench.flop_per_token("medium") == 2272002048
+
+
+def test_data_parallel_runs_split_the_micro_steps():
+    a = bench.ddp_shape(_parse("--ddp", "--gpus", "4"), 4)
+    assert (a.accum, a.ddp_world) == (8, 4)
+    cfg = bench.workload_config(a)
+    assert cfg["tokens_per_step"] == 524288 and cfg["parallelism"] == "ddp4"
+    a = bench.ddp_shape(_parse("--gpus", "4"), 4)          # replicas: each rank runs the whole step
+    assert (a.accum, a.ddp_world) == (32, 1)
+    assert bench.workload_config(a)["parallelism"] == "replicas"
+    a = bench.ddp_shape(_parse("--ddp"), 1)                 # one rank: nothing to average
+    assert (a.accum, a.ddp_world) == (32, 1)
+    try:
+        bench.ddp_shape(_parse("--ddp", "--accum", "6"), 4)
+        raise AssertionError("6 micro-steps do not split over 4 ranks")
+    except SystemExit:
+        pass

@@ -194,6 +194,62 @@ def test_resume_from_saved_state_continues_bit_for_bit():
     assert np.array_equal(m_a, m_b) and np.array_equal(v_a, v_b) and t_a == t_b == 3
 
 
+def test_gradient_buffer_view_and_a_one_rank_data_parallel_step():
+    """grad_tensor() aliases the library's gradient buffer (what a data-parallel all-reduce
+    averages in place), and a step whose gradients go through a one-rank NCCL average equals
+    the plain step bit for bit (one rank only: no two kernels here wait on each other)."""
+    import socket
+    import datetime
+    import torch.distributed as dist
+    B, T, k = 2, 64, 2
+    batches = [S.token_batch(31, B, T, TINY.vocab_size, micro_step=i) for i in range(k)]
+
+    def run(average: bool):
+        model = BD.GPT2(_bd_config(TINY, B, k, BD.GPT2_BF16), seed=4)
+        model.set_graphs(False)
+        model.zero_grad()
+        for x, y in batches:
+            model.forward(cuda_i32(x), cuda_i32(y))
+            model.backward()
+        g = model.grad_tensor()
+        model.synchronize()
+        assert g.numel() == model.num_params and g.dtype == torch.float32 and g.is_cuda
+        assert np.array_equal(g.cpu().numpy(), model.get_grads())
+        if average:
+            dist.all_reduce(g, op=dist.ReduceOp.AVG)
+            torch.cuda.synchronize()
+        model.adamw_step(6e-4)
+        out = model.get_params()
+        del g
+        model.close()
+        return out
+
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        plain, averaged = run(False), run(True)
+    finally:
+        dist.destroy_process_group()
+    assert np.array_equal(plain, averaged)
+
+    # writes through the view land in the library's buffer, which the optimizer reads
+    model = BD.GPT2(_bd_config(TINY, B, k, BD.GPT2_BF16), seed=4)
+    model.zero_grad()
+    x, y = batches[0]
+    model.forward(cuda_i32(x), cuda_i32(y))
+    model.backward()
+    g0 = model.get_grads()
+    view = model.grad_tensor()
+    view.mul_(0.5)
+    torch.cuda.synchronize()
+    assert np.array_equal(model.get_grads(), g0 * np.float32(0.5))
+    del view
+    model.close()
+
+
 def test_graph_replay_matches_direct_launches():
     """Two optimizer steps of three micro-steps each: with graphs on, the first call of a
     shape runs directly, the second is captured and the rest replay the graph.  Every loss

@@ -27,10 +27,12 @@ def _rank_main(rank: int, world: int, port: int, out):
     bench.barrier(w)
     # each rank "measures" a different time; every rank must see the slowest
     ms = bench.dist_max(10.0 + 5.0 * r, w, "cpu")
+    # the data-parallel run's logged loss: each rank's share of the mean, summed
+    loss = bench.dist_max((2.0 + 4.0 * r) / w, w, "cpu", op="sum")
     stream = S.zipf_tokens(3 + r, 4097, 50257)          # the bench's per-replica token stream
     bench.barrier(w)
     dist.destroy_process_group()
-    out.put((r, ms, stream[:64].tolist()))
+    out.put((r, ms, stream[:64].tolist(), loss))
 
 
 def test_two_gloo_ranks_share_max_time_and_draw_distinct_streams():
@@ -44,9 +46,10 @@ def test_two_gloo_ranks_share_max_time_and_draw_distinct_streams():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    (r0, ms0, s0), (r1, ms1, s1) = res
+    (r0, ms0, s0, l0), (r1, ms1, s1, l1) = res
     assert (r0, r1) == (0, 1)
     assert ms0 == ms1 == 15.0
+    assert l0 == l1 == 4.0
     assert not np.array_equal(s0, s1)
 
 
