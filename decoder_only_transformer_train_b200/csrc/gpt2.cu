@@ -184,9 +184,6 @@ const void* W(gpt2_ctx* c, int idx) {
   if (c->bf16) return c->shadow + c->views[idx].off;
   return c->params + c->views[idx].off;
 }
-void* actp(gpt2_ctx* c, void* base, long long elems) {
-  return reinterpret_cast<char*>(base) + elems * (long long)c->act;
-}
 
 int build_views(gpt2_ctx* c) {
   const gpt2_config& g = c->cfg;
