@@ -14,7 +14,6 @@ enum DeviceError : int {
   DEVERR_TARGET = 2,    // target outside [0, vocab_size) and not the ignore index -1
   DEVERR_TIMEOUT = 3,   // a bounded wait on an mbarrier gave up
   DEVERR_INTERNAL = 4,
-  DEVERR_ROW = 5,       // a sampled row index outside the logits
 };
 
 extern __device__ int g_device_error;

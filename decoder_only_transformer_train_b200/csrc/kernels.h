@@ -4,6 +4,10 @@
 #include <stdint.h>
 #include "gemm.h"
 
+// Device error code of the top-k sampling kernel, next to the codes of the training step
+// (DEVERR_NONE .. DEVERR_INTERNAL = 4 in common.cuh).
+constexpr int DEVERR_ROW = 5;   // a sampled row index outside the logits
+
 struct AdamBlock {      // one block of the multi-tensor AdamW launch
   long long off;        // first element (flat parameter index)
   int n;                // elements in this block
