@@ -69,10 +69,12 @@ def parse():
                          "micro-steps and average the gradients with one all-reduce before AdamW")
     args = ap.parse_args()
     m = MODELS[args.model]
-    # a longer context keeps the model's tokens per micro-step (the embedding backward sorts
-    # at most 32768 positions) and per step (e.g. T=2048: B=16, 16 micro-steps for the 124M model)
+    # the 124M model at a longer context takes the pages' GPT-3 batch ("3:41:50 – 3:53:37" of the
+    # Lecture 9 notes: T = 2048 with B = 32), at most 131072 positions per micro-step; the step
+    # keeps its tokens (T = 2048: B = 32, 8 micro-steps of 65,536 tokens)
     if args.micro_batch is None:
-        args.micro_batch = max(1, min(m["micro_batch"], 32768 // args.seq))
+        b = 32 if (args.model == "124m" and args.seq > 1024) else m["micro_batch"]
+        args.micro_batch = max(1, min(b, 131072 // args.seq))
     if args.accum is None:
         args.accum = max(1, m["micro_batch"] * m["accum"] * 1024 // (args.micro_batch * args.seq))
     return args
@@ -199,6 +201,23 @@ def dist_max(x: float, world: int, device, op: str = "max") -> float:
     return float(t.item())
 
 
+def average_gradients(grads, world: int):
+    """Data-parallel gradient exchange ("2:46:43 – 2:59:25 Going multi-GPU with DDP" and
+    "2:59:25 – 3:10:20 Synchronizing gradients and losses" of the Lecture 9 notes): every
+    rank's gradient of its own loss / k_local is replaced, in place, by the mean over the
+    ranks, once per optimizer step after the rank's last micro-step.  With k_local micro-steps
+    on each of `world` ranks that is the gradient of the global batch's mean loss.  A sum
+    followed by one division, so the same code runs on NCCL and on gloo (which has no
+    average)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        assert world == 1, "a data-parallel exchange needs a process group"
+        return grads
+    dist.all_reduce(grads, op=dist.ReduceOp.SUM)
+    grads.div_(world)
+    return grads
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -206,6 +225,44 @@ def barrier(world):
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
+def cpu_oracle_configs():
+    """Wall time of the oracle (fp32, as it stands) on the small workloads: the tiny model's
+    full step (B=2, T=64: forward, backward, clip, AdamW), the 124M B=1 x T=1024 forward +
+    backward on one thread, and one 124M step on B=4 x T=1024 on all host threads."""
+    import torch
+    import oracle as O
+    from decoder_only_transformer_train_b200 import synthetic as S
+    out = {}
+
+    def step(params, cfg, B, T, seed):
+        m = {n: torch.zeros_like(t) for n, t in params.items()}
+        v = {n: torch.zeros_like(t) for n, t in params.items()}
+        x, y = S.token_batch(seed, B, T, cfg.vocab_size)
+        t0 = time.perf_counter()
+        O.train_step(params, m, v, 1, cfg, [(torch.from_numpy(x), torch.from_numpy(y))], O.get_lr(1000))
+        return time.perf_counter() - t0
+
+    out["tiny_step_s"] = round(step(O.init_params(O.TINY, 1, dtype=torch.float32), O.TINY, 2, 64, 2), 4)
+    cfg = O.GPT2_124M
+    params = O.init_params(cfg, 1, dtype=torch.float32)
+    threads = torch.get_num_threads()
+    torch.set_num_threads(1)
+    try:
+        x, y = S.token_batch(3, 1, 1024, cfg.vocab_size)
+        t0 = time.perf_counter()
+        _, cache = O.forward(params, cfg, torch.from_numpy(x), torch.from_numpy(y))
+        O.backward(params, cfg, cache)
+        t1 = time.perf_counter() - t0
+        del cache
+    finally:
+        torch.set_num_threads(threads)
+    out["gpt2_124m_b1_fwd_bwd_1_thread_s"] = round(t1, 2)
+    out["gpt2_124m_tokens_per_s_1_thread"] = round(1024 / t1, 1)
+    out["gpt2_124m_b4_step_s"] = round(step(params, cfg, 4, 1024, 2), 2)
+    out["threads"] = threads
+    return out
+
+
 def cpu_oracle_sample(seq: int, samples: int = 1, model: str = "124m", seqs_per_step: int = 512):
     """Times the CPU oracle (fp32, as it stands) on B=1 x `seq` tokens of the same model:
     forward + backward per sample, plus one clip + AdamW step amortised over the
@@ -252,7 +309,12 @@ def run_reference(args, world, rank):
     ms = args.micro_batch * args.seq * args.accum / value * 1000.0
     line = {
         "metric": metric_name(args.model, args.micro_batch, args.seq), "impl": "reference", "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        # each timed step is one B=1 sequence plus its share of the optimizer step; ms_per_step
+        # is that rate extrapolated to the whole optimizer step, which was not run
+        "extrapolated": True, "timed_samples": args.steps,
+        "timed_sample": f"B=1 x T={args.seq} forward+backward plus 1/{args.micro_batch * args.accum} of clip+AdamW",
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": workload_config(args),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
@@ -307,8 +369,7 @@ def run_ours(args, world, rank, local):
         # data-parallel: every rank's gradient (of its loss / k) averaged across ranks, once
         # per optimizer step, on the model's stream before the clip and AdamW
         if ddp:
-            import torch.distributed as dist
-            dist.all_reduce(grads, op=dist.ReduceOp.AVG)
+            average_gradients(grads, world)
 
     def step():
         model.zero_grad()
@@ -392,6 +453,8 @@ def run_ours(args, world, rank, local):
         cpu = {"value": r, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                "sample": f"{MODELS[args.model]['label']} fp32 CPU oracle, B=1 x T={T} forward+backward ({t_fb:.2f} s) plus "
                          f"1/{B * k} of clip+AdamW ({t_opt:.2f} s)"}
+        if args.model == "124m" and T == 1024:
+            cpu["other_workloads"] = cpu_oracle_configs()
 
     if rank == 0:
         pk = peaks()

@@ -73,6 +73,7 @@ _PROTOS = {
     "gpt2op_classifier_aux_floats": (_i64, [_i, _i]),
     "gpt2op_classifier_fwd_bwd": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "gpt2op_device_error": (_i, []),
+    "gpt2op_bounded_wait_selftest": (_i, [_vp, _i64, _vp, _vp]),
     "gpt2_lr_cosine": (ctypes.c_double, [_i64, ctypes.c_double, _i64, _i64, ctypes.c_double]),
     "gpt2_kernel_launches": (_i64, []),
     "gpt2_profile_start": (_i, [_vp]),
@@ -364,3 +365,7 @@ def classifier_fwd_bwd(h, W, targets, N, V, C, logits_ws, ldl, aux_ws, loss, lse
 
 def device_error() -> int:
     return int(lib().gpt2op_device_error())
+
+
+def bounded_wait_selftest(limit_ns: int, src16, status, stream=None):
+    _check(lib().gpt2op_bounded_wait_selftest(_stream(stream), limit_ns, _ptr(src16), _ptr(status)))

@@ -306,7 +306,7 @@ int launch_attn_fwd(cudaStream_t st, bool is_bf16, const void* qkv, void* out, f
   return launch_attn_fwd_simt(st, is_bf16, qkv, out, lse, B, T, H, hd);
 }
 int launch_attn_bwd(cudaStream_t st, bool is_bf16, const void* qkv, const void* out, const void* dout,
-                    const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd) {
+                    const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd, float* bias_part) {
   if (is_bf16 && hd == 64) {
     const long long ntok = (long long)B * T;
     if ((reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(dout)) % 16 == 0) {
@@ -320,7 +320,8 @@ int launch_attn_bwd(cudaStream_t st, bool is_bf16, const void* qkv, const void* 
     }
     note_kernel_launches(1);
     if (cudaGetLastError() != cudaSuccess) return -3;
-    return launch_attn_bwd_tc(st, qkv, dout, lse, Dbuf, dqkv, B, T, H, hd);
+    return launch_attn_bwd_tc(st, qkv, dout, lse, Dbuf, dqkv, B, T, H, hd, bias_part);
   }
+  if (bias_part != nullptr) return -4;   // the column sums come only with the tensor-core path
   return launch_attn_bwd_simt(st, is_bf16, qkv, out, dout, lse, Dbuf, dqkv, B, T, H, hd);
 }

@@ -13,11 +13,11 @@
 //   warps 2..9  : two softmax groups of four warps; the CTA's key tiles alternate between
 //                 them (global tile counter parity).  Thread r of a group owns query row r
 //                 (= TMEM lane r): it reads S_j, applies the causal mask, and writes
-//                 P_j = 2^(s*log2e/sqrt(hd) - m_ref) (bf16) to shared memory in the
-//                 128-byte-swizzled K-major layout the MMA reads.  Each group accumulates
-//                 its own O in TMEM; m_ref only moves when a row's max grows by more than
-//                 2^8, and then the thread rescales its O row in TMEM before the next MMA.
-//                 At the end of an item the two groups' (m_ref, l, O) are merged.
+//                 P_j = 2^(s*log2e/sqrt(hd) - m_ref) as bf16 pairs into the group's P columns
+//                 of TMEM, from where the P V product reads it as its A operand.  Each group
+//                 accumulates its own O in TMEM; m_ref only moves when a row's max grows by
+//                 more than 2^8, and then the thread rescales its O row in TMEM before the
+//                 next MMA.  At the end of an item the two groups' (m_ref, l, O) are merged.
 #include <math.h>
 #include "sm100.cuh"
 #include "kernels.h"
@@ -27,19 +27,16 @@ namespace {
 constexpr int QT = 128;          // queries per item
 constexpr int KT = 128;          // keys per tile
 constexpr int HD = 64;
-constexpr int KV_STAGES = 3;
+constexpr int KV_STAGES = 5;
 constexpr int NUM_THREADS = 320;
 constexpr int TILE_BYTES = KT * HD * 2;        // 16 KB: one Q, K or V tile
-constexpr int P_BYTES = QT * KT * 2;           // 32 KB
-constexpr int SMEM_BYTES = 2 * TILE_BYTES + 2 * KV_STAGES * TILE_BYTES + 2 * P_BYTES + QT * 8 + 512 + 1024;
+constexpr int SMEM_BYTES = 2 * TILE_BYTES + 2 * KV_STAGES * TILE_BYTES + QT * 8 + 512 + 1024;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t S_COL = 0;                  // S of group g: columns [128 g, 128 g + 128)
 constexpr uint32_t O_COL = 256;                // O of group g: columns [256 + 64 g, 256 + 64 g + 64)
+constexpr uint32_t P_COL = 384;                // P of group g (bf16 pairs): columns [384 + 64 g, 384 + 64 g + 64)
 constexpr float RESCALE_THRESHOLD = 8.0f;      // log2 units
 
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // Row max of a 128-column S tile in TMEM (64 columns per round trip); on the diagonal
 // tile the keys after query row r are left out.  Four independent max chains.
@@ -48,6 +45,8 @@ __device__ __forceinline__ float s_row_max(uint32_t taddr, int r) {
   float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int c0 = 0; c0 < 128; c0 += 64) {
+    // on the diagonal tile rows below 64 (warps of lane quarters 0 and 1) see only the first half
+    if (DIAG && c0 == 64 && r < 64) break;
     uint32_t v[64];
     tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
     tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
@@ -65,56 +64,57 @@ __device__ __forceinline__ float s_row_max(uint32_t taddr, int r) {
   return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 }
 
-// P = 2^(s * scale_log2 - m_ref) for a 128-column S row, written as bf16 into row r of a
-// 128 x 128 K-major SW128 operand; returns the row sum of P (four independent partial sums).
-// With MAX, the same pass also returns the row's raw max in *mx (masked keys left out), so
-// that a tile whose max stays within the rescale threshold of m_ref is read from TMEM once.
+// P = 2^(s * scale_log2 - m_ref) for a 128-column S row, written as bf16 pairs into the 64
+// P columns at TMEM address pcol (this thread's lane); returns the row sum of P (four
+// independent partial sums).  With MAX, the same pass also returns the row's raw max in *mx
+// (masked keys left out), so that a tile whose max stays within the rescale threshold of m_ref
+// is read from TMEM once.
 template <bool DIAG, bool MAX = false>
-__device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint8_t* prow,
+__device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint32_t pcol,
                                              float* mx = nullptr) {
   float2 sum[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
   float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   const float2 sc = make_float2(scale_log2, scale_log2);
   const float2 nm = make_float2(-m_ref, -m_ref);
-  auto half = [&](int c0, const uint32_t* v) {
+  auto half = [&](int c0, const uint32_t* v, uint32_t* w) {
 #pragma unroll
-    for (int g8 = 0; g8 < 8; ++g8) {
-      float p[8];
-#pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const float sa = __uint_as_float(v[g8 * 8 + e]), sb = __uint_as_float(v[g8 * 8 + e + 1]);
-        const float2 x = ffma2(make_float2(sa, sb), sc, nm);
-        p[e] = ex2(x.x);
-        p[e + 1] = ex2(x.y);
-        if (DIAG) {
-          const int col = c0 + g8 * 8 + e;
-          if (col > r) p[e] = 0.f;
-          if (col + 1 > r) p[e + 1] = 0.f;
-        }
-        if (MAX) {
-          const int col = c0 + g8 * 8 + e;
-          const float ma = (DIAG && col > r) ? -INFINITY : sa;
-          const float mb = (DIAG && col + 1 > r) ? -INFINITY : sb;
-          m4[e >> 1] = max3f(m4[e >> 1], ma, mb);
-        }
-        sum[e >> 1] = fadd2(sum[e >> 1], make_float2(p[e], p[e + 1]));
+    for (int e = 0; e < 64; e += 2) {
+      const float sa = __uint_as_float(v[e]), sb = __uint_as_float(v[e + 1]);
+      const float2 x = ffma2(make_float2(sa, sb), sc, nm);
+      float pa = ex2(x.x), pb = ex2(x.y);
+      if (DIAG) {
+        const int col = c0 + e;
+        if (col > r) pa = 0.f;
+        if (col + 1 > r) pb = 0.f;
       }
-      uint4 w;
-      w.x = pack_bf16x2(p[0], p[1]);
-      w.y = pack_bf16x2(p[2], p[3]);
-      w.z = pack_bf16x2(p[4], p[5]);
-      w.w = pack_bf16x2(p[6], p[7]);
-      *reinterpret_cast<uint4*>(prow + (c0 >> 6) * 16384 + ((g8 ^ (r & 7)) << 4)) = w;
+      if (MAX) {
+        const int col = c0 + e;
+        const float ma = (DIAG && col > r) ? -INFINITY : sa;
+        const float mb = (DIAG && col + 1 > r) ? -INFINITY : sb;
+        m4[(e >> 1) & 3] = max3f(m4[(e >> 1) & 3], ma, mb);
+      }
+      sum[(e >> 1) & 3] = fadd2(sum[(e >> 1) & 3], make_float2(pa, pb));
+      w[e >> 1] = pack_bf16x2(pa, pb);
     }
   };
 #pragma unroll 1
   for (int c0 = 0; c0 < 128; c0 += 64) {
-    uint32_t v[64];
-    tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-    tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-    tmem_wait_ld();
-    half(c0, v);
+    uint32_t w[32];
+    if (DIAG && c0 == 64 && r < 64) {
+      // a wholly masked half (rows below 64 of the diagonal tile; warp-uniform): P = 0
+#pragma unroll
+      for (int e = 0; e < 32; ++e) w[e] = 0u;
+    } else {
+      uint32_t v[64];
+      tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_wait_ld();
+      half(c0, v, w);
+    }
+    tmem_st16(pcol + (c0 >> 1), *reinterpret_cast<uint32_t(*)[16]>(w));
+    tmem_st16(pcol + (c0 >> 1) + 16, *reinterpret_cast<uint32_t(*)[16]>(w + 16));
   }
+  tmem_wait_st();
   if (MAX) *mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
   const float2 s01 = fadd2(sum[0], sum[1]), s23 = fadd2(sum[2], sum[3]);
   return (s01.x + s01.y) + (s23.x + s23.y);
@@ -137,8 +137,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
   uint8_t* sQ = smem;                                    // [2]
   uint8_t* sK = sQ + 2 * TILE_BYTES;                     // [KV_STAGES]
   uint8_t* sV = sK + KV_STAGES * TILE_BYTES;             // [KV_STAGES]
-  uint8_t* sP = sV + KV_STAGES * TILE_BYTES;             // [2]
-  float* sML = reinterpret_cast<float*>(sP + 2 * P_BYTES);   // [QT][2]: handed-over (m_ref, l)
+  float* sML = reinterpret_cast<float*>(sV + KV_STAGES * TILE_BYTES);   // [QT][2]: handed-over (m_ref, l)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sML + 2 * QT);
   uint64_t* q_full = bars;                       // 2
   uint64_t* q_empty = q_full + 2;                // 2
@@ -192,6 +191,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       // ---------------------------------------------------------------- TMA producer
       int G = 0;                                   // global key-tile counter
       bool ok = true;
+      InflightTx tx{bars, 0u, 0u};
       for (int t = blockIdx.x, k = 0; t < items.total && ok; t += gridDim.x, ++k) {
         int qt, bh;
         items.get(t, qt, bh);
@@ -200,20 +200,23 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         if (!mbar_wait(&q_empty[qb], ((k >> 1) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[qb], TILE_BYTES);
         tma_load_2d(sQ + qb * TILE_BYTES, &tm_qkv, h * HD, row0 + qt * QT, &q_full[qb]);
+        tx.note(&q_full[qb], (k >> 1) & 1);
         for (int j = 0; j <= qt; ++j, ++G) {
           const int s = G % KV_STAGES;
           if (!mbar_wait(&kv_empty[s], ((G / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&kv_full[s], 2 * TILE_BYTES);
           tma_load_2d(sK + s * TILE_BYTES, &tm_qkv, C + h * HD, row0 + j * KT, &kv_full[s]);
           tma_load_2d(sV + s * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + j * KT, &kv_full[s]);
+          tx.note(&kv_full[s], (G / KV_STAGES) & 1);
         }
       }
+      if (*abort_flag) tx.drain();   // copies still in flight land before the CTA leaves
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = make_idesc_bf16(QT, KT, false, false);   // Q, K both K-major
-      constexpr uint32_t idesc_o = make_idesc_bf16(QT, HD, false, true);    // P K-major, V MN-major
+      constexpr uint32_t idesc_o = make_idesc_bf16(QT, HD, false, true);    // P from TMEM, V MN-major
       // tile iterator over the CTA's flattened (item, j) sequence
       struct It {
         int t, k, qt, j, G;
@@ -267,12 +270,12 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         if (g) ++co1; else ++co0;
         tc_fence_after();
         const bool first_of_group = (cur.j < 2);          // the group's first tile of this item
-        const uint32_t aP = smem_u32(sP + g * P_BYTES);
         const uint32_t bV = smem_u32(sV + s * TILE_BYTES);
+        // A: 16 keys of P = 8 TMEM columns per step; B: 16 rows of V, MN-major
 #pragma unroll
         for (int kk = 0; kk < KT / 16; ++kk)
-          tc_mma_bf16(tmem + O_COL + g * HD, make_sdesc_sw128(aP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                      make_sdesc_sw128(bV + kk * 2048, 8192, 1024), idesc_o, (kk > 0 || !first_of_group) ? 1u : 0u);
+          tc_mma_bf16_ts(tmem + O_COL + g * HD, tmem + P_COL + g * 64 + kk * 8,
+                         make_sdesc_sw128(bV + kk * 2048, 8192, 1024), idesc_o, (kk > 0 || !first_of_group) ? 1u : 0u);
         tc_commit(&kv_empty[s]);
         tc_commit(&p_empty[g]);
         if (cur.j + 2 > cur.qt) tc_commit(&o_done[g]);    // the group's last tile of this item
@@ -287,7 +290,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
     const int r = q * 32 + lane;                 // query row within the item
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t s_col = S_COL + grp * KT;
-    uint8_t* prow = sP + grp * P_BYTES + r * 128;
+    const uint32_t pcol = tmem + lane_off + P_COL + grp * 64;   // this row's P columns
     int c = 0, d = 0, hcount = 0;                // this group's tiles, items, handovers
     bool pending = false;                        // an O handover the finisher has not released yet
     bool ok = true;
@@ -301,7 +304,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       float m_ref = -INFINITY, l = 0.f;
       bool has = false;
       for (int j = ((G0 & 1) == grp) ? 0 : 1; j < n_kv; j += 2) {
-        if (!mbar_wait(&s_full[grp], c & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&s_full[grp], c & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const bool diag = (j == qt);
         const uint32_t srow = tmem + lane_off + s_col;
@@ -310,16 +313,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
           // the group's first tile of the item: its row max sets m_ref (two TMEM passes)
           const float mx = diag ? s_row_max<true>(srow, r) : s_row_max<false>(srow, r);
           // the group's previous P.V MMA must be done: P buffer free, O stable
-          if (!mbar_wait(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
           m_ref = mx * scale_log2;
-          sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, prow)
-                     : p_row_store<false>(srow, r, scale_log2, m_ref, prow);
+          sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, pcol)
+                     : p_row_store<false>(srow, r, scale_log2, m_ref, pcol);
         } else {
           // one pass: P against the current m_ref, and the tile's row max alongside
-          if (!mbar_wait(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
           float mx;
-          sum = diag ? p_row_store<true, true>(srow, r, scale_log2, m_ref, prow, &mx)
-                     : p_row_store<false, true>(srow, r, scale_log2, m_ref, prow, &mx);
+          sum = diag ? p_row_store<true, true>(srow, r, scale_log2, m_ref, pcol, &mx)
+                     : p_row_store<false, true>(srow, r, scale_log2, m_ref, pcol, &mx);
           const float m_new = mx * scale_log2;
           const bool grow = m_new > m_ref + RESCALE_THRESHOLD;
           // tcgen05.ld / st are warp-collective, so the whole warp takes this branch when
@@ -341,8 +344,8 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
             tmem_wait_st();
             l *= f;
             if (grow) m_ref = m_new;
-            sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, prow)
-                       : p_row_store<false>(srow, r, scale_log2, m_ref, prow);
+            sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, pcol)
+                       : p_row_store<false>(srow, r, scale_log2, m_ref, pcol);
           }
         }
         l += sum;
@@ -350,17 +353,16 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         mbar_arrive(&s_empty[grp]);
         // an O row handed over at the previous item must be read before this group's next MMA
         if (pending) {
-          if (!mbar_wait(merge_empty, (hcount & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(merge_empty, (hcount & 1) ^ 1, abort_flag)) { ok = false; break; }
           pending = false;
         }
-        fence_async_smem();
-        mbar_arrive(&p_full[grp]);
+        mbar_arrive(&p_full[grp]);   // P is in TMEM (tcgen05.wait::st, then the fence above)
         has = true;
         ++c;
       }
       if (!ok) break;
       if (has) {
-        if (!mbar_wait(&o_done[grp], d & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&o_done[grp], d & 1, abort_flag)) { ok = false; break; }
         ++d;
       }
       const int finisher = (G0 + n_kv - 1) & 1;
@@ -368,7 +370,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       if (grp != finisher) {
         if (both) {
           // hand (m_ref, l) over; O stays in this group's TMEM columns for the finisher
-          if (pending && !mbar_wait(merge_empty, (hcount & 1) ^ 1, abort_flag)) { ok = false; break; }
+          if (pending && !mbar_wait_warp(merge_empty, (hcount & 1) ^ 1, abort_flag)) { ok = false; break; }
           sML[r * 2] = m_ref;
           sML[r * 2 + 1] = l;
           mbar_arrive(merge_full);
@@ -379,7 +381,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         const int qi = qt * QT + r;
         float m1 = -INFINITY, l1 = 0.f;
         if (both) {
-          if (!mbar_wait(merge_full, hcount & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(merge_full, hcount & 1, abort_flag)) { ok = false; break; }
           m1 = sML[r * 2];
           l1 = sML[r * 2 + 1];
         }
@@ -421,7 +423,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         }
       }
     }
-    if (ok && pending) mbar_wait(merge_empty, (hcount & 1) ^ 1, abort_flag);
+    if (ok && pending) mbar_wait_warp(merge_empty, (hcount & 1) ^ 1, abort_flag);
   }
 
   tc_fence_before();
@@ -468,16 +470,8 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return -3;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-        cudaSuccess)
-      return -3;
-    attr = true;
-  }
-  int dev = 0, nsm = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (set_dynamic_smem_once((const void*)attn_fwd_tc_kernel, SMEM_BYTES)) return -3;
+  const int nsm = current_device_sms();
   const int total = cdiv(T, QT) * B * H;
   const int grid = total < nsm ? total : nsm;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
@@ -493,26 +487,21 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
 //   dV = P^T dO,   dZ = P * (dO V^T - D),   dQ = dZ K / sqrt(hd),   dK = dZ^T Q / sqrt(hd).
 // Two kernels keep every sum in a fixed order (no atomics): the dK/dV kernel accumulates
 // each 128-key tile over the query tiles at or after it, the dQ kernel each 128-query tile
-// over the key tiles at or before it.
+// over the key tiles at or before it.  P and dZ never leave the SM: the elementwise warps
+// write them as bf16 into tensor memory, from where the MMAs read them as their A operand.
 namespace {
 
 constexpr int BWD_THREADS = 576;   // producer, MMA, 16 elementwise warps (4 per TMEM lane quarter)
-constexpr int BWD_STAGES = 3;
+constexpr int BWD_STAGES = 4;
 // smem: two buffers of the 2 resident tiles (K_j,V_j or Q_i,dO_i: this item's and the next
-// one's), BWD_STAGES x 2 streamed tiles, the 128x128 bf16 operands (P and dZ) and barriers
-constexpr int BWD_SMEM = 4 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + 2 * P_BYTES + 512 + 1024;
+// one's), BWD_STAGES x 2 streamed tiles, per-warp column scalars and barriers
+constexpr int BWD_VEC_BYTES = 16 * 64 * 4;
+constexpr int BWD_SMEM = 4 * TILE_BYTES + BWD_STAGES * 2 * TILE_BYTES + BWD_VEC_BYTES + 512 + 1024;
 static_assert(BWD_SMEM <= 232448, "attention backward shared memory");
-
-// Writes 32 bf16 values, packed in pairs (columns col0 .. col0+31, col0 a multiple of 32),
-// into row r of a 128 x 128 operand stored as two 64-column halves of 128-byte swizzled rows.
-__device__ __forceinline__ void store_32_sw128(uint8_t* base, int r, int col0, const uint32_t* w16) {
-  uint8_t* row = base + (col0 >> 6) * 16384 + r * 128;
-  const int g0 = (col0 & 63) >> 3;
-#pragma unroll
-  for (int g = 0; g < 4; ++g)
-    *reinterpret_cast<uint4*>(row + (((g0 + g) ^ (r & 7)) << 4)) =
-        make_uint4(w16[g * 4 + 0], w16[g * 4 + 1], w16[g * 4 + 2], w16[g * 4 + 3]);
-}
+// TMEM columns: S [0,128) and dP [128,256) in fp32; P [256,320) and dZ [320,384) as bf16 pairs;
+// accumulators from 384: the dK/dV kernel's dV [384,448) and dK [448,512), the dQ kernel's dQ
+// in two buffers [384,448) and [448,512)
+constexpr uint32_t BS_C = 0, BDP_C = 128, BP_C = 256, BDS_C = 320, BACC_C = 384;
 
 // Work items of the backward: (128-row tile, batch*head), heaviest first.
 //   MODE 0 (dK/dV): item = key tile j, streams the query tiles i >= j  (n_t - j of them)
@@ -535,31 +524,54 @@ __device__ __forceinline__ int bwd_turn_item(int k) {
   return k * (int)gridDim.x + ((k & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
 }
 
-// MODE 0: dK/dV kernel;  MODE 1: dQ kernel.  Persistent: each CTA walks its items in turn.
-// Both hold S and dP with a query per TMEM lane.  Resident tiles and the TMEM accumulators
-// are double-buffered across items, so the next item's loads and first S / dP products
+// MODE 0: dK/dV kernel, a key per TMEM lane: S^T = K_j Q_i^T and dP^T = V_j dO_i^T, then
+//         dV += P^T dO_i and dK += dZ^T Q_i with P^T and dZ^T read from TMEM.
+// MODE 1: dQ kernel, a query per TMEM lane: S = Q_i K_j^T and dP = dO_i V_j^T, then
+//         dQ += dZ K_j with dZ read from TMEM.
+// Persistent: each CTA walks its items in turn.  Resident tiles are double-buffered across
+// items (and the dQ accumulator too), so the next item's loads and first S / dP products
 // overlap the current item's last tile and epilogue.
+// With bias_part non-null the epilogue also writes column sums of the gradients it produces
+// (the bias gradient of c_attn, before the bf16 rounding of dqkv): row (tile * B + b) * 4 + q,
+// columns [0, 3C), sums over the 32 rows of TMEM lane quarter q of the 128-row tile; every
+// (row, column) is written by exactly one item of one of the two kernels.
+// Column sums of one warp's 32 rows of 16 values (x[j] = row `lane`, column j): lane l returns
+// the sum of column l >> 1 (lanes l and l ^ 1 agree).  Each step halves the values a lane
+// keeps, adding its partner's half: 8 + 4 + 2 + 1 shuffles, then one for the last pair.
+__device__ __forceinline__ float warp_colsum16(float (&x)[16], int lane) {
+#pragma unroll
+  for (int s = 16, n = 16; s >= 2; s >>= 1, n >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = upper ? x[j] : x[j + n / 2];
+      const float keep = upper ? x[j + n / 2] : x[j];
+      x[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
+}
+
 template <int MODE>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                   const float* __restrict__ lse, const float* __restrict__ Dbuf, bf16* __restrict__ dqkv, int B,
-                   int T, int H, float scale, float scale_log2) {
+                   const float* __restrict__ lse, const float* __restrict__ Dbuf, bf16* __restrict__ dqkv,
+                   float* __restrict__ bias_part, int B, int T, int H, float scale, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sRes = smem;                                  // [2][K_j,V_j (MODE 0) / Q_i,dO_i (MODE 1)]
   uint8_t* sA = sRes + 4 * TILE_BYTES;                   // streamed: Q_i (MODE 0) / K_j (MODE 1)
   uint8_t* sB = sA + BWD_STAGES * TILE_BYTES;            // streamed: dO_i (MODE 0) / V_j (MODE 1)
-  uint8_t* sP = sB + BWD_STAGES * TILE_BYTES;            // P (MODE 0), a query per row
-  uint8_t* sDS = sP + P_BYTES;                           // dZ, a query per row
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + P_BYTES);
+  float* sVec = reinterpret_cast<float*>(sB + BWD_STAGES * TILE_BYTES);   // [16 warps][64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sVec) + BWD_VEC_BYTES);
   uint64_t* r_full = bars;                               // [2] resident tiles loaded
   uint64_t* r_empty = r_full + 2;                        // [2] resident tiles no longer read
   uint64_t* t_full = r_empty + 2;                        // [BWD_STAGES]
   uint64_t* t_empty = t_full + BWD_STAGES;               // [BWD_STAGES]
   uint64_t* sd_full = t_empty + BWD_STAGES;              // S and dP in TMEM
   uint64_t* sd_empty = sd_full + 1;                      // S and dP read out
-  uint64_t* ps_full = sd_empty + 1;                      // operands in smem
-  uint64_t* ps_empty = ps_full + 1;                      // operands consumed
+  uint64_t* ps_full = sd_empty + 1;                      // P and dZ written to TMEM
+  uint64_t* ps_empty = ps_full + 1;                      // P and dZ consumed by the MMAs
   uint64_t* acc_full = ps_empty + 1;                     // [2] an item's accumulation done
   uint64_t* acc_empty = acc_full + 2;                    // [2] an item's accumulators read out
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
@@ -570,9 +582,6 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   const int BH = B * H;
   const int n_items = n_t * BH;
   const int C = H * HD;
-  // TMEM columns: S [0,128), dP [128,256); accumulator buffer a at 256 + 128 a:
-  // acc0 (dV or dQ) 64 columns, acc1 (dK) the next 64
-  const uint32_t S_C = 0, DP_C = 128, ACC_C = 256;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -607,6 +616,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
     if (lane == 0) {
       // ---------------------------------------------------------------- TMA producer
       int g = 0;   // streamed tiles issued by this CTA (stage ring position)
+      InflightTx tx{bars, 0u, 0u};
       for (int k = 0;; ++k) {
         const int idx = bwd_turn_item(k);
         if (idx >= n_items) break;
@@ -623,6 +633,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
           tma_load_2d(r0, &tm_qkv, h * HD, row0 + w.tile * 128, &r_full[rb]);                      // Q_i
           tma_load_2d(r0 + TILE_BYTES, &tm_do, h * HD, row0 + w.tile * 128, &r_full[rb]);           // dO_i
         }
+        tx.note(&r_full[rb], (k >> 1) & 1);
         bool ok = true;
         for (int t = w.it0; t < w.it1; ++t, ++g) {
           const int st = g % BWD_STAGES;
@@ -635,17 +646,20 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
             tma_load_2d(sA + st * TILE_BYTES, &tm_qkv, C + h * HD, row0 + t * 128, &t_full[st]);      // K_j
             tma_load_2d(sB + st * TILE_BYTES, &tm_qkv, 2 * C + h * HD, row0 + t * 128, &t_full[st]);  // V_j
           }
+          tx.note(&t_full[st], (g / BWD_STAGES) & 1);
         }
         if (!ok) break;
       }
+      if (*abort_flag) tx.drain();   // copies still in flight land before the CTA leaves
     }
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_sq = make_idesc_bf16(128, 128, false, false);     // 128x128, K=64, both K-major
-      constexpr uint32_t idesc_acc = make_idesc_bf16(128, HD, MODE == 0, true);  // 128x64, K=128, B MN-major;
-                                                                                 // A MN-major in MODE 0
-      // S / dP of the CTA's g-th streamed tile, read against resident buffer rb
+      constexpr uint32_t idesc_sq = make_idesc_bf16(128, 128, false, false);   // 128x128, K=64, both K-major
+      constexpr uint32_t idesc_acc = make_idesc_bf16(128, HD, false, true);    // 128x64, K=128: A from TMEM,
+                                                                               // B MN-major
+      // S / dP of the CTA's g-th streamed tile, read against resident buffer rb: the resident
+      // tiles are the A operands in MODE 0 (rows: keys) and in MODE 1 (rows: queries)
       auto issue_sd = [&](int g, int rb) -> bool {
         const int st = g % BWD_STAGES;
         if (!mbar_wait(&t_full[st], (g / BWD_STAGES) & 1, abort_flag)) return false;
@@ -655,19 +669,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         const uint32_t r0 = smem_u32(sRes + rb * 2 * TILE_BYTES), r1 = r0 + TILE_BYTES;
 #pragma unroll
         for (int k = 0; k < HD / 16; ++k) {
-          if (MODE == 0) {
-            // S = Q_i K_j^T ; dP = dO_i V_j^T   (rows: the streamed query tile)
-            tc_mma_bf16(tmem + S_C, make_sdesc_sw128(a + k * 32, 16, 1024), make_sdesc_sw128(r0 + k * 32, 16, 1024),
-                        idesc_sq, k > 0 ? 1u : 0u);
-            tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(bq + k * 32, 16, 1024), make_sdesc_sw128(r1 + k * 32, 16, 1024),
-                        idesc_sq, k > 0 ? 1u : 0u);
-          } else {
-            // S = Q_i K_j^T ; dP = dO_i V_j^T   (rows: the resident query tile)
-            tc_mma_bf16(tmem + S_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
-                        idesc_sq, k > 0 ? 1u : 0u);
-            tc_mma_bf16(tmem + DP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024), make_sdesc_sw128(bq + k * 32, 16, 1024),
-                        idesc_sq, k > 0 ? 1u : 0u);
-          }
+          // MODE 0: S^T = K_j Q_i^T, dP^T = V_j dO_i^T;  MODE 1: S = Q_i K_j^T, dP = dO_i V_j^T
+          tc_mma_bf16(tmem + BS_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
+                      idesc_sq, k > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + BDP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024), make_sdesc_sw128(bq + k * 32, 16, 1024),
+                      idesc_sq, k > 0 ? 1u : 0u);
         }
         tc_commit(sd_full);
         return true;
@@ -680,8 +686,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         const BwdItem w = bwd_item<MODE>(idx, BH, n_t);
         const int n_it = w.it1 - w.it0;
         const int nidx = bwd_turn_item(k + 1);
-        const int ab = k & 1;
-        const uint32_t acc0 = tmem + ACC_C + ab * 128, acc1 = acc0 + 64;
+        const int ab = (MODE == 0) ? 0 : (k & 1);            // dK/dV: one accumulator buffer; dQ: two
+        const uint32_t acc0 = tmem + BACC_C + ab * 64, acc1 = acc0 + 64;
         for (int n = 0; n < n_it && ok; ++n, ++g) {
           // S / dP one tile ahead, possibly the next item's first
           if (n + 1 < n_it) {
@@ -690,29 +696,30 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
             ok = mbar_wait(&r_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag) && issue_sd(g + 1, (k + 1) & 1);
           }
           if (!ok) break;
-          // the accumulator buffer must have been read out by item k - 2's epilogue
-          if (n == 0 && !mbar_wait(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          // the accumulator buffer must have been read out by the epilogue of the item that
+          // last used it (item k - 1 for dK/dV, k - 2 for dQ)
+          if (n == 0) {
+            const bool got = (MODE == 0) ? mbar_wait(&acc_empty[0], (k & 1) ^ 1, abort_flag)
+                                         : mbar_wait(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag);
+            if (!got) { ok = false; break; }
+          }
           const int st = g % BWD_STAGES;
           if (!mbar_wait(ps_full, g & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a = smem_u32(sA + st * TILE_BYTES), bq = smem_u32(sB + st * TILE_BYTES);
-          const uint32_t dsA = smem_u32(sDS);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t accum = (n > 0 || kk > 0) ? 1u : 0u;
+            // A: 16 queries (MODE 0) or keys (MODE 1) of P / dZ = 8 TMEM columns per step;
+            // B: the same 16 rows of a [128 x 64] tile, MN-major (2 KB per step)
             if (MODE == 0) {
-              // dV += P^T dO_i ; dK += dZ^T Q_i.  P and dZ are stored with a query per row (keys in
-              // two 64-column halves 16 KB apart), which read as MN-major A operands (M = keys,
-              // K = queries: 16 query rows = 2 KB per step); B operands MN-major: [128 queries x 64]
-              tc_mma_bf16(acc0, make_sdesc_sw128(smem_u32(sP) + kk * 2048, 16384, 1024),
-                          make_sdesc_sw128(bq + kk * 2048, 8192, 1024), idesc_acc, accum);
-              tc_mma_bf16(acc1, make_sdesc_sw128(dsA + kk * 2048, 16384, 1024),
-                          make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc, accum);
+              tc_mma_bf16_ts(acc0, tmem + BP_C + kk * 8, make_sdesc_sw128(bq + kk * 2048, 8192, 1024), idesc_acc,
+                             accum);                                                    // dV += P^T dO_i
+              tc_mma_bf16_ts(acc1, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
+                             accum);                                                    // dK += dZ^T Q_i
             } else {
-              // dQ += dZ K_j   (A K-major: 16 keys = 32 bytes per step within a 64-key half)
-              const uint32_t koff = (kk >> 2) * 16384 + (kk & 3) * 32;
-              tc_mma_bf16(acc0, make_sdesc_sw128(dsA + koff, 16, 1024), make_sdesc_sw128(a + kk * 2048, 8192, 1024),
-                          idesc_acc, accum);
+              tc_mma_bf16_ts(acc0, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
+                             accum);                                                    // dQ += dZ K_j
             }
           }
           tc_commit(&t_empty[st]);
@@ -728,42 +735,55 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
     // ------------------------------------------------------------------ elementwise
     const int q = warp & 3;
     const int part = (warp - 2) >> 2;            // columns [32*part, 32*part + 32) of each tile
-    const int r = q * 32 + lane;
+    const int r = q * 32 + lane;                 // TMEM lane: a key (MODE 0) or a query (MODE 1)
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const float LOG2E = 1.4426950408889634f;
     const int c0 = part * 32;
     const float2 sc = make_float2(scale_log2, scale_log2);
+    float* vec = sVec + (warp - 2) * 64;         // MODE 0: -lse*log2e and -D of this warp's 32 queries
     // Epilogue of the CTA's k-th item: accumulators -> dqkv (bf16).  The TMEM buffer is
-    // released before the global stores.
+    // released after the last read, before the global stores.
     auto epilogue = [&](const BwdItem& w, int k) -> bool {
-      const int ab = k & 1;
-      if (!mbar_wait(&acc_full[ab], (k >> 1) & 1, abort_flag)) return false;
+      const int ab = (MODE == 0) ? 0 : (k & 1);
+      if (!mbar_wait_warp(&acc_full[ab], (MODE == 0) ? (k & 1) : ((k >> 1) & 1), abort_flag)) return false;
       tc_fence_after();
       const int gi = w.tile * 128 + r;
       const int row0 = (w.bh / H) * T, h = w.bh % H;
       bf16* row = dqkv + (long long)(row0 + gi) * (3 * C) + h * HD + part * 16;
-      // MODE 0: dV (column block 2C) and dK (column block C, times scale); MODE 1: dQ (times scale).
-      // Each of the 4 warps of a lane quarter writes 16 of the 64 head columns; the TMEM
-      // buffer is released after the last read, before the last stores.
+      // MODE 0: dV (column block 2C) and dK (column block C, times scale); MODE 1: dQ (times
+      // scale).  Each of the 4 warps of a lane quarter writes 16 of the 64 head columns.
+      constexpr int NA = (MODE == 0) ? 2 : 1;
+      uint32_t u[NA][16];
 #pragma unroll
-      for (int a = 0; a < ((MODE == 0) ? 2 : 1); ++a) {
-        uint32_t u[16];
-        tmem_ld16(tmem + lane_off + ACC_C + ab * 128 + a * 64 + part * 16, u);
-        tmem_wait_ld();
-        if (a + 1 == ((MODE == 0) ? 2 : 1)) {
-          tc_fence_before();
-          mbar_arrive(&acc_empty[ab]);
+      for (int a = 0; a < NA; ++a) tmem_ld16(tmem + lane_off + BACC_C + ab * 64 + a * 64 + part * 16, u[a]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
+      if (bias_part != nullptr) {
+        const int b = w.bh / H;
+        float* prow = bias_part + ((long long)(w.tile * B + b) * 4 + q) * (3 * C) + h * HD + part * 16 + (lane >> 1);
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+          const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
+          float x[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) x[j] = (gi < T) ? __uint_as_float(u[a][j]) * mul : 0.f;
+          const float cs = warp_colsum16(x, lane);
+          if ((lane & 1) == 0) prow[(MODE == 1) ? 0 : (a == 0 ? 2 * C : C)] = cs;
         }
-        const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
-        if (gi < T) {
+      }
+      if (gi < T) {
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+          const float mul = (MODE == 0 && a == 0) ? 1.0f : scale;
           bf16* dst = row + ((MODE == 1) ? 0 : (a == 0 ? 2 * C : C));
 #pragma unroll
           for (int gq = 0; gq < 2; ++gq) {
             uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(u[gq * 8 + 0]) * mul, __uint_as_float(u[gq * 8 + 1]) * mul);
-            v.y = pack_bf16x2(__uint_as_float(u[gq * 8 + 2]) * mul, __uint_as_float(u[gq * 8 + 3]) * mul);
-            v.z = pack_bf16x2(__uint_as_float(u[gq * 8 + 4]) * mul, __uint_as_float(u[gq * 8 + 5]) * mul);
-            v.w = pack_bf16x2(__uint_as_float(u[gq * 8 + 6]) * mul, __uint_as_float(u[gq * 8 + 7]) * mul);
+            v.x = pack_bf16x2(__uint_as_float(u[a][gq * 8 + 0]) * mul, __uint_as_float(u[a][gq * 8 + 1]) * mul);
+            v.y = pack_bf16x2(__uint_as_float(u[a][gq * 8 + 2]) * mul, __uint_as_float(u[a][gq * 8 + 3]) * mul);
+            v.z = pack_bf16x2(__uint_as_float(u[a][gq * 8 + 4]) * mul, __uint_as_float(u[a][gq * 8 + 5]) * mul);
+            v.w = pack_bf16x2(__uint_as_float(u[a][gq * 8 + 6]) * mul, __uint_as_float(u[a][gq * 8 + 7]) * mul);
             reinterpret_cast<uint4*>(dst)[gq] = v;
           }
         }
@@ -780,58 +800,80 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       const BwdItem w = bwd_item<MODE>(idx, BH, n_t);
       const float* lse_bh = lse + (long long)w.bh * T;
       const float* D_bh = Dbuf + (long long)w.bh * T;
-      float row_lse2 = 0.f, row_D = 0.f;
+      // MODE 1: this thread's query row; a row past T gets P = 0 (its lse taken as +inf)
+      float nl1 = 0.f, nd1 = 0.f;
       if (MODE == 1) {
         const int qi = w.tile * 128 + r;
-        row_lse2 = (qi < T) ? __ldg(lse_bh + qi) * LOG2E : 0.f;
-        row_D = (qi < T) ? __ldg(D_bh + qi) : 0.f;
+        nl1 = (qi < T) ? -__ldg(lse_bh + qi) * LOG2E : -INFINITY;
+        nd1 = (qi < T) ? -__ldg(D_bh + qi) : 0.f;
       }
       for (int t = w.it0; t < w.it1; ++t, ++g) {
-        // MODE 0 streams the query tiles, so its row's lse and D change with t: load them
-        // before waiting for the scores
-        bool row_out = false;   // a query row past T (MODE 0, last tile only)
         if (MODE == 0) {
-          const int qi = t * 128 + r;
-          row_out = qi >= T;
-          row_lse2 = row_out ? 0.f : __ldg(lse_bh + qi) * LOG2E;
-          row_D = row_out ? 0.f : __ldg(D_bh + qi);
+          // the 32 queries of this warp's columns: lane i stages query t*128 + c0 + i's scalars
+          // (a query past T gets P = 0), then every lane reads all 32 of them
+          const int qi = t * 128 + c0 + lane;
+          const float nl = (qi < T) ? -__ldg(lse_bh + qi) * LOG2E : -INFINITY;
+          const float nd = (qi < T) ? -__ldg(D_bh + qi) : 0.f;
+          __syncwarp();                            // the previous tile's reads of vec are done
+          vec[lane] = nl;
+          vec[32 + lane] = nd;
+          __syncwarp();
         }
-        if (!mbar_wait(sd_full, g & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(sd_full, g & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        // causal mask on the diagonal tile: MODE 0 drops queries before key r, MODE 1 keys after
+        // query r.  There a warp's whole 32 x 32 chunk is masked when its columns all lie on the
+        // masked side of its 32 rows (MODE 0: part < q; MODE 1: part > q): its P and dZ are zero
+        // and its scores are not read.
+        const bool diag = (t == w.tile);
+        const bool all_masked = diag && ((MODE == 0) ? (part < q) : (part > q));
         // this thread's 32 columns of S and dP, then the TMEM buffer is released at once
         uint32_t us[32], ud[32];
-        tmem_ld32(tmem + lane_off + S_C + c0, us);
-        tmem_ld32(tmem + lane_off + DP_C + c0, ud);
-        tmem_wait_ld();
+        if (!all_masked) {
+          tmem_ld32(tmem + lane_off + BS_C + c0, us);
+          tmem_ld32(tmem + lane_off + BDP_C + c0, ud);
+          tmem_wait_ld();
+        }
         tc_fence_before();
         mbar_arrive(sd_empty);
-        const bool diag = (t == w.tile);
-        const bool need_mask = diag || row_out;
-        const float2 nl = make_float2(-row_lse2, -row_lse2);
-        const float2 nd = make_float2(-row_D, -row_D);
         uint32_t pw[16], dw[16];
+        if (all_masked) {
+#pragma unroll
+          for (int d = 0; d < 16; ++d) pw[d] = dw[d] = 0u;
+        } else
 #pragma unroll
         for (int d = 0; d < 32; d += 2) {
           const int c = c0 + d;
+          float2 nl, nd;
+          if (MODE == 0) {
+            nl = *reinterpret_cast<const float2*>(vec + d);
+            nd = *reinterpret_cast<const float2*>(vec + 32 + d);
+          } else {
+            nl = make_float2(nl1, nl1);
+            nd = make_float2(nd1, nd1);
+          }
           const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
           float2 pp = make_float2(ex2(x.x), ex2(x.y));
-          if (need_mask) {
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int cm = c + h2;
-              const bool masked = row_out || (diag && cm > r);   // causal: key cm after query r
-              if (masked) (h2 ? pp.y : pp.x) = 0.f;
+          if (diag) {
+            if (MODE == 0) {
+              if (c < r) pp.x = 0.f;
+              if (c + 1 < r) pp.y = 0.f;
+            } else {
+              if (c > r) pp.x = 0.f;
+              if (c + 1 > r) pp.y = 0.f;
             }
           }
           const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])), nd));
           pw[d >> 1] = pack_bf16x2(pp.x, pp.y);
           dw[d >> 1] = pack_bf16x2(gz.x, gz.y);
         }
-        // the previous tile's MMAs must be done reading the P / dZ operands
-        if (!mbar_wait(ps_empty, (g & 1) ^ 1, abort_flag)) { ok = false; break; }
-        if (MODE == 0) store_32_sw128(sP, r, c0, pw);
-        store_32_sw128(sDS, r, c0, dw);
-        fence_async_smem();
+        // the previous tile's MMAs must be done reading P / dZ in TMEM
+        if (!mbar_wait_warp(ps_empty, (g & 1) ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (MODE == 0) tmem_st16(tmem + lane_off + BP_C + (c0 >> 1), pw);
+        tmem_st16(tmem + lane_off + BDS_C + (c0 >> 1), dw);
+        tmem_wait_st();
+        tc_fence_before();
         mbar_arrive(ps_full);
         // the previous item's epilogue runs once this item's first tile is handed over, so
         // its wait for the last accumulation overlaps this item's products
@@ -869,7 +911,7 @@ int encode_rows64(CUtensorMap* tm, const void* base, int cols, long long rows) {
 
 // Tensor-core backward for head size 64 in bf16 (D = rowsum(dO * O) precomputed).
 int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const float* lse, const float* Dbuf,
-                       void* dqkv, int B, int T, int H, int hd) {
+                       void* dqkv, int B, int T, int H, int hd, float* bias_part) {
   if (hd != HD) return -4;
   if ((reinterpret_cast<uintptr_t>(dqkv) & 15) != 0) return -1;   // 16-byte stores of dQ, dK, dV
   const int C = H * HD;
@@ -878,30 +920,18 @@ int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const
   if (rc) return rc;
   rc = encode_rows64(&td, dout, C, (long long)B * T);
   if (rc) return rc;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(attn_bwd_tc_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, BWD_SMEM) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(attn_bwd_tc_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, BWD_SMEM) !=
-            cudaSuccess)
-      return -3;
-    attr = true;
-  }
-  static int nsm = 0;
-  if (nsm == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    if (nsm <= 0) nsm = 148;
-  }
+  if (set_dynamic_smem_once((const void*)attn_bwd_tc_kernel<0>, BWD_SMEM) ||
+      set_dynamic_smem_once((const void*)attn_bwd_tc_kernel<1>, BWD_SMEM))
+    return -3;
+  const int nsm = current_device_sms();
   const int items = cdiv(T, 128) * B * H;
   const int grid = items < nsm ? items : nsm;   // persistent: one CTA per SM
   const float scale = 1.0f / sqrtf((float)HD);
   const float scale_log2 = 1.4426950408889634f * scale;
-  attn_bwd_tc_kernel<0><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv), B, T,
-                                                             H, scale, scale_log2);
-  attn_bwd_tc_kernel<1><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv), B, T,
-                                                             H, scale, scale_log2);
+  attn_bwd_tc_kernel<0><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv),
+                                                             bias_part, B, T, H, scale, scale_log2);
+  attn_bwd_tc_kernel<1><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv),
+                                                             bias_part, B, T, H, scale, scale_log2);
   note_kernel_launches(2);
   return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }

@@ -181,6 +181,7 @@ struct EpiRing {
   uint8_t* boxes;
   uint64_t* bars;
   uint32_t phases;          // bit i: parity of the next completion of bars[i]
+  uint32_t inflight;        // bit i: a load into box i not yet waited for
   int alloc;                // boxes handed out so far
   int stores;               // store groups committed so far
   volatile int* abort_flag;
@@ -199,15 +200,27 @@ struct EpiRing {
     return a % NB;
   }
   __device__ __forceinline__ void issue_load(int i, const CUtensorMap* map, int x, int y) {
+    inflight |= 1u << i;
     if (lane == 0) {
       mbar_arrive_expect_tx(&bars[i], BOX_BYTES);
       tma_load_2d(box(i), map, x, y, &bars[i]);
     }
   }
+  // the whole warp waits (warp-uniform outcome)
   __device__ __forceinline__ bool wait_load(int i) {
-    const bool ok = mbar_wait(&bars[i], (phases >> i) & 1u, abort_flag);
-    phases ^= 1u << i;
+    const bool ok = mbar_wait_warp(&bars[i], (phases >> i) & 1u, abort_flag);
+    if (ok) {
+      phases ^= 1u << i;
+      inflight &= ~(1u << i);
+    }
     return ok;
+  }
+  // after an abort: lets the loads still in flight land before the CTA leaves
+  __device__ __forceinline__ void drain() {
+    if (lane == 0)
+      for (int i = 0; i < NB; ++i)
+        if ((inflight >> i) & 1u) mbar_drain(&bars[i], (phases >> i) & 1u);
+    __syncwarp();
   }
   __device__ __forceinline__ void store(int i, const CUtensorMap* map, int x, int y) {
     fence_proxy_async_smem();
@@ -282,6 +295,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // ------------------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
+      int issued = 0;            // stages filled so far
       bool ok = true;
       // this CTA's rows of A and of B within a tile; with a CTA pair both halves complete
       // on the leader's full barrier, which the leader arms for the bytes of both
@@ -312,8 +326,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int j = 0; j < Cfg::B_ROWS / 64; ++j) load(sB + j * 8192, &tmB, n0 + 64 * j, k0, stage);
           }
           if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1; }
+          ++issued;
         }
       }
+      // after an abort, the loads still in flight land before the CTA leaves (the leader's
+      // full barriers count the bytes of both CTAs of a pair)
+      if (*abort_flag && rank == 0)
+        for (int s = 0; s < Cfg::STAGES && s < issued; ++s) {
+          const int fills = (issued - 1 - s) / Cfg::STAGES + 1;
+          mbar_drain(&full_bar[s], (uint32_t)((fills - 1) & 1));
+        }
     }
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
@@ -368,6 +390,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     E.boxes = stg + ew * NB * BOX_BYTES;
     E.bars = &epi_bar[ew * NB];
     E.phases = 0;
+    E.inflight = 0;
     E.alloc = 0;
     E.stores = 0;
     E.abort_flag = abort_flag;
@@ -413,7 +436,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int c = 0; c < min(depth, nch); ++c) load_chunk(c);
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0.0f, 0x7fffffff};
       const int y_row = (kind == EPI_CE_FWD && m < ep.M) ? ep.targets[m] : -1;
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
+      if (!mbar_wait_warp(&tfull_bar[acc], acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < nch && ok; ++c) {
@@ -518,6 +541,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       acc ^= 1;
       if (acc == 0) acc_phase ^= 1;
     }
+    if (!ok) E.drain();
     if (lane == 0) bulk_wait_group<0>();      // every store of this warp has landed
     __syncwarp();
   }
@@ -620,12 +644,11 @@ int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, con
               const CUtensorMap& tin, const CUtensorMap& tout2, TileSched sched, const EpiParams& ep, int num_sms) {
   using Cfg = TileCfg<BN, CG>;
   auto kern = gemm_tc_kernel<BN, A_MN, B_MN, CG>;
-  static bool attr_set = false;
-  static int max_groups = 0;   // co-resident CTA groups of this kernel
-  if (!attr_set) {
+  // co-resident CTA groups of this kernel on the current device (its shared-memory limit set)
+  const int max_groups = per_device_once((const void*)kern, [&]() -> int {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
       return -3;
-    max_groups = num_sms / CG;
+    int groups = num_sms / CG;
     if (CG == 2) {
       cudaLaunchConfig_t cfg{};
       cudaLaunchAttribute at[1];
@@ -633,17 +656,18 @@ int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, con
       at[0].val.clusterDim.x = 2;
       at[0].val.clusterDim.y = 1;
       at[0].val.clusterDim.z = 1;
-      cfg.gridDim = dim3(2 * max_groups);
+      cfg.gridDim = dim3(2 * groups);
       cfg.blockDim = dim3(NUM_THREADS);
       cfg.dynamicSmemBytes = Cfg::SMEM;
       cfg.attrs = at;
       cfg.numAttrs = 1;
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return -3;
-      if (n < max_groups) max_groups = n;
+      if (n < groups) groups = n;
     }
-    attr_set = true;
-  }
+    return groups;
+  });
+  if (max_groups <= 0) return -3;
   const int tiles = sched.m_tiles * sched.n_tiles * sched.splits;
   const int groups = tiles < max_groups ? tiles : max_groups;
   if (CG == 1) {

@@ -109,10 +109,12 @@ struct gpt2_ctx {
   void* dqkv = nullptr;
   void* dattn = nullptr;
   float* attnD = nullptr;
+  float* attn_bias_part = nullptr;   // c_attn bias column sums from the attention backward
   float* ln_part = nullptr;
   int ln_blocks = 0;
   float* colsum_part = nullptr;
-  uint32_t* enc_sorted = nullptr;
+  uint64_t* enc_sorted = nullptr;
+  uint32_t* enc_seg = nullptr;
   float* enc_part = nullptr;
   float* splitk_ws = nullptr;
   size_t splitk_ws_elems = 0;
@@ -477,16 +479,24 @@ int backward_impl(gpt2_ctx* c) {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * Cd * Cd, 0);
       RC(gemm(c, N, C, C, c->dres_act, C, false, W(c, pi(PROJ_W)), C, true, e));
     }
+    // the tensor-core path also leaves the column sums of dqkv (the c_attn bias gradient) per
+    // 32-row group, so dqkv is not read again for them
+    const bool fused_qkv_bias = c->attn_bias_part != nullptr;
     {
       PROF(PROF_ATTN_BWD, 4.0 * B * (double)T * T * Cd, 0);
-      RC(launch_attn_bwd(st, c->bf16, a.qkv, a.attn, c->dattn, a.attn_lse, c->attnD, c->dqkv, B, T, H, hd));
+      RC(launch_attn_bwd(st, c->bf16, a.qkv, a.attn, c->dattn, a.attn_lse, c->attnD, c->dqkv, B, T, H, hd,
+                         fused_qkv_bias ? c->attn_bias_part : nullptr));
     }
     e = epi_make(EPI_ACCUM_F32, G(c, pi(ATTN_W)), C);
     {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * 3 * Cd * Cd, 0);
       RC(gemm(c, 3 * C, C, N, c->dqkv, 3 * C, true, a.ln1, C, true, e));
     }
-    {
+    if (fused_qkv_bias) {
+      const int rows = attn_bwd_bias_rows(B, T);
+      PROF(PROF_BIAS, 0, 4.0 * rows * 3 * Cd);
+      RC(launch_colsum_reduce(st, c->attn_bias_part, rows, 3 * C, G(c, pi(ATTN_B))));
+    } else {
       PROF(PROF_BIAS, 0, A * Nd * 3 * Cd);
       RC(launch_colsum(st, c->bf16, c->dqkv, 3 * C, N, 3 * C, c->colsum_part, ncs, G(c, pi(ATTN_B))));
     }
@@ -506,7 +516,7 @@ int backward_impl(gpt2_ctx* c) {
   // token + position embedding
   {
     PROF(PROF_EMBED, 0, 8.0 * Nd * Cd + 8.0 * T * Cd);
-    RC(launch_encoder_bwd(st, c->tokens, c->dres, G(c, 0), G(c, 1), B, T, C, c->enc_sorted, c->enc_part,
+    RC(launch_encoder_bwd(st, c->tokens, c->dres, G(c, 0), G(c, 1), B, T, C, c->enc_sorted, c->enc_seg, c->enc_part,
                           g.vocab_size));
   }
   return GPT2_OK;
@@ -522,7 +532,7 @@ int validate_cfg(const gpt2_config* g) {
   const int hd = g->n_embd / g->n_head;
   if (hd != 16 && hd != 32 && hd != 64) return GPT2_ERR_SHAPE;
   if (g->n_embd % 32 || g->n_embd > 1024) return GPT2_ERR_SHAPE;
-  if ((long long)g->max_batch * g->block_size > 32768) return GPT2_ERR_SHAPE;
+  if ((long long)g->max_batch * g->block_size > ENC_MAX_POSITIONS) return GPT2_ERR_SHAPE;
   if (g->padded_vocab_size >= 131072) return GPT2_ERR_SHAPE;
   return GPT2_OK;
 }
@@ -688,19 +698,27 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
   AL(dalloc_bytes(c, &c->dqkv, N * 3 * C * A));
   AL(dalloc_bytes(c, &c->dattn, N * C * A));
   AL(dalloc(c, &c->attnD, N * H));
+  if (c->bf16 && C / H == 64)
+    AL(dalloc(c, &c->attn_bias_part, (size_t)attn_bwd_bias_rows(g.max_batch, g.block_size) * 3 * C));
   c->ln_blocks = layernorm_bwd_blocks(c->num_sms);
   AL(dalloc(c, &c->ln_part, (size_t)c->ln_blocks * 3 * C));
   AL(dalloc(c, &c->colsum_part, (size_t)colsum_chunks((int)N) * 4 * C));
   AL(dalloc(c, &c->enc_sorted, N));
+  AL(dalloc(c, &c->enc_seg, encoder_bwd_seg_words((int)N)));
   AL(dalloc(c, &c->enc_part, encoder_bwd_part_floats((int)N, (int)C)));
   c->splitk_ws_elems = (size_t)8 * 4 * C * C;
   AL(dalloc(c, &c->splitk_ws, c->splitk_ws_elems));
   c->norm_nparts = 4 * c->num_sms;
   AL(dalloc(c, &c->norm_part, c->norm_nparts));
   {
-    // AdamW block table: each tensor split into blocks of 8192 elements
+    // AdamW block table: each tensor split into blocks of 8192 elements; the kernel's 16-byte
+    // accesses need every block to start and end on a multiple of 4 elements
     std::vector<AdamBlock> blocks;
-    for (const ParamView& v : c->views)
+    for (const ParamView& v : c->views) {
+      if (v.off % 4 || v.n % 4) {
+        rc = GPT2_ERR_SHAPE;
+        goto fail_out;
+      }
       for (long long o = 0; o < v.n; o += 8192) {
         AdamBlock b;
         b.off = v.off + o;
@@ -708,6 +726,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
         b.decay = v.decay;
         blocks.push_back(b);
       }
+    }
     c->n_adam_blocks = (int)blocks.size();
     AL(dalloc(c, &c->adam_blocks, blocks.size()));
     if (cudaMemcpy(c->adam_blocks, blocks.data(), blocks.size() * sizeof(AdamBlock), cudaMemcpyHostToDevice) !=

@@ -14,7 +14,43 @@
 __device__ int g_device_error = 0;
 
 #include <atomic>
+#include <map>
+#include <mutex>
+#include <utility>
 static std::atomic<long long> g_kernel_launches{0};
+
+int per_device_once(const void* key, const std::function<int()>& compute) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -3;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto k = std::make_pair(key, dev);
+  const auto it = cache.find(k);
+  if (it != cache.end()) return it->second;
+  const int v = compute();
+  if (v >= 0) cache[k] = v;
+  return v;
+}
+
+int current_device_sms() {
+  static const int tag = 0;
+  const int n = per_device_once(&tag, [] {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                     cudaSuccess || sms <= 0)
+      return -3;
+    return sms;
+  });
+  return n > 0 ? n : 148;
+}
+
+int set_dynamic_smem_once(const void* func, int bytes) {
+  const int rc = per_device_once(func, [=] {
+    return cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess ? 1 : -3;
+  });
+  return rc < 0 ? -3 : 0;
+}
 void note_kernel_launches(int n) { g_kernel_launches.fetch_add(n, std::memory_order_relaxed); }
 long long kernel_launch_count() { return g_kernel_launches.load(std::memory_order_relaxed); }
 
@@ -471,16 +507,21 @@ __global__ void __launch_bounds__(512) ce_dz_bf16x8_kernel(uint4* __restrict__ z
 // dwte[v] += sum of dx0 rows at positions holding token v; dwpe[t] += sum_b dx0[b, t]
 // (L9, "Code you'll write": wte and wpe receive the gradient of the residual stream at
 // the first block's input; wte's share adds to the lm_head's, the weight being tied).
-// Deterministic, with no atomics: the (token, position) keys are sorted in one CTA; runs of
-// equal tokens are summed in position order inside fixed ENC_CHUNK-entry chunks; a run that
+// Deterministic, with no atomics.  The (token, position) keys are put in order in two steps:
+// CTAs sort segments of at most ENC_SEG consecutive positions each, then every key finds its
+// place in the whole order by binary searches in the other segments (a merge by ranks).  Runs
+// of equal tokens are summed in position order inside fixed ENC_CHUNK-entry chunks; a run that
 // crosses chunk boundaries is finished by the chunk where it starts, which adds the later
 // chunks' partial sums through eight interleaved accumulators combined in a fixed order.
 constexpr int ENC_CHUNK = 32;
-constexpr int ENC_POS_BITS = 15;   // positions < 32768
 constexpr int ENC_SORT_THREADS = 1024;
+constexpr int ENC_SEG = 4096;        // positions per sorted segment (4 keys per thread)
+constexpr int ENC_SEG_BITS = 12;     // a position inside a segment
+constexpr int ENC_MAX_TOKENS = 1 << (32 - ENC_SEG_BITS);   // ids below 2^20 in a segment key
 
-__device__ __forceinline__ int key_tok(uint32_t k) { return static_cast<int>(k >> ENC_POS_BITS); }
-__device__ __forceinline__ int key_pos(uint32_t k) { return static_cast<int>(k & ((1u << ENC_POS_BITS) - 1)); }
+// whole-order keys: token << 32 | position
+__device__ __forceinline__ int key_tok(uint64_t k) { return static_cast<int>(k >> 32); }
+__device__ __forceinline__ int key_pos(uint64_t k) { return static_cast<int>(k & 0xFFFFFFFFull); }
 // one spare word after every 32, so that a warp reading E consecutive keys per lane
 // (E a power of two up to 32) hits 32 distinct banks
 __device__ __forceinline__ int enc_pad(int i) { return i + (i >> 5); }
@@ -509,22 +550,26 @@ __device__ __forceinline__ void enc_reg_stages(uint32_t (&r)[E], int base, int j
   if constexpr (E > 1) if (j == 1) enc_reg_stage<1>(r, base, k);
 }
 
-// Bitonic sort of P = 1024 E keys (tokens clamped to [0, V), key = token << 15 | position;
-// 0xFFFFFFFF past N).  Thread t keeps keys tE .. tE + E-1 in registers: a compare-exchange
-// at distance j < E stays in the thread, E <= j < 32E is one warp shuffle per key, and only
-// the longer distances go through shared memory (15 of the 105 stages for P = 16384).
+// Bitonic sort of one segment: CTA s takes positions [sP, sP + P), P = 1024 E <= ENC_SEG
+// (tokens clamped to [0, V), key = token << 12 | position - sP; 0xFFFFFFFF past N) and writes
+// the segment's keys in order to seg_keys[sP ..].  Thread t keeps keys tE .. tE + E-1 in
+// registers: a compare-exchange at distance j < E stays in the thread, E <= j < 32E is one
+// warp shuffle per key, and only the longer distances go through shared memory.
 template <int E>
 __global__ void __launch_bounds__(ENC_SORT_THREADS) enc_sort_kernel(const int* __restrict__ tok, int N, int V,
-                                                                     uint32_t* __restrict__ sorted) {
+                                                                     uint32_t* __restrict__ seg_keys) {
   constexpr int P = ENC_SORT_THREADS * E;
+  static_assert(P <= ENC_SEG, "segment larger than its position field");
   extern __shared__ uint32_t s[];   // enc_pad(P) words
   const int tid = threadIdx.x;
+  const int p0 = blockIdx.x * P;
+  const int n = min(P, N - p0);
   for (int i = tid; i < P; i += ENC_SORT_THREADS) {
     uint32_t key = 0xFFFFFFFFu;
-    if (i < N) {
-      int t = tok[i];
+    if (i < n) {
+      int t = tok[p0 + i];
       t = t < 0 ? 0 : (t >= V ? V - 1 : t);
-      key = (static_cast<uint32_t>(t) << ENC_POS_BITS) | static_cast<uint32_t>(i);
+      key = (static_cast<uint32_t>(t) << ENC_SEG_BITS) | static_cast<uint32_t>(i);
     }
     s[enc_pad(i)] = key;
   }
@@ -567,7 +612,36 @@ __global__ void __launch_bounds__(ENC_SORT_THREADS) enc_sort_kernel(const int* _
 #pragma unroll
   for (int e = 0; e < E; ++e) s[enc_pad(base + e)] = r[e];
   __syncthreads();
-  for (int i = tid; i < N; i += ENC_SORT_THREADS) sorted[i] = s[enc_pad(i)];
+  for (int i = tid; i < n; i += ENC_SORT_THREADS) seg_keys[p0 + i] = s[enc_pad(i)];
+}
+
+// Merge by ranks: the key at index i of segment s (segment size P) goes to index i + (keys of
+// every earlier segment with a token <= its token) + (keys of every later segment with a
+// token < its token).  Equal tokens thus keep segment order, and inside a segment position
+// order, so the whole is the stable (token, position) order.  One thread per key.
+__global__ void __launch_bounds__(256) enc_merge_kernel(const uint32_t* __restrict__ seg_keys, int N, int P,
+                                                        int nseg, uint64_t* __restrict__ sorted) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= N) return;
+  const int s = i / P;
+  const uint32_t key = seg_keys[i];
+  const uint32_t t = key >> ENC_SEG_BITS;
+  long long dst = i - (long long)s * P;
+  for (int s2 = 0; s2 < nseg; ++s2) {
+    if (s2 == s) continue;
+    const uint32_t* a = seg_keys + (long long)s2 * P;
+    const int n2 = min(P, N - s2 * P);
+    const uint32_t bound = (s2 < s ? t + 1 : t) << ENC_SEG_BITS;   // count the keys below it
+    int lo = 0, hi = n2;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(a + mid) < bound) lo = mid + 1;
+      else hi = mid;
+    }
+    dst += lo;
+  }
+  const uint32_t pos = static_cast<uint32_t>(s * P) + (key & ((1u << ENC_SEG_BITS) - 1));
+  sorted[dst] = (static_cast<uint64_t>(t) << 32) | pos;
 }
 
 // One block per chunk of ENC_CHUNK sorted keys; thread x sums channels 4x .. 4x+3 of the
@@ -575,7 +649,7 @@ __global__ void __launch_bounds__(ENC_SORT_THREADS) enc_sort_kernel(const int* _
 // is a whole run goes straight into dwte; otherwise it is stored as the chunk's partial:
 // slot 0 for the segment at the chunk's start, slot 1 for a run that starts later and
 // leaves through the chunk's end.
-__global__ void __launch_bounds__(256) enc_chunk_kernel(const uint32_t* __restrict__ sorted,
+__global__ void __launch_bounds__(256) enc_chunk_kernel(const uint64_t* __restrict__ sorted,
                                                         const float* __restrict__ dx0, float* __restrict__ dwte,
                                                         float* __restrict__ part, int N, int C) {
   __shared__ int tk[ENC_CHUNK + 2];   // tk[1 + i]: token of the chunk's i-th key; tk[0], tk[n + 1]: neighbours or -1
@@ -586,7 +660,7 @@ __global__ void __launch_bounds__(256) enc_chunk_kernel(const uint32_t* __restri
     const int i = i0 - 1 + x;
     int t = -1;
     if (i >= 0 && i < N && x <= n + 1) {
-      const uint32_t key = sorted[i];
+      const uint64_t key = sorted[i];
       t = key_tok(key);
       if (x >= 1 && x <= n) ps[x - 1] = key_pos(key);
     }
@@ -630,7 +704,7 @@ __global__ void __launch_bounds__(256) enc_chunk_kernel(const uint32_t* __restri
 // The chunk where a boundary-crossing run starts adds its own partial and, over eight
 // interleaved accumulators (chunk c + 1 + q goes to accumulator q mod 8, each in chunk
 // order, then accumulators 0..7 in turn), slot 0 of every later chunk the run covers.
-__global__ void __launch_bounds__(256) enc_fixup_kernel(const uint32_t* __restrict__ sorted,
+__global__ void __launch_bounds__(256) enc_fixup_kernel(const uint64_t* __restrict__ sorted,
                                                         float* __restrict__ dwte, const float* __restrict__ part,
                                                         int N, int C, int nchunks) {
   __shared__ int last_chunk;
@@ -804,15 +878,29 @@ __global__ void __launch_bounds__(256) dwpe_kernel(const float4* __restrict__ dx
 __global__ void __launch_bounds__(512) sumsq_kernel(const float* __restrict__ g, long long n,
                                                     double* __restrict__ part) {
   __shared__ double sd[512];
-  double s = 0.0;
+  // four independent 16-byte loads in flight per thread, each squared in fp32 and summed in
+  // double along its own chain; the chains and then the threads are added in a fixed order
+  double s4[4] = {0.0, 0.0, 0.0, 0.0};
   const long long n4 = n / 4;
   const float4* g4 = reinterpret_cast<const float4*>(g);
-  for (long long i = blockIdx.x * 512LL + threadIdx.x; i < n4; i += (long long)gridDim.x * 512) {
-    const float4 v = g4[i];
-    s += (double)(v.x * v.x) + (double)(v.y * v.y) + (double)(v.z * v.z) + (double)(v.w * v.w);
+  const long long stride = (long long)gridDim.x * 512;
+  long long i = blockIdx.x * 512LL + threadIdx.x;
+  for (; i + 3 * stride < n4; i += 4 * stride) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldcs(g4 + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      s4[u] += (double)(v[u].x * v[u].x) + (double)(v[u].y * v[u].y) + (double)(v[u].z * v[u].z) +
+               (double)(v[u].w * v[u].w);
   }
+  for (; i < n4; i += stride) {
+    const float4 v = __ldcs(g4 + i);
+    s4[0] += (double)(v.x * v.x) + (double)(v.y * v.y) + (double)(v.z * v.z) + (double)(v.w * v.w);
+  }
+  double s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
   if (blockIdx.x == 0)
-    for (long long i = n4 * 4 + threadIdx.x; i < n; i += 512) s += (double)g[i] * (double)g[i];
+    for (long long j = n4 * 4 + threadIdx.x; j < n; j += 512) s += (double)g[j] * (double)g[j];
   sd[threadIdx.x] = s;
   __syncthreads();
   for (int o = 256; o > 0; o >>= 1) {
@@ -841,6 +929,18 @@ __global__ void norm_finalize_kernel(const double* __restrict__ part, int nparts
 // AdamW with decoupled weight decay and bias correction (torch.optim.AdamW semantics; L9
 // "2:14:58 – 2:25:57" betas/eps, "2:25:57 – 2:34:49" decay on >= 2-D tensors only).
 // One launch updates every tensor; each block reads its (offset, count, decay) entry.
+// Blocks start on 16-byte boundaries and hold a multiple of 4 elements (every tensor size is
+// a multiple of n_embd), so each thread moves 4 elements per access with 16-byte loads and
+// stores, two groups in flight (p, g, m and v: eight loads).
+__device__ __forceinline__ float adamw_one(float& mi, float& vi, float pi, float gi, float s, float b1, float b2,
+                                           float lr, float eps, float decay, float bc1, float bc2) {
+  gi *= s;
+  mi = b1 * mi + (1.0f - b1) * gi;
+  vi = b2 * vi + (1.0f - b2) * gi * gi;
+  const float mh = mi / bc1;
+  const float vh = vi / bc2;
+  return pi * decay - lr * mh / (sqrtf(vh) + eps);
+}
 __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const float* __restrict__ g,
                                                     float* __restrict__ m, float* __restrict__ v,
                                                     bf16* __restrict__ shadow, const AdamBlock* __restrict__ blocks,
@@ -849,18 +949,39 @@ __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, const
   const AdamBlock blk = blocks[blockIdx.x];
   const float s = *clip_scale;
   const float decay = blk.decay ? (1.0f - lr * wd) : 1.0f;
-  for (int i = threadIdx.x; i < blk.n; i += blockDim.x) {
-    const long long idx = blk.off + i;
-    const float gi = g[idx] * s;
-    const float mi = b1 * m[idx] + (1.0f - b1) * gi;
-    const float vi = b2 * v[idx] + (1.0f - b2) * gi * gi;
-    const float mh = mi / bc1;
-    const float vh = vi / bc2;
-    const float pi = p[idx] * decay - lr * mh / (sqrtf(vh) + eps);
-    p[idx] = pi;
-    m[idx] = mi;
-    v[idx] = vi;
-    if (shadow != nullptr && blk.decay) shadow[idx] = __float2bfloat16_rn(pi);
+  const bool write_shadow = shadow != nullptr && blk.decay;
+  float4* p4 = reinterpret_cast<float4*>(p + blk.off);
+  const float4* g4 = reinterpret_cast<const float4*>(g + blk.off);
+  float4* m4 = reinterpret_cast<float4*>(m + blk.off);
+  float4* v4 = reinterpret_cast<float4*>(v + blk.off);
+  uint2* sh4 = reinterpret_cast<uint2*>(shadow + blk.off);
+  const int n4 = blk.n >> 2;
+  for (int i0 = threadIdx.x; i0 < n4; i0 += 2 * blockDim.x) {
+    float4 pv[2], gv[2], mv[2], vv[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < n4) {
+        pv[u] = p4[i];
+        gv[u] = __ldcs(g4 + i);
+        mv[u] = __ldcs(m4 + i);
+        vv[u] = __ldcs(v4 + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i >= n4) continue;
+      float4 o;
+      o.x = adamw_one(mv[u].x, vv[u].x, pv[u].x, gv[u].x, s, b1, b2, lr, eps, decay, bc1, bc2);
+      o.y = adamw_one(mv[u].y, vv[u].y, pv[u].y, gv[u].y, s, b1, b2, lr, eps, decay, bc1, bc2);
+      o.z = adamw_one(mv[u].z, vv[u].z, pv[u].z, gv[u].z, s, b1, b2, lr, eps, decay, bc1, bc2);
+      o.w = adamw_one(mv[u].w, vv[u].w, pv[u].w, gv[u].w, s, b1, b2, lr, eps, decay, bc1, bc2);
+      p4[i] = o;
+      __stcs(m4 + i, mv[u]);
+      __stcs(v4 + i, vv[u]);
+      if (write_shadow) sh4[i] = make_uint2(pack_bf16x2(o.x, o.y), pack_bf16x2(o.z, o.w));
+    }
   }
 }
 
@@ -962,13 +1083,7 @@ int ln_fwd_dispatch(cudaStream_t st, const float* x, const float* w, const float
   // 16-byte path: x, w, b, y 16-byte aligned and C a multiple of 128
   const bool vec = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(b) |
                      reinterpret_cast<uintptr_t>(y)) % 16) == 0;
-  static int nsm = 0;
-  if (nsm == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    if (nsm <= 0) nsm = 148;
-  }
+  const int nsm = current_device_sms();
   const int vgrid = grid < nsm * 2 ? grid : nsm * 2;   // 2 resident blocks per SM (registers), rows strided
   if (vec && (C == 768 || C == 1024 || C == 512 || C == 384 || C == 256 || C == 128)) {
     switch (C) {
@@ -1179,6 +1294,13 @@ int launch_colsum(cudaStream_t st, bool is_bf16, const void* x, long long ldx, i
   return ok();
 }
 
+int launch_colsum_reduce(cudaStream_t st, const float* part, int rows, int N, float* out) {
+  if (rows <= 0 || N <= 0) return -4;
+  colsum_reduce_kernel<<<cdiv(N, 32), 32 * CSR_GROUPS, 0, st>>>(part, rows, N, out);
+  note_kernel_launches(1);
+  return ok();
+}
+
 int launch_ce_finalize(cudaStream_t st, const CePartial* part, int n_tiles, const float* zt, const int* targets,
                        int N, int V, float* lse, float* loss_row, int* argmax) {
   ce_finalize_kernel<<<cdiv(N, 8), 256, 0, st>>>(part, n_tiles, zt, targets, N, V, lse, loss_row, argmax);
@@ -1204,13 +1326,7 @@ int launch_ce_dz(cudaStream_t st, bool is_bf16, void* logits, long long ld, cons
                  const float* dz_scale, int N, int Vp) {
   if (is_bf16 && Vp % 8 == 0 && ld % 8 == 0) {
     const int v8 = Vp / 8;
-    static int nsm = 0;
-    if (nsm == 0) {
-      int dev = 0;
-      cudaGetDevice(&dev);
-      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-      if (nsm <= 0) nsm = 148;
-    }
+    const int nsm = current_device_sms();
     const int grid = N < nsm * 4 ? N : nsm * 4;   // 4 blocks of 512 threads per SM
     ce_dz_bf16x8_kernel<<<grid, 512, 0, st>>>(reinterpret_cast<uint4*>(logits), ld / 8, lse, targets, dz_scale, v8,
                                               N);
@@ -1226,38 +1342,36 @@ int launch_ce_dz(cudaStream_t st, bool is_bf16, void* logits, long long ld, cons
 size_t encoder_bwd_part_floats(int N, int C) { return (size_t)cdiv(N, ENC_CHUNK) * 2 * (size_t)C; }
 
 template <int E>
-static int enc_sort_launch(cudaStream_t st, const int* tok, int N, int V, uint32_t* sorted) {
-  const int smem = (ENC_SORT_THREADS * E + ENC_SORT_THREADS * E / 32) * (int)sizeof(uint32_t);
-  if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(enc_sort_kernel<E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return -3;
-  enc_sort_kernel<E><<<1, ENC_SORT_THREADS, smem, st>>>(tok, N, V, sorted);
+static int enc_sort_launch(cudaStream_t st, const int* tok, int N, int V, uint32_t* seg_keys) {
+  constexpr int P = ENC_SORT_THREADS * E;
+  const int smem = (P + P / 32) * (int)sizeof(uint32_t);
+  if (smem > 48 * 1024 && set_dynamic_smem_once((const void*)enc_sort_kernel<E>, smem)) return -3;
+  enc_sort_kernel<E><<<cdiv(N, P), ENC_SORT_THREADS, smem, st>>>(tok, N, V, seg_keys);
   return 0;
 }
 
+size_t encoder_bwd_seg_words(int N) { return ((size_t)N + 63) / 64 * 64; }
+
 int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float* dwte, float* dwpe, int B, int T,
-                       int C, uint32_t* sorted_keys, float* chunk_part, int V) {
+                       int C, uint64_t* sorted_keys, uint32_t* seg_keys, float* chunk_part, int V) {
   const long long Nll = (long long)B * T;
-  if (B <= 0 || T <= 0 || Nll > (1 << ENC_POS_BITS) || V <= 0 || V > (1 << (32 - ENC_POS_BITS)) || C <= 0 ||
-      C % 4)
-    return -4;
+  if (B <= 0 || T <= 0 || Nll > ENC_MAX_POSITIONS || V <= 0 || V >= ENC_MAX_TOKENS || C <= 0 || C % 4) return -4;
   // 16-byte accesses to dx0, the gradients and the chunk partials
   if ((reinterpret_cast<uintptr_t>(dx0) | reinterpret_cast<uintptr_t>(dwte) | reinterpret_cast<uintptr_t>(dwpe) |
        reinterpret_cast<uintptr_t>(chunk_part)) % 16)
     return -1;
   const int N = (int)Nll;
+  // one segment of 1024 E keys for short inputs, segments of ENC_SEG keys otherwise
   int P = ENC_SORT_THREADS;
-  while (P < N) P <<= 1;
+  while (P < N && P < ENC_SEG) P <<= 1;
   int rc;
   switch (P / ENC_SORT_THREADS) {
-    case 1: rc = enc_sort_launch<1>(st, tok, N, V, sorted_keys); break;
-    case 2: rc = enc_sort_launch<2>(st, tok, N, V, sorted_keys); break;
-    case 4: rc = enc_sort_launch<4>(st, tok, N, V, sorted_keys); break;
-    case 8: rc = enc_sort_launch<8>(st, tok, N, V, sorted_keys); break;
-    case 16: rc = enc_sort_launch<16>(st, tok, N, V, sorted_keys); break;
-    default: rc = enc_sort_launch<32>(st, tok, N, V, sorted_keys); break;
+    case 1: rc = enc_sort_launch<1>(st, tok, N, V, seg_keys); break;
+    case 2: rc = enc_sort_launch<2>(st, tok, N, V, seg_keys); break;
+    default: rc = enc_sort_launch<4>(st, tok, N, V, seg_keys); break;
   }
   if (rc) return rc;
+  enc_merge_kernel<<<cdiv(N, 256), 256, 0, st>>>(seg_keys, N, P, cdiv(N, P), sorted_keys);
   const int nchunks = cdiv(N, ENC_CHUNK);
   const int c4 = C / 4;
   const int threads = c4 <= 256 ? (c4 + 31) / 32 * 32 : 256;
@@ -1267,7 +1381,7 @@ int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float*
   const int tc4 = T * c4;
   dwpe_kernel<<<grid_for(tc4, 256), 256, 0, st>>>(reinterpret_cast<const float4*>(dx0),
                                                   reinterpret_cast<float4*>(dwpe), B, tc4);
-  note_kernel_launches(4);
+  note_kernel_launches(5);
   return ok();
 }
 

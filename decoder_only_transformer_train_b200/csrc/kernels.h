@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <functional>
 #include "gemm.h"
 
 // Device error code of the top-k sampling kernel, next to the codes of the training step
@@ -35,9 +36,14 @@ int launch_loss_reduce(cudaStream_t st, const float* loss_row, const int* target
                        float* loss_out, float* dz_scale_out, int* count_out);
 int launch_ce_dz(cudaStream_t st, bool bf16, void* logits, long long ld, const float* lse, const int* targets,
                  const float* dz_scale, int N, int Vp);
+// Positions one embedding backward may take (B*T).
+constexpr int ENC_MAX_POSITIONS = 131072;
+// sorted_keys: N uint64 (token << 32 | position, ascending); seg_keys: encoder_bwd_seg_words(N)
+// uint32 of scratch; chunk_part: encoder_bwd_part_floats(N, C) floats.
 int launch_encoder_bwd(cudaStream_t st, const int* tok, const float* dx0, float* dwte, float* dwpe, int B, int T,
-                       int C, uint32_t* sorted_keys, float* chunk_part, int V);
+                       int C, uint64_t* sorted_keys, uint32_t* seg_keys, float* chunk_part, int V);
 size_t encoder_bwd_part_floats(int N, int C);
+size_t encoder_bwd_seg_words(int N);
 int launch_topk_sample(cudaStream_t st, bool is_bf16, const void* logits, long long ld, int n_rows, const int* rows,
                        const float* u, int n, int V, int k, int* out, int* out_topk);
 int launch_global_norm(cudaStream_t st, const float* g, long long n, double* part, int nparts, float clip,
@@ -50,12 +56,27 @@ int launch_fill(cudaStream_t st, float* p, long long n, float value);
 int launch_cast_bf16(cudaStream_t st, const float* src, uint16_t* dst, long long n);
 int launch_attn_fwd(cudaStream_t st, bool bf16, const void* qkv, void* out, float* lse, int B, int T, int H,
                     int hd);
+// bias_part (may be null; the bf16 head-size-64 path only): column sums of dqkv per 32-row
+// lane quarter of each 128-row tile, attn_bwd_bias_rows(B, T) rows of 3C floats, to be
+// reduced by launch_colsum_reduce into the c_attn bias gradient.
 int launch_attn_bwd(cudaStream_t st, bool bf16, const void* qkv, const void* out, const void* dout,
-                    const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd);
+                    const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd,
+                    float* bias_part = nullptr);
 int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, int B, int T, int H, int hd);
 int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const float* lse, const float* Dbuf,
-                       void* dqkv, int B, int T, int H, int hd);
+                       void* dqkv, int B, int T, int H, int hd, float* bias_part);
+inline int attn_bwd_bias_rows(int B, int T) { return (T + 127) / 128 * B * 4; }
+// out[n] += sum over rows k of part[k * N + n], in a fixed order
+int launch_colsum_reduce(cudaStream_t st, const float* part, int rows, int N, float* out);
 int read_and_clear_device_error(int* code);
+// Host-side values computed once per (key, device) under a lock: a process may drive several
+// GPUs, from several threads, and a kernel attribute set on one device is unset on the others.
+// compute() runs with the key's device current; negative results are returned, not cached.
+int per_device_once(const void* key, const std::function<int()>& compute);
+int current_device_sms();   // SM count of the current device (148 if the query fails)
+// Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// device (0, or -3 if the runtime refuses).
+int set_dynamic_smem_once(const void* func, int bytes);
 // Host-side count of the kernels launched by this library (for benchmark reporting).
 void note_kernel_launches(int n);
 long long kernel_launch_count();

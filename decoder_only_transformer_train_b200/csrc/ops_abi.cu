@@ -101,21 +101,27 @@ int gpt2op_embedding_fwd(void* stream, const int32_t* tokens, const float* wte, 
   return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA));
 }
 
-static int64_t embedding_keys_bytes(int N) { return ((int64_t)N * 4 + 255) / 256 * 256; }
+// workspace of the embedding backward: the sorted keys (N uint64), the segment keys and the
+// chunk partials, each starting on a 256-byte boundary
+static int64_t round256(int64_t b) { return (b + 255) / 256 * 256; }
+static int64_t embedding_keys_bytes(int N) { return round256((int64_t)N * 8); }
+static int64_t embedding_seg_bytes(int N) { return round256((int64_t)encoder_bwd_seg_words(N) * 4); }
 
 int64_t gpt2op_embedding_bwd_ws_bytes(int N, int C) {
   if (N <= 0 || C <= 0) return 0;
-  return embedding_keys_bytes(N) + (int64_t)encoder_bwd_part_floats(N, C) * 4;
+  return embedding_keys_bytes(N) + embedding_seg_bytes(N) + (int64_t)encoder_bwd_part_floats(N, C) * 4;
 }
 
 int gpt2op_embedding_bwd(void* stream, const int32_t* tokens, const float* dx0, float* dwte, float* dwpe, int B,
                          int T, int C, int V, void* ws) {
   if (!tokens || !dx0 || !dwte || !dwpe || !ws) return GPT2_ERR_ARG;
-  if (B <= 0 || T <= 0 || C <= 0 || V <= 0 || C % 4 || (long long)B * T > 32768) return GPT2_ERR_SHAPE;
+  if (B <= 0 || T <= 0 || C <= 0 || V <= 0 || C % 4 || (long long)B * T > ENC_MAX_POSITIONS) return GPT2_ERR_SHAPE;
   char* w = static_cast<char*>(ws);
+  const int N = B * T;
   const int rc = launch_encoder_bwd(reinterpret_cast<cudaStream_t>(stream), tokens, dx0, dwte, dwpe, B, T, C,
-                                    reinterpret_cast<uint32_t*>(w),
-                                    reinterpret_cast<float*>(w + embedding_keys_bytes(B * T)), V);
+                                    reinterpret_cast<uint64_t*>(w),
+                                    reinterpret_cast<uint32_t*>(w + embedding_keys_bytes(N)),
+                                    reinterpret_cast<float*>(w + embedding_keys_bytes(N) + embedding_seg_bytes(N)), V);
   return rc == 0 ? GPT2_OK : (rc == -4 ? GPT2_ERR_SHAPE : (rc == -1 ? GPT2_ERR_ARG : GPT2_ERR_CUDA));
 }
 

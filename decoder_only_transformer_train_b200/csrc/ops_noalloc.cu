@@ -22,8 +22,10 @@
 
 namespace {
 
-// Fixed scratch: GPT2OP_NOALLOC_ATTN_MAX_ROWS floats (1 MiB), 256-byte aligned so that the
-// bulk copies of 128-row slices of D start on a 16-byte boundary.
+// Fixed scratch: GPT2OP_NOALLOC_ATTN_MAX_ROWS floats (1 MiB).  The kernels write and read D
+// one float per (batch, head, query) row, so float alignment is all they need; the array is
+// 256-byte aligned like cudaMalloc memory, so it meets anything the caller-scratch path may
+// assume of its D buffer.
 static __device__ __align__(256) float g_attn_rowsum_scratch[GPT2OP_NOALLOC_ATTN_MAX_ROWS];
 
 constexpr int kMaxDevices = 64;

@@ -43,8 +43,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait until the phase of parity `parity` has completed.  Returns false (and raises the
-// CTA abort flag) on timeout or if another role of the CTA already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// CTA abort flag) after limit_ns of waiting, or if another role of the CTA already aborted.
+// The calling lane decides alone: use it for single-lane roles (a TMA producer, an MMA
+// issuer), and mbar_wait_warp where a whole warp waits.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = SM100_TIMEOUT_NS) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -53,13 +56,49 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > SM100_TIMEOUT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       raise_device_error(DEVERR_TIMEOUT);
       *abort_flag = 1;
       return false;
     }
   }
 }
+// The same wait made by all 32 lanes of a warp together.  Each lane polls, then the warp
+// votes: it goes on only if every lane saw the phase complete, so all lanes leave together
+// even when one of them gave up first, and whatever follows (a warp-collective tcgen05.ld /
+// st, a shuffle, __syncwarp) finds the whole warp.  Every lane of the warp must call it.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               uint64_t limit_ns = SM100_TIMEOUT_NS) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// After an abort: wait, for at most limit_ns, until the phase of parity `parity` of a
+// barrier that still has copies in flight completes, so that no TMA write lands in shared
+// memory after the CTA has left.  Raises no error (the abort already did).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 100000000ull) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity))
+    if (globaltimer_ns() - t0 > limit_ns) return;
+}
+
+// The barriers (up to 32, addressed from `base`) on which a TMA producer has armed copies,
+// with the parity of each one's last armed phase: after an abort the producer waits for
+// those phases, so that no copy is still in flight when the CTA leaves.
+struct InflightTx {
+  uint64_t* base;
+  uint32_t armed, parity;
+  __device__ __forceinline__ void note(uint64_t* bar, uint32_t par) {
+    const int i = static_cast<int>(bar - base);
+    armed |= 1u << i;
+    parity = (parity & ~(1u << i)) | ((par & 1u) << i);
+  }
+  __device__ __forceinline__ void drain() const {
+    for (int i = 0; i < 32; ++i)
+      if ((armed >> i) & 1u) mbar_drain(base + i, (parity >> i) & 1u);
+  }
+};
 
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
@@ -139,6 +178,18 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uin
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T with A read from tensor memory: M rows on the lanes of
+// the accumulator, K along the columns, two bf16 per 32-bit column (the lower half holds the
+// even k); B from shared memory by descriptor.  Issued by one thread.
+__device__ __forceinline__ void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread completes.
@@ -230,7 +281,8 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint64_t limit_ns = SM100_TIMEOUT_NS) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait_cluster(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -239,7 +291,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait_cluster(a, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > SM100_TIMEOUT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       raise_device_error(DEVERR_TIMEOUT);
       *abort_flag = 1;
       return false;

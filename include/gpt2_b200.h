@@ -47,7 +47,7 @@ extern "C" {
  * the vocabulary padded to 50304; "2:34:49 – 2:46:43": gradient accumulation).
  * Constraints: n_embd % n_head == 0, head size in {16, 32, 64}, n_embd a multiple of 32
  * and at most 1024, vocab_size <= padded_vocab_size < 131072, max_batch * block_size
- * <= 32768. */
+ * <= 131072. */
 typedef struct {
   int n_layer;            /* 12 for GPT-2 124M */
   int n_embd;             /* 768 */
@@ -261,10 +261,10 @@ int gpt2op_layernorm_fwd(void* stream, int precision, const float* x, const floa
  * token v, dwpe[t] += sum over b of dx0[b*T + t]; ids are clamped into [0, V).  The sums
  * are deterministic (no atomics; a fixed order that depends only on the ids).  ws is
  * device scratch of gpt2op_embedding_bwd_ws_bytes(B*T, C) bytes, 256-byte aligned; after
- * the call its first B*T uint32 words hold the sort keys token << 15 | position in
+ * the call its first B*T uint64 words hold the sort keys token << 32 | position in
  * ascending order.  The f32 tables, x, dx0, dwte, dwpe and ws must be 16-byte aligned.
  * Both: GPT2_ERR_ARG for a null or misaligned pointer; GPT2_ERR_SHAPE unless B, T,
- * C, V > 0, C % 4 == 0, and for the backward B*T <= 32768 and V <= 131072. */
+ * C, V > 0, C % 4 == 0, and for the backward B*T <= 131072 and V < 2^20. */
 int gpt2op_embedding_fwd(void* stream, const int32_t* tokens, const float* wte, const float* wpe, float* x, int B,
                          int T, int C, int V);
 int64_t gpt2op_embedding_bwd_ws_bytes(int N, int C);
@@ -311,6 +311,16 @@ int gpt2op_classifier_fwd_bwd(void* stream, const void* h, const void* W, const 
 #define GPT2_PROF_OPTIM 11      /* global norm and AdamW */
 int gpt2_profile_start(gpt2_ctx* ctx);
 int gpt2_profile_stop(gpt2_ctx* ctx, double* ms, int64_t* launches, double* flops, double* bytes);
+
+/* Self-test of the bounded waits inside the pipelined kernels (no counterpart on the pages):
+ * one kernel in which a single lane and then a whole warp wait on mbarriers that nothing will
+ * ever complete, each for at most limit_ns (1 .. 1e9) nanoseconds.  Both waits must give up,
+ * record GPT2_ERR_TIMEOUT in the device error word (read it with gpt2op_device_error), let a
+ * 16-byte bulk copy from src16 that is still in flight land, and return; status (DEVICE int
+ * [2], caller-owned) receives 0 for each wait that gave up, 1 for one that succeeded.  src16:
+ * DEVICE, 16-byte aligned, 16 readable bytes.  Asynchronous on `stream`.  GPT2_ERR_ARG for a
+ * null or misaligned pointer or a limit outside the range. */
+int gpt2op_bounded_wait_selftest(void* stream, int64_t limit_ns, const void* src16, int* status);
 
 /* Reads and clears the device error word of the current device (GPT2_OK if none). */
 int gpt2op_device_error(void);

@@ -26,12 +26,12 @@ def test_default_run_is_the_headline_workload():
 
 def test_longer_context_keeps_the_tokens_per_step():
     a = _parse("--seq", "2048")
-    assert (a.micro_batch, a.accum) == (16, 16)
+    assert (a.micro_batch, a.accum) == (32, 8)         # the pages' GPT-3 batch: B = 32 at T = 2048
     assert a.micro_batch * a.seq * a.accum == 524288
     name = bench.metric_name(a.model, a.micro_batch, a.seq)
     assert name != bench.METRIC and "T=2048" in name
     a = _parse("--seq", "512")
-    assert a.micro_batch * a.seq * a.accum == 524288 and a.micro_batch * a.seq <= 32768
+    assert a.micro_batch * a.seq * a.accum == 524288 and a.micro_batch * a.seq <= 131072
 
 
 def test_medium_model_defaults():

@@ -13,7 +13,6 @@ from decoder_only_transformer_train_b200 import synthetic as S
 from gpu_common import cuda_i32, rel_l2, require_gpu
 
 V = 50257
-POS_BITS = 15
 
 
 def _tokens(kind, B, T, seed):
@@ -41,7 +40,7 @@ def _run_bwd(tok, dx0, dwte0, dwpe0, B, T, C):
     BD.embedding_bwd(tok_d, dx_d, dwte, dwpe, B, T, C, V, ws)
     torch.cuda.synchronize()
     assert BD.device_error() == 0
-    keys = ws[: 4 * B * T].view(torch.int32).cpu().numpy().view(np.uint32)
+    keys = ws[: 8 * B * T].view(torch.int64).cpu().numpy().view(np.uint64)
     return dwte.cpu(), dwpe.cpu(), keys
 
 
@@ -52,7 +51,9 @@ CASES = [
     ("uniform", 2, 513, 128),    # 1026 keys: the two-keys-per-thread sort
     ("same", 4, 1024, 96),       # one run through all 128 chunks (several ballot rounds)
     ("clamped", 5, 700, 1032),   # C above 1024: two column blocks
-    ("zipf", 32, 1024, 64),      # 32768 keys, the largest sort
+    ("zipf", 32, 1024, 64),      # 32768 keys: eight sorted segments merged
+    ("uniform", 3, 5001, 32),    # a ragged last segment (15003 keys, 4 segments)
+    ("zipf", 32, 2048, 64),      # 65536 keys: the GPT-3 context at B = 32, sixteen segments
 ]
 
 
@@ -70,7 +71,7 @@ def test_embedding_bwd_matches_oracle(kind, B, T, C):
     # keys: the stable order of the clamped ids, bit for bit
     clamped = np.clip(tok.reshape(-1).astype(np.int64), 0, V - 1)
     order = np.argsort(clamped, kind="stable")
-    want = ((clamped[order] << POS_BITS) | order).astype(np.uint32)
+    want = ((clamped[order].astype(np.uint64) << np.uint64(32)) | order.astype(np.uint64))
     assert np.array_equal(keys, want)
 
     grads = {"wte": dwte0.clone(), "wpe": dwpe0.clone()}
@@ -134,13 +135,15 @@ def test_embedding_entry_points_reject_bad_shapes_before_any_cuda_call():
     buf = np.zeros(64, dtype=np.float32)
     p = (buf.ctypes.data + 15) // 16 * 16
     err_shape, err_arg = -4, -1
-    assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 32, 1025, 64, V, p) == err_shape   # > 32768 positions
+    assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 64, 2049, 64, V, p) == err_shape   # > 131072 positions
     assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 2, 8, 66, V, p) == err_shape       # C % 4
     assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 0, 8, 64, V, p) == err_shape
     assert lib.gpt2op_embedding_bwd(None, p, p, p, p, 2, 8, 64, V, None) == err_arg
     assert lib.gpt2op_embedding_fwd(None, p, p, p, p, 2, 8, 62, V) == err_shape
     assert lib.gpt2op_embedding_fwd(None, None, p, p, p, 2, 8, 64, V) == err_arg
-    assert BD.embedding_bwd_ws_bytes(16384, 768) == 16384 * 4 + 512 * 2 * 768 * 4
+    # sorted keys (uint64), segment keys (uint32), chunk partials: each on a 256-byte boundary
+    assert BD.embedding_bwd_ws_bytes(16384, 768) == 16384 * 8 + 16384 * 4 + 512 * 2 * 768 * 4
+    assert BD.embedding_bwd_ws_bytes(77, 64) == 768 + 512 + 3 * 2 * 64 * 4
     # 16-byte accesses: a misaligned table, output or gradient is refused before any launch
     q = p + 4
     assert lib.gpt2op_embedding_fwd(None, p, q, p, p, 2, 8, 64, V) == err_arg
