@@ -808,64 +808,70 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         nd1 = (qi < T) ? -__ldg(D_bh + qi) : 0.f;
       }
       for (int t = w.it0; t < w.it1; ++t, ++g) {
+        // MODE 0: the 32 queries of this warp's columns.  Lane i loads query t*128 + c0 + i's
+        // scalars (a query past T gets P = 0) before the wait for the scores, stages them after
+        // it (so the load latency hides behind the wait), and every lane then reads all 32.
+        float nl0 = 0.f, nd0 = 0.f;
         if (MODE == 0) {
-          // the 32 queries of this warp's columns: lane i stages query t*128 + c0 + i's scalars
-          // (a query past T gets P = 0), then every lane reads all 32 of them
           const int qi = t * 128 + c0 + lane;
-          const float nl = (qi < T) ? -__ldg(lse_bh + qi) * LOG2E : -INFINITY;
-          const float nd = (qi < T) ? -__ldg(D_bh + qi) : 0.f;
-          __syncwarp();                            // the previous tile's reads of vec are done
-          vec[lane] = nl;
-          vec[32 + lane] = nd;
-          __syncwarp();
+          nl0 = (qi < T) ? -__ldg(lse_bh + qi) * LOG2E : -INFINITY;
+          nd0 = (qi < T) ? -__ldg(D_bh + qi) : 0.f;
         }
         if (!mbar_wait_warp(sd_full, g & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
+        if (MODE == 0) {
+          __syncwarp();                            // the previous tile's reads of vec are done
+          vec[lane] = nl0;
+          vec[32 + lane] = nd0;
+          __syncwarp();
+        }
         // causal mask on the diagonal tile: MODE 0 drops queries before key r, MODE 1 keys after
         // query r.  There a warp's whole 32 x 32 chunk is masked when its columns all lie on the
         // masked side of its 32 rows (MODE 0: part < q; MODE 1: part > q): its P and dZ are zero
-        // and its scores are not read.
+        // and its scores need no exponentials.
         const bool diag = (t == w.tile);
         const bool all_masked = diag && ((MODE == 0) ? (part < q) : (part > q));
-        // this thread's 32 columns of S and dP, then the TMEM buffer is released at once
-        uint32_t us[32], ud[32];
-        if (!all_masked) {
-          tmem_ld32(tmem + lane_off + BS_C + c0, us);
-          tmem_ld32(tmem + lane_off + BDP_C + c0, ud);
-          tmem_wait_ld();
-        }
-        tc_fence_before();
-        mbar_arrive(sd_empty);
+        // the thread's 32 columns in two halves of 16: S and dP of a half read from TMEM (the
+        // wait for them also keeps the compiler from hoisting the next half's work, which bounds
+        // the registers live at once), P and dZ computed; the S / dP buffer is released after
+        // the second half's read
         uint32_t pw[16], dw[16];
-        if (all_masked) {
 #pragma unroll
-          for (int d = 0; d < 16; ++d) pw[d] = dw[d] = 0u;
-        } else
-#pragma unroll
-        for (int d = 0; d < 32; d += 2) {
-          const int c = c0 + d;
-          float2 nl, nd;
-          if (MODE == 0) {
-            nl = *reinterpret_cast<const float2*>(vec + d);
-            nd = *reinterpret_cast<const float2*>(vec + 32 + d);
-          } else {
-            nl = make_float2(nl1, nl1);
-            nd = make_float2(nd1, nd1);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t us[16], ud[16];
+          tmem_ld16(tmem + lane_off + BS_C + c0 + 16 * hf, us);
+          tmem_ld16(tmem + lane_off + BDP_C + c0 + 16 * hf, ud);
+          tmem_wait_ld();
+          if (hf == 1) {
+            tc_fence_before();
+            mbar_arrive(sd_empty);
           }
-          const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
-          float2 pp = make_float2(ex2(x.x), ex2(x.y));
-          if (diag) {
+#pragma unroll
+          for (int d = 0; d < 16; d += 2) {
+            const int c = c0 + 16 * hf + d;
+            float2 nl, nd;
             if (MODE == 0) {
-              if (c < r) pp.x = 0.f;
-              if (c + 1 < r) pp.y = 0.f;
+              nl = *reinterpret_cast<const float2*>(vec + 16 * hf + d);
+              nd = *reinterpret_cast<const float2*>(vec + 32 + 16 * hf + d);
             } else {
-              if (c > r) pp.x = 0.f;
-              if (c + 1 > r) pp.y = 0.f;
+              nl = make_float2(nl1, nl1);
+              nd = make_float2(nd1, nd1);
             }
+            const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
+            float2 pp = all_masked ? make_float2(0.f, 0.f) : make_float2(ex2(x.x), ex2(x.y));
+            if (diag) {
+              if (MODE == 0) {
+                if (c < r) pp.x = 0.f;
+                if (c + 1 < r) pp.y = 0.f;
+              } else {
+                if (c > r) pp.x = 0.f;
+                if (c + 1 > r) pp.y = 0.f;
+              }
+            }
+            const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])), nd));
+            pw[8 * hf + (d >> 1)] = pack_bf16x2(pp.x, pp.y);
+            dw[8 * hf + (d >> 1)] = pack_bf16x2(gz.x, gz.y);
           }
-          const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])), nd));
-          pw[d >> 1] = pack_bf16x2(pp.x, pp.y);
-          dw[d >> 1] = pack_bf16x2(gz.x, gz.y);
         }
         // the previous tile's MMAs must be done reading P / dZ in TMEM
         if (!mbar_wait_warp(ps_empty, (g & 1) ^ 1, abort_flag)) { ok = false; break; }

@@ -104,7 +104,7 @@ struct gpt2_ctx {
 
   float* dres = nullptr;
   void* dres_act = nullptr;
-  float* dy = nullptr;
+  void* dy = nullptr;       // gradient of a LayerNorm output (activation type)
   void* d4c = nullptr;
   void* dqkv = nullptr;
   void* dattn = nullptr;
@@ -154,6 +154,16 @@ int fail(gpt2_ctx* c, int code, const char* msg) {
 int cuda_fail(gpt2_ctx* c, cudaError_t e, const char* where) {
   if (c) c->err = std::string(where) + ": " + cudaGetErrorString(e);
   return GPT2_ERR_CUDA;
+}
+
+// Host-to-device copy ordered on the context stream and complete on return.  A plain
+// cudaMemcpy from pageable host memory may return before its DMA has landed, and runs on the
+// legacy default stream, which does not order against the context's non-blocking stream: a
+// kernel launched right after could read the old contents.
+cudaError_t h2d_ordered(gpt2_ctx* c, void* dst, const void* src, size_t bytes) {
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, c->stream);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(c->stream);
 }
 
 template <typename T>
@@ -409,7 +419,9 @@ int backward_impl(gpt2_ctx* c) {
   }
   // dh = dz wte ; dwte += dz^T h
   const double head_flops = 2.0 * Nd * Vp * Cd;
-  EpiParams e = epi_make(EPI_STORE_F32, c->dy, C);
+  // the dX products write the LayerNorm output gradient in the activation type (bf16 in bf16 mode)
+  const int dy_kind = c->bf16 ? EPI_STORE_ACT : EPI_STORE_F32;
+  EpiParams e = epi_make(dy_kind, c->dy, C);
   {
     PROF(PROF_HEAD_BWD, head_flops, 0);
     RC(gemm(c, N, C, Vp, c->logits, c->ldl, false, W(c, 0), C, true, e));
@@ -421,7 +433,7 @@ int backward_impl(gpt2_ctx* c) {
   }
   const int lf = lnf_w_index(g);
   float* xL = c->resid + (long long)L * c->Nmax * C;
-  const double ln_bwd_bytes = Nd * Cd * (4.0 * 4 + A) + 8.0 * Nd;
+  const double ln_bwd_bytes = Nd * Cd * (4.0 * 3 + 2.0 * A) + 8.0 * Nd;   // dy, x, dres in; dres, dres_act out
   {
     PROF(PROF_LN_BWD, 0, ln_bwd_bytes - 4.0 * Nd * Cd);
     // the new dres is d loss / d x_L: its column sums are the last mlp.c_proj bias gradient
@@ -456,7 +468,7 @@ int backward_impl(gpt2_ctx* c) {
       PROF(PROF_BIAS, 0, A * Nd * 4 * Cd);
       RC(launch_colsum(st, c->bf16, c->d4c, 4 * C, N, 4 * C, c->colsum_part, ncs, G(c, pi(FC_B))));
     }
-    e = epi_make(EPI_STORE_F32, c->dy, C);
+    e = epi_make(dy_kind, c->dy, C);
     {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * 4 * Cd * Cd, 0);
       RC(gemm(c, N, C, 4 * C, c->d4c, 4 * C, false, W(c, pi(FC_W)), C, true, e));
@@ -500,7 +512,7 @@ int backward_impl(gpt2_ctx* c) {
       PROF(PROF_BIAS, 0, A * Nd * 3 * Cd);
       RC(launch_colsum(st, c->bf16, c->dqkv, 3 * C, N, 3 * C, c->colsum_part, ncs, G(c, pi(ATTN_B))));
     }
-    e = epi_make(EPI_STORE_F32, c->dy, C);
+    e = epi_make(dy_kind, c->dy, C);
     {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * 3 * Cd * Cd, 0);
       RC(gemm(c, N, C, 3 * C, c->dqkv, 3 * C, false, W(c, pi(ATTN_W)), C, true, e));
@@ -693,7 +705,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
   AL(dalloc(c, &c->targets, N));
   AL(dalloc(c, &c->dres, N * C));
   AL(dalloc_bytes(c, &c->dres_act, N * C * A));
-  AL(dalloc(c, &c->dy, N * C));
+  AL(dalloc_bytes(c, &c->dy, N * C * A));
   AL(dalloc_bytes(c, &c->d4c, N * 4 * C * A));
   AL(dalloc_bytes(c, &c->dqkv, N * 3 * C * A));
   AL(dalloc_bytes(c, &c->dattn, N * C * A));
@@ -729,7 +741,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
     }
     c->n_adam_blocks = (int)blocks.size();
     AL(dalloc(c, &c->adam_blocks, blocks.size()));
-    if (cudaMemcpy(c->adam_blocks, blocks.data(), blocks.size() * sizeof(AdamBlock), cudaMemcpyHostToDevice) !=
+    if (h2d_ordered(c, c->adam_blocks, blocks.data(), blocks.size() * sizeof(AdamBlock)) !=
         cudaSuccess) {
       rc = GPT2_ERR_CUDA;
       goto fail_out;
@@ -894,7 +906,7 @@ int gpt2_set_params(gpt2_ctx* c, const float* src) {
   if (c == nullptr || src == nullptr) return GPT2_ERR_ARG;
   int rc = check_device(c);
   if (rc) return rc;
-  cudaError_t e = cudaMemcpy(c->params, src, c->nparams * sizeof(float), cudaMemcpyHostToDevice);
+  cudaError_t e = h2d_ordered(c, c->params, src, c->nparams * sizeof(float));
   if (e != cudaSuccess) return cuda_fail(c, e, "set_params copy");
   RC(refresh_shadow(c));
   return check_device(c);
@@ -910,8 +922,8 @@ int gpt2_set_optimizer_state(gpt2_ctx* c, const float* m_src, const float* v_src
   if (c == nullptr || m_src == nullptr || v_src == nullptr || t < 0) return GPT2_ERR_ARG;
   int rc = check_device(c);
   if (rc) return rc;
-  if (cudaMemcpy(c->m, m_src, c->nparams * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy(c->v, v_src, c->nparams * sizeof(float), cudaMemcpyHostToDevice) != cudaSuccess)
+  if (h2d_ordered(c, c->m, m_src, c->nparams * sizeof(float)) != cudaSuccess ||
+      h2d_ordered(c, c->v, v_src, c->nparams * sizeof(float)) != cudaSuccess)
     return fail(c, GPT2_ERR_CUDA, "set_optimizer_state copy");
   c->step_t = t;
   return GPT2_OK;

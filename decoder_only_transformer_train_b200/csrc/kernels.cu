@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(256) ln_fwd_kernel(const float* __restrict__ x
 // dres rows, which is the bias gradient of the Linear layer whose output this residual
 // stream position receives (attn.c_proj or mlp.c_proj).
 template <typename ActT, int CPL>
-__global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict__ dy, const float* __restrict__ x,
+__global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const ActT* __restrict__ dy, const float* __restrict__ x,
                                                         const float* __restrict__ mean, const float* __restrict__ rstd,
                                                         const float* __restrict__ w, float* __restrict__ dres,
                                                         ActT* __restrict__ dres_act, int accumulate,
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict_
     mine[2 * C + lane + 32 * k] = 0.f;
   }
   for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
-    const float* dyr = dy + (long long)row * C;
+    const ActT* dyr = dy + (long long)row * C;
     const float* xr = x + (long long)row * C;
     float* dr = dres + (long long)row * C;
     const float mu = mean[row], r = rstd[row];
@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const float* __restrict_
 #pragma unroll
     for (int k = 0; k < CPL; ++k) {
       const int c = lane + 32 * k;
-      const float d = dyr[c];
+      const float d = ld_f(dyr + c);
       xh[k] = (xr[c] - mu) * r;
       g[k] = d * __ldg(w + c);
       s1 += g[k];
@@ -1107,8 +1107,18 @@ int ln_fwd_dispatch(cudaStream_t st, const float* x, const float* w, const float
 // Same with 16-byte accesses (C a multiple of 128): lane l holds float4 column groups
 // l, l + 32, ...; gamma stays in registers and the per-warp accumulators are updated four
 // columns at a time.
+// Four consecutive values (16-byte aligned group c4 of a row) as fp32, streaming load.
+__device__ __forceinline__ float4 ld4_stream(const float* row, int c4) {
+  return __ldcs(reinterpret_cast<const float4*>(row) + c4);
+}
+__device__ __forceinline__ float4 ld4_stream(const bf16* row, int c4) {
+  const uint2 q = __ldcs(reinterpret_cast<const uint2*>(row) + c4);
+  const float2 a = unpack_bf16x2(q.x), b = unpack_bf16x2(q.y);
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
 template <typename ActT, int V4>
-__global__ void __launch_bounds__(256, 2) ln_bwd_vec_kernel(const float* __restrict__ dy, const float* __restrict__ x,
+__global__ void __launch_bounds__(256, 2) ln_bwd_vec_kernel(const ActT* __restrict__ dy, const float* __restrict__ x,
                                                             const float* __restrict__ mean,
                                                             const float* __restrict__ rstd, const float* __restrict__ w,
                                                             float* __restrict__ dres, ActT* __restrict__ dres_act,
@@ -1128,7 +1138,7 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_vec_kernel(const float* __restr
     if (HOIST_W) wv[HOIST_W ? k : 0] = __ldg(reinterpret_cast<const float4*>(w) + lane + 32 * k);
   }
   for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
-    const float4* dyr = reinterpret_cast<const float4*>(dy + (long long)row * C);
+    const ActT* dyr = dy + (long long)row * C;
     const float4* xr = reinterpret_cast<const float4*>(x + (long long)row * C);
     float4* dr = reinterpret_cast<float4*>(dres + (long long)row * C);
     const float mu = mean[row], r = rstd[row];
@@ -1139,7 +1149,7 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_vec_kernel(const float* __restr
 #pragma unroll
     for (int k = 0; k < V4; ++k) {
       const int c = lane + 32 * k;
-      const float4 d = __ldcs(dyr + c), xv = __ldcs(xr + c);
+      const float4 d = ld4_stream(dyr, c), xv = __ldcs(xr + c);
       xh[k] = make_float4((xv.x - mu) * r, (xv.y - mu) * r, (xv.z - mu) * r, (xv.w - mu) * r);
       const float4 wk = HOIST_W ? wv[HOIST_W ? k : 0] : __ldg(reinterpret_cast<const float4*>(w) + c);
       g[k] = make_float4(d.x * wk.x, d.y * wk.y, d.z * wk.z, d.w * wk.w);
@@ -1187,7 +1197,7 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_vec_kernel(const float* __restr
 }
 
 template <typename ActT>
-int ln_bwd_dispatch(cudaStream_t st, const float* dy, const float* x, const float* mean, const float* rstd,
+int ln_bwd_dispatch(cudaStream_t st, const ActT* dy, const float* x, const float* mean, const float* rstd,
                     const float* w, float* dres, ActT* dres_act, int acc, float* part, int nblocks, int N, int C) {
   const int smem = 8 * 3 * C * (int)sizeof(float);
   const bool vec = ((reinterpret_cast<uintptr_t>(dy) | reinterpret_cast<uintptr_t>(x) |
@@ -1260,13 +1270,13 @@ int launch_layernorm_fwd(cudaStream_t st, bool is_bf16, const float* x, const fl
 
 int layernorm_bwd_blocks(int num_sms) { return 2 * num_sms; }
 
-int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const float* dy, const float* x, const float* mean,
+int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const void* dy, const float* x, const float* mean,
                          const float* rstd, const float* w, float* dres, void* dres_act, bool accumulate, float* part,
                          int nblocks, float* dw, float* db, float* dbias_out, int N, int C) {
-  int rc = is_bf16 ? ln_bwd_dispatch<bf16>(st, dy, x, mean, rstd, w, dres, reinterpret_cast<bf16*>(dres_act),
-                                           accumulate, part, nblocks, N, C)
-                   : ln_bwd_dispatch<float>(st, dy, x, mean, rstd, w, dres, reinterpret_cast<float*>(dres_act),
-                                            accumulate, part, nblocks, N, C);
+  int rc = is_bf16 ? ln_bwd_dispatch<bf16>(st, reinterpret_cast<const bf16*>(dy), x, mean, rstd, w, dres,
+                                           reinterpret_cast<bf16*>(dres_act), accumulate, part, nblocks, N, C)
+                   : ln_bwd_dispatch<float>(st, reinterpret_cast<const float*>(dy), x, mean, rstd, w, dres,
+                                            reinterpret_cast<float*>(dres_act), accumulate, part, nblocks, N, C);
   if (rc) return rc;
   ln_param_reduce_kernel<<<cdiv(dbias_out ? 3 * C : 2 * C, 32), 32 * LNP_GROUPS, 0, st>>>(part, nblocks, C, dw, db,
                                                                                          dbias_out);

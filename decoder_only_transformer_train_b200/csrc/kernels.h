@@ -20,8 +20,10 @@ int launch_encoder_fwd(cudaStream_t st, const int* tok, const float* wte, const 
                        int C, int V);
 int launch_layernorm_fwd(cudaStream_t st, bool bf16, const float* x, const float* w, const float* b, void* y,
                          float* mean, float* rstd, int N, int C);
-// dbias_out (may be null): receives the column sums of the new dres rows.
-int launch_layernorm_bwd(cudaStream_t st, bool bf16, const float* dy, const float* x, const float* mean,
+// dy: the gradient of the LayerNorm output, of the activation type (bf16 in bf16 mode, as the
+// bf16 product that makes it returns it).  dbias_out (may be null): receives the column sums of
+// the new dres rows.
+int launch_layernorm_bwd(cudaStream_t st, bool bf16, const void* dy, const float* x, const float* mean,
                          const float* rstd, const float* w, float* dres, void* dres_act, bool accumulate,
                          float* part, int nblocks, float* dw, float* db, float* dbias_out, int N, int C);
 int layernorm_bwd_blocks(int num_sms);

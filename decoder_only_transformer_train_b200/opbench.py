@@ -212,12 +212,16 @@ def main(argv=None):
         # model's width and vocabulary but two layers (53.5M parameters, about 1.8 GB of state)
         cfg = BD.Config(n_layer=2, n_embd=C, n_head=H, block_size=T, vocab_size=50257, padded_vocab_size=V,
                         max_batch=1, grad_accum_steps=1, precision=BD.GPT2_BF16)
-        model = BD.GPT2(cfg, seed=1, stream=torch.cuda.current_stream().cuda_stream)
+        # the model's work goes to its own (non-default) stream, on which the timer records
+        stream = torch.cuda.Stream()
+        model = BD.GPT2(cfg, seed=1, stream=stream.cuda_stream)
         g = model.grad_tensor()
         g.normal_(generator=gen)
+        torch.cuda.synchronize()
         n = model.num_params
         fn = lambda: model.adamw_step(6e-4, sync_norm=False)
-        ms = timer(fn, args.iters, args.warmup)
+        with torch.cuda.stream(stream):
+            ms = timer(fn, args.iters, args.warmup)
         # norm: read g; AdamW: read p, g, m, v, write p, m, v and the bf16 copy of the >= 2-D tensors
         nbytes = 4 * n + 28 * n + 2 * n
         report("optimizer", ms, params=n, gbs=round(nbytes / (ms * 1e-3) / 1e9, 1))
