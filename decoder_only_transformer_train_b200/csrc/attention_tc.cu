@@ -38,28 +38,22 @@ constexpr uint32_t P_COL = 384;                // P of group g (bf16 pairs): col
 constexpr float RESCALE_THRESHOLD = 8.0f;      // log2 units
 
 
-// Row max of a 128-column S tile in TMEM (64 columns per round trip); on the diagonal
-// tile the keys after query row r are left out.  Four independent max chains.
+// Row max over the first 32 columns of an S tile in TMEM; on the diagonal tile the keys after
+// query row r are left out (key 0 never is).
 template <bool DIAG>
-__device__ __forceinline__ float s_row_max(uint32_t taddr, int r) {
+__device__ __forceinline__ float s_chunk32_max(uint32_t taddr, int r) {
+  uint32_t v[32];
+  tmem_ld32(taddr, v);
+  tmem_wait_ld();
   float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int c0 = 0; c0 < 128; c0 += 64) {
-    // on the diagonal tile rows below 64 (warps of lane quarters 0 and 1) see only the first half
-    if (DIAG && c0 == 64 && r < 64) break;
-    uint32_t v[64];
-    tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-    tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-    tmem_wait_ld();
-#pragma unroll
-    for (int e = 0; e < 64; e += 2) {
-      float a = __uint_as_float(v[e]), b = __uint_as_float(v[e + 1]);
-      if (DIAG) {
-        if (c0 + e > r) a = -INFINITY;
-        if (c0 + e + 1 > r) b = -INFINITY;
-      }
-      m4[(e >> 1) & 3] = max3f(m4[(e >> 1) & 3], a, b);
+  for (int e = 0; e < 32; e += 2) {
+    float a = __uint_as_float(v[e]), b = __uint_as_float(v[e + 1]);
+    if (DIAG) {
+      if (e > r) a = -INFINITY;
+      if (e + 1 > r) b = -INFINITY;
     }
+    m4[(e >> 1) & 3] = max3f(m4[(e >> 1) & 3], a, b);
   }
   return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 }
@@ -310,27 +304,26 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         const uint32_t srow = tmem + lane_off + s_col;
         float sum;
         if (!has) {
-          // the group's first tile of the item: its row max sets m_ref (two TMEM passes)
-          const float mx = diag ? s_row_max<true>(srow, r) : s_row_max<false>(srow, r);
-          // the group's previous P.V MMA must be done: P buffer free, O stable
-          if (!mbar_wait_warp(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
-          m_ref = mx * scale_log2;
-          sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, pcol)
-                     : p_row_store<false>(srow, r, scale_log2, m_ref, pcol);
-        } else {
-          // one pass: P against the current m_ref, and the tile's row max alongside
-          if (!mbar_wait_warp(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
-          float mx;
-          sum = diag ? p_row_store<true, true>(srow, r, scale_log2, m_ref, pcol, &mx)
-                     : p_row_store<false, true>(srow, r, scale_log2, m_ref, pcol, &mx);
-          const float m_new = mx * scale_log2;
-          const bool grow = m_new > m_ref + RESCALE_THRESHOLD;
-          // tcgen05.ld / st are warp-collective, so the whole warp takes this branch when
-          // any of its rows' max grew past the threshold: those rows rescale O and l and
-          // write P again against the new max; the others scale by exactly 1 and write the
-          // same P again.
-          if (__any_sync(0xffffffffu, grow)) {
-            const float f = grow ? ex2(m_ref - m_new) : 1.0f;
+          // the group's first tile of the item: a first m_ref from the row's max over the tile's
+          // first 32 keys (on the diagonal tile key 0 is always valid); the pass below tracks
+          // the true max and writes P again if it grew past the threshold
+          m_ref = (diag ? s_chunk32_max<true>(srow, r) : s_chunk32_max<false>(srow, r)) * scale_log2;
+        }
+        // the group's previous P.V MMA must be done: P columns free, O stable
+        if (!mbar_wait_warp(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
+        // one pass: P against the current m_ref, and the tile's row max alongside
+        float mx;
+        sum = diag ? p_row_store<true, true>(srow, r, scale_log2, m_ref, pcol, &mx)
+                   : p_row_store<false, true>(srow, r, scale_log2, m_ref, pcol, &mx);
+        const float m_new = mx * scale_log2;
+        const bool grow = m_new > m_ref + RESCALE_THRESHOLD;
+        // tcgen05.ld / st are warp-collective, so the whole warp takes this branch when any of
+        // its rows' max grew past the threshold: those rows rescale O (from the item's second
+        // tile of the group on; before it O holds nothing of this item) and l and write P again
+        // against the new max; the others scale by exactly 1 and write the same P again.
+        if (__any_sync(0xffffffffu, grow)) {
+          const float f = grow ? ex2(m_ref - m_new) : 1.0f;
+          if (has) {
             tc_fence_after();
 #pragma unroll
             for (int c0 = 0; c0 < HD; c0 += 16) {
@@ -342,11 +335,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
               tmem_st16(tmem + lane_off + O_COL + grp * HD + c0, v);
             }
             tmem_wait_st();
-            l *= f;
-            if (grow) m_ref = m_new;
-            sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, pcol)
-                       : p_row_store<false>(srow, r, scale_log2, m_ref, pcol);
           }
+          l *= f;
+          if (grow) m_ref = m_new;
+          sum = diag ? p_row_store<true>(srow, r, scale_log2, m_ref, pcol)
+                     : p_row_store<false>(srow, r, scale_log2, m_ref, pcol);
         }
         l += sum;
         tc_fence_before();

@@ -1038,11 +1038,32 @@ __global__ void __launch_bounds__(256) ln_fwd_vec_kernel(const float* __restrict
     wv[k] = reinterpret_cast<const float4*>(w)[lane + 32 * k];
     bv[k] = reinterpret_cast<const float4*>(b)[lane + 32 * k];
   }
-  for (int row = blockIdx.x * 8 + warp; row < N; row += gridDim.x * 8) {
+  // rows up to 768 columns also load the warp's next row before working on the current one,
+  // so that two rows' loads are in flight (wider rows have no registers to spare for it)
+  constexpr bool PREFETCH = V4 <= 6;
+  const int stride = gridDim.x * 8;
+  float4 nv[PREFETCH ? V4 : 1];
+  int row = blockIdx.x * 8 + warp;
+  if (PREFETCH && row < N) {
     const float4* xr = reinterpret_cast<const float4*>(x + (long long)row * C);
-    float4 v[V4];
 #pragma unroll
-    for (int k = 0; k < V4; ++k) v[k] = __ldcs(xr + lane + 32 * k);
+    for (int k = 0; k < V4; ++k) nv[PREFETCH ? k : 0] = __ldcs(xr + lane + 32 * k);
+  }
+  for (; row < N; row += stride) {
+    float4 v[V4];
+    if (PREFETCH) {
+#pragma unroll
+      for (int k = 0; k < V4; ++k) v[k] = nv[PREFETCH ? k : 0];
+      if (row + stride < N) {
+        const float4* xn = reinterpret_cast<const float4*>(x + (long long)(row + stride) * C);
+#pragma unroll
+        for (int k = 0; k < V4; ++k) nv[PREFETCH ? k : 0] = __ldcs(xn + lane + 32 * k);
+      }
+    } else {
+      const float4* xr = reinterpret_cast<const float4*>(x + (long long)row * C);
+#pragma unroll
+      for (int k = 0; k < V4; ++k) v[k] = __ldcs(xr + lane + 32 * k);
+    }
     float s = 0.f;
 #pragma unroll
     for (int k = 0; k < V4; ++k) s += (v[k].x + v[k].y) + (v[k].z + v[k].w);
