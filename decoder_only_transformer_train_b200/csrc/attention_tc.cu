@@ -19,6 +19,7 @@
 //                 more than 2^8, and then the thread rescales its O row in TMEM before the
 //                 next MMA.  At the end of an item the two groups' (m_ref, l, O) are merged.
 #include <math.h>
+#include <stdlib.h>
 #include "sm100.cuh"
 #include "kernels.h"
 
@@ -44,7 +45,7 @@ template <bool DIAG>
 __device__ __forceinline__ float s_chunk32_max(uint32_t taddr, int r) {
   uint32_t v[32];
   tmem_ld32(taddr, v);
-  tmem_wait_ld();
+  tmem_wait_ld_regs(v);
   float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
@@ -62,7 +63,9 @@ __device__ __forceinline__ float s_chunk32_max(uint32_t taddr, int r) {
 // P columns at TMEM address pcol (this thread's lane); returns the row sum of P (four
 // independent partial sums).  With MAX, the same pass also returns the row's raw max in *mx
 // (masked keys left out), so that a tile whose max stays within the rescale threshold of m_ref
-// is read from TMEM once.
+// is read from TMEM once.  The row goes in 16-column chunks, the next chunk's TMEM load in
+// flight while the current one is computed (the loop over chunk pairs is kept rolled, which
+// keeps the pipeline within the registers).
 template <bool DIAG, bool MAX = false>
 __device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_log2, float m_ref, uint32_t pcol,
                                              float* mx = nullptr) {
@@ -70,9 +73,13 @@ __device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_
   float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
   const float2 sc = make_float2(scale_log2, scale_log2);
   const float2 nm = make_float2(-m_ref, -m_ref);
-  auto half = [&](int c0, const uint32_t* v, uint32_t* w) {
+  // on the diagonal tile rows below 64 (warps of lane quarters 0 and 1; warp-uniform) have no
+  // unmasked key in the second half: P is zero there
+  const int nch = (DIAG && r < 64) ? 4 : 8;   // 16-column chunks holding unmasked keys
+  uint32_t w[16];
+  auto chunk = [&](int c0, const uint32_t (&v)[16]) {
 #pragma unroll
-    for (int e = 0; e < 64; e += 2) {
+    for (int e = 0; e < 16; e += 2) {
       const float sa = __uint_as_float(v[e]), sb = __uint_as_float(v[e + 1]);
       const float2 x = ffma2(make_float2(sa, sb), sc, nm);
       float pa = ex2(x.x), pb = ex2(x.y);
@@ -88,25 +95,26 @@ __device__ __forceinline__ float p_row_store(uint32_t taddr, int r, float scale_
         m4[(e >> 1) & 3] = max3f(m4[(e >> 1) & 3], ma, mb);
       }
       sum[(e >> 1) & 3] = fadd2(sum[(e >> 1) & 3], make_float2(pa, pb));
-      w[e >> 1] = pack_bf16x2(pa, pb);
+      w[((c0 & 31) >> 1) + (e >> 1)] = pack_bf16x2(pa, pb);
     }
   };
+  uint32_t va[16], vb[16];
+  tmem_ld16(taddr, va);
+  tmem_wait_ld_regs16(va);
 #pragma unroll 1
-  for (int c0 = 0; c0 < 128; c0 += 64) {
-    uint32_t w[32];
-    if (DIAG && c0 == 64 && r < 64) {
-      // a wholly masked half (rows below 64 of the diagonal tile; warp-uniform): P = 0
-#pragma unroll
-      for (int e = 0; e < 32; ++e) w[e] = 0u;
+  for (int c = 0; c < 8; c += 2) {
+    if (c < nch) {
+      tmem_ld16(taddr + 16 * (c + 1), vb);
+      chunk(16 * c, va);
+      tmem_wait_ld_regs16(vb);
+      if (c + 2 < nch) tmem_ld16(taddr + 16 * (c + 2), va);
+      chunk(16 * (c + 1), vb);
+      if (c + 2 < nch) tmem_wait_ld_regs16(va);
     } else {
-      uint32_t v[64];
-      tmem_ld32(taddr + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-      tmem_ld32(taddr + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-      tmem_wait_ld();
-      half(c0, v, w);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) w[e] = 0u;
     }
-    tmem_st16(pcol + (c0 >> 1), *reinterpret_cast<uint32_t(*)[16]>(w));
-    tmem_st16(pcol + (c0 >> 1) + 16, *reinterpret_cast<uint32_t(*)[16]>(w + 16));
+    tmem_st16(pcol + 8 * c, w);
   }
   tmem_wait_st();
   if (MAX) *mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
@@ -463,11 +471,11 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return -3;
-  if (set_dynamic_smem_once((const void*)attn_fwd_tc_kernel, SMEM_BYTES)) return -3;
   const int nsm = current_device_sms();
   const int total = cdiv(T, QT) * B * H;
   const int grid = total < nsm ? total : nsm;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  if (set_dynamic_smem_once((const void*)attn_fwd_tc_kernel, SMEM_BYTES)) return -3;
   attn_fwd_tc_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(tm, reinterpret_cast<bf16*>(out), lse, B, T, H,
                                                             scale_log2);
   note_kernel_launches(1);
@@ -834,7 +842,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
           uint32_t us[16], ud[16];
           tmem_ld16(tmem + lane_off + BS_C + c0 + 16 * hf, us);
           tmem_ld16(tmem + lane_off + BDP_C + c0 + 16 * hf, ud);
-          tmem_wait_ld();
+          tmem_wait_ld_regs16x2(us, ud);
           if (hf == 1) {
             tc_fence_before();
             mbar_arrive(sd_empty);
@@ -919,18 +927,19 @@ int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const
   if (rc) return rc;
   rc = encode_rows64(&td, dout, C, (long long)B * T);
   if (rc) return rc;
-  if (set_dynamic_smem_once((const void*)attn_bwd_tc_kernel<0>, BWD_SMEM) ||
-      set_dynamic_smem_once((const void*)attn_bwd_tc_kernel<1>, BWD_SMEM))
-    return -3;
   const int nsm = current_device_sms();
   const int items = cdiv(T, 128) * B * H;
   const int grid = items < nsm ? items : nsm;   // persistent: one CTA per SM
   const float scale = 1.0f / sqrtf((float)HD);
   const float scale_log2 = 1.4426950408889634f * scale;
+  if (set_dynamic_smem_once((const void*)attn_bwd_tc_kernel<0>, BWD_SMEM) ||
+      set_dynamic_smem_once((const void*)attn_bwd_tc_kernel<1>, BWD_SMEM))
+    return -3;
   attn_bwd_tc_kernel<0><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv),
                                                              bias_part, B, T, H, scale, scale_log2);
   attn_bwd_tc_kernel<1><<<grid, BWD_THREADS, BWD_SMEM, st>>>(tq, td, lse, Dbuf, reinterpret_cast<bf16*>(dqkv),
                                                              bias_part, B, T, H, scale, scale_log2);
+  if (rc) return rc;
   note_kernel_launches(2);
   return cudaGetLastError() == cudaSuccess ? 0 : -3;
 }

@@ -207,6 +207,20 @@ def main(argv=None):
         report(name, ms, N=ntok, V=Vc, C=C, tflops=round(6.0 * ntok * Vc * C / (ms * 1e-3) / 1e12, 1))
         del h, W, logits, dW
 
+    if sel.search("sample"):
+        # top-k sampling (k = 50, the pages' value) of 64 rows of bf16 logits over the padded vocabulary
+        nr, k = 64, 50
+        logits = rnd(nr, V)
+        rows = torch.arange(nr, dtype=torch.int32, device=dev)
+        u = torch.rand(nr, device=dev, generator=gen)
+        out = torch.empty(nr, dtype=torch.int32, device=dev)
+        fn = lambda: BD.sample_top_k(logits, V, nr, rows, u, nr, 50257, k, BD.GPT2_BF16, out)
+        ms = timer(fn, args.iters, args.warmup)
+        # each sampled row read once (bf16)
+        nbytes = nr * 50257 * 2
+        report("sample", ms, rows=nr, k=k, gbs=round(nbytes / (ms * 1e-3) / 1e9, 1))
+        del logits
+
     if sel.search("optimizer"):
         # global norm + clip + AdamW through the model's entry point, on a context with the 124M
         # model's width and vocabulary but two layers (53.5M parameters, about 1.8 GB of state)
