@@ -710,7 +710,7 @@ struct TileChoice {
   int bn, splits, cg;
 };
 TileChoice choose_tiles(int M, int N, int K, bool can_split, size_t ws_elems, int num_sms, bool fixed_bn,
-                        bool b_mn, bool heavy_epilogue) {
+                        bool a_mn, bool b_mn, bool heavy_epilogue) {
   const int nk = cdiv(K, BK);
   const int bns[3] = {256, 192, 128};
   const double eff[3] = {1.0, 0.96, 0.88};
@@ -728,13 +728,23 @@ TileChoice choose_tiles(int M, int N, int K, bool can_split, size_t ws_elems, in
       if (bn > 128 && N <= 128) continue;
       if (cg == 2 && b_mn && bn == 192) continue;   // MN-major B is staged in 64-column boxes
       const int tiles = cdiv(M, BM * cg) * cdiv(N, bn);
-      if (cg == 2 && pairs != 1 && tiles < num_sms / 2) continue;   // pairs only with a full wave of tiles
+      // Weight gradients (both operands MN-major, K = tokens): narrower tiles issue more L2
+      // requests per MMA clock and run slower than the single-CTA model says, and large ones
+      // may split K on CTA pairs, whose halved operand traffic outweighs the partial sums.
+      // Measured over 16384 tokens: 768 x 3072 and 3072 x 768 take 66-68 us as 256-column
+      // pairs split in two, 74 us as 256-column single CTAs split in two, 91-96 us as 128-column
+      // tiles (single or pairs); 2304 x 768 takes 59 us as pairs split in two against 63 us.
+      const bool dw_pairs = a_mn && b_mn && (long long)M * N >= (1LL << 20);
+      if (cg == 2 && pairs != 1 && tiles < num_sms / 2 && !dw_pairs) continue;   // pairs only with a full wave of tiles
       for (int sp = 1; sp <= (can_split ? 8 : 1); ++sp) {
         if (sp > 1 && (nk / sp < 8 || N % 4 != 0 || (size_t)sp * cdiv(M, BM * cg) * BM * cg * N > ws_elems)) break;
-        if (sp > 1 && cg == 2 && pairs != 1) break;
+        if (sp > 1 && cg == 2 && pairs != 1 && !dw_pairs) break;
+        if (cg == 2 && pairs != 1 && dw_pairs && tiles * sp * 10 < (num_sms / 2) * 7) continue;   // most of a wave
+        if (cg == 2 && pairs != 1 && dw_pairs && sp > 2) break;   // splits measured: 1 and 2
         const int kb = cdiv(nk, sp);
         // MMA clocks per SM of a (128 cg) x bn x 64kb tile + overhead
-        const double per_tile = ((double)bn * kb * 2.0 / eff[i] + 1500.0) / (cg == 2 ? 1.2 : 1.0);
+        const double eff_i = dw_pairs ? (bn == 256 ? 1.0 : (bn == 192 ? 0.88 : 0.62)) : eff[i];
+        const double per_tile = ((double)bn * kb * 2.0 / eff_i + 1500.0) / (cg == 2 ? 1.2 : 1.0);
         const double waves = (double)cdiv(tiles * sp, num_sms / cg);
         double cost = waves * per_tile;
         if (sp > 1) cost += (double)(sp + 2) * M * N * 4.0 / 6.0e12 * 1.9e9 + 3000.0;   // partial traffic + reduce launch
@@ -762,7 +772,8 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   // the softmax partials of EPI_CE_FWD are laid out per 256/128-column tile
   const bool heavy = (ep.kind == EPI_RESID_F32 || ep.kind == EPI_GELU_FWD || ep.kind == EPI_GELU_BWD ||
                      ep.kind == EPI_CE_FWD);
-  const TileChoice tc = choose_tiles(M, N, K, can_split, ws_elems, num_sms, ep.kind == EPI_CE_FWD, b_mn, heavy);
+  const TileChoice tc = choose_tiles(M, N, K, can_split, ws_elems, num_sms, ep.kind == EPI_CE_FWD, a_mn, b_mn,
+                                     heavy);
   const int BN = tc.bn;
   const int CG = tc.cg;
   CUtensorMap ta, tb;

@@ -26,11 +26,15 @@ def _randn(shape, seed, scale=1.0):
 
 
 # ------------------------------------------------------------------ GEMM
-@pytest.fixture(params=["0", "1"], ids=["cta", "cta_pair"])
+@pytest.fixture(params=["0", "1", "default"], ids=["cta", "cta_pair", "cost_model"])
 def gemm_pairs(request, monkeypatch):
-    """Every GEMM test runs twice: with one CTA per 128-row tile, and with CTA pairs
-    (tcgen05 cta_group::2, 256-row tiles) wherever the shape allows them."""
-    monkeypatch.setenv("GPT2_B200_GEMM_PAIRS", request.param)
+    """Every GEMM test runs three times: with one CTA per 128-row tile, with CTA pairs
+    (tcgen05 cta_group::2, 256-row tiles) wherever the shape allows them, and with the
+    launcher's own choice (what the training step runs)."""
+    if request.param == "default":
+        monkeypatch.delenv("GPT2_B200_GEMM_PAIRS", raising=False)
+    else:
+        monkeypatch.setenv("GPT2_B200_GEMM_PAIRS", request.param)
     return request.param
 
 
