@@ -93,6 +93,19 @@ __device__ __forceinline__ float gelu_tanh_grad_fast(float x) {
   return 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * GELU_A * (1.0f + 3.0f * GELU_C * x * x);
 }
 
+// gelu(x) and gelu'(x) together from one tanh, in fp32 (tanhf) and with the hardware tanh
+// approximation (results rounded to bf16).
+__device__ __forceinline__ void gelu_tanh_and_grad_f(float x, float& g, float& gp) {
+  const float t = tanhf(GELU_A * (x + GELU_C * x * x * x));
+  g = 0.5f * x * (1.0f + t);
+  gp = 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * GELU_A * (1.0f + 3.0f * GELU_C * x * x);
+}
+__device__ __forceinline__ void gelu_tanh_and_grad_fast(float x, float& g, float& gp) {
+  const float t = tanh_approx(GELU_A * (x + GELU_C * x * x * x));
+  g = 0.5f * x * (1.0f + t);
+  gp = 0.5f * (1.0f + t) + 0.5f * x * (1.0f - t * t) * GELU_A * (1.0f + 3.0f * GELU_C * x * x);
+}
+
 // ---------------------------------------------------------------- single PTX instructions
 // 2^x by the hardware approximation (ex2.approx.ftz; subnormal results flushed to zero),
 // the 3-input maximum of sm_100, and paired fp32 arithmetic.

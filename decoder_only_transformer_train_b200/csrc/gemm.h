@@ -15,8 +15,8 @@ enum EpiKind : int {
   EPI_STORE_F32 = 1,   // C(f32) = alpha*D + bias
   EPI_ACCUM_F32 = 2,   // C(f32) += alpha*D                 (weight gradients)
   EPI_RESID_F32 = 3,   // C(f32) = aux(f32) + alpha*D + bias (residual stream)
-  EPI_GELU_FWD = 4,    // u = alpha*D + bias; aux_out(act) = u; C(act) = gelu(u)
-  EPI_GELU_BWD = 5,    // C(act) = alpha*D * gelu'(aux(act))
+  EPI_GELU_FWD = 4,    // u = alpha*D + bias; aux_out(act) = gelu'(u); C(act) = gelu(u)
+  EPI_GELU_BWD = 5,    // C(act) = alpha*D * aux(act)   (aux: the gelu'(u) the forward kept)
   EPI_CE_FWD = 6,      // C(act) = alpha*D (logits) + per-(row, column-tile) softmax partials
   EPI_SPLITK = 7,      // ws[split][m][n] = D   (internal: split-K partial products)
 };

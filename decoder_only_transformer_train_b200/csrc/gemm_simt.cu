@@ -24,13 +24,14 @@ __device__ __forceinline__ void epi_elem_f32(const EpiParams& ep, int m, int n, 
       *C = reinterpret_cast<const float*>(ep.aux)[(long long)m * ep.ld_aux + n] + ep.alpha * v + b;
       break;
     case EPI_GELU_FWD: {
-      const float u = ep.alpha * v + b;
-      reinterpret_cast<float*>(ep.aux_out)[(long long)m * ep.ld_aux_out + n] = u;
-      *C = gelu_tanh_f(u);
+      float g, gp;
+      gelu_tanh_and_grad_f(ep.alpha * v + b, g, gp);
+      reinterpret_cast<float*>(ep.aux_out)[(long long)m * ep.ld_aux_out + n] = gp;
+      *C = g;
       break;
     }
     case EPI_GELU_BWD:
-      *C = ep.alpha * v * gelu_tanh_grad_f(reinterpret_cast<const float*>(ep.aux)[(long long)m * ep.ld_aux + n]);
+      *C = ep.alpha * v * reinterpret_cast<const float*>(ep.aux)[(long long)m * ep.ld_aux + n];
       break;
     default:
       break;

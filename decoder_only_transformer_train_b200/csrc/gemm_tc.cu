@@ -462,14 +462,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int j = 0; j < 32; ++j) b[j] = (use_bias && n0 + j < ep.N) ? ep.bias[n0 + j] : 0.f;
           }
           if (kind == EPI_GELU_FWD) {
-            float u[32], g[32];
+            // gelu(u) and gelu'(u) from one tanh; gelu'(u) is what the backward needs
+            float gp[32], g[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              u[j] = alpha * v[j] + b[j];
-              g[j] = gelu_tanh_fast(u[j]);
-            }
+            for (int j = 0; j < 32; ++j) gelu_tanh_and_grad_fast(alpha * v[j] + b[j], g[j], gp[j]);
             int bx = E.take();
-            box_put_bf16(E.box(bx), lane, u);
+            box_put_bf16(E.box(bx), lane, gp);
             E.store(bx, &tmOut2, n0, m_warp);
             bx = E.take();
             box_put_bf16(E.box(bx), lane, g);
@@ -481,7 +479,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             box_get_bf16(E.box(bx), lane, u);
             __syncwarp();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] = alpha * v[j] * gelu_tanh_grad_fast(u[j]);
+            for (int j = 0; j < 32; ++j) u[j] = alpha * v[j] * u[j];
             box_put_bf16(E.box(bx), lane, u);
             E.store(bx, &tmOut, n0, m_warp);
             if (c + depth < nch) load_chunk(c + depth);

@@ -49,7 +49,7 @@ struct LayerActs {
   void* ln2;
   float* ln2_mean;
   float* ln2_rstd;
-  void* fc_pre;
+  void* fc_pre;     // gelu'(u) of the fc pre-activation u, kept for the backward
   void* fc_act;
 };
 

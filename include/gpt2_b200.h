@@ -204,9 +204,11 @@ int gpt2op_gemm_bf16(void* stream, int M, int N, int K, const void* A, int64_t l
  * the tanh GELU) and "1:48:25 – 2:00:19 torch.compile and the GPU memory hierarchy" (the
  * elementwise work fused with the kernel that produces its input):
  *   epilogue 3 (residual):  C(f32)[m*ldc + n] = aux(f32)[m*ld_aux + n] + alpha D + bias[n]
- *   epilogue 4 (GELU):      u = alpha D + bias[n];  aux_out(bf16)[m*ld_aux_out + n] = u;
+ *   epilogue 4 (GELU):      u = alpha D + bias[n];  aux_out(bf16)[m*ld_aux_out + n] = gelu_tanh'(u);
  *                           C(bf16)[m*ldc + n] = gelu_tanh(u)
- *   epilogue 5 (GELU grad): C(bf16)[m*ldc + n] = alpha D * gelu_tanh'(aux(bf16)[m*ld_aux + n])
+ *   epilogue 5 (GELU grad): C(bf16)[m*ldc + n] = alpha D * aux(bf16)[m*ld_aux + n]
+ *                           (aux: the gelu_tanh'(u) epilogue 4 kept, so the backward of the MLP
+ *                           multiplies by it instead of evaluating tanh again)
  * bias (f32 [N]) may be NULL for 3 and 4 and is ignored by 5.  aux / aux_out are device
  * buffers the caller owns, 16-byte aligned, with ld_aux / ld_aux_out multiples of 8
  * elements; aux may equal C for epilogue 3 (an in-place residual update).  GELU uses the
