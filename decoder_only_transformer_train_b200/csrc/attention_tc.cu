@@ -215,8 +215,11 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       if (*abort_flag) tx.drain();   // copies still in flight land before the CTA leaves
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ---------------------------------------------------------------- MMA issuer
+      // the whole warp runs the loop (its descriptors and counters stay warp-uniform); one
+      // elected lane issues the MMAs and commits
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc_s = make_idesc_bf16(QT, KT, false, false);   // Q, K both K-major
       constexpr uint32_t idesc_o = make_idesc_bf16(QT, HD, false, true);    // P from TMEM, V MN-major
       // tile iterator over the CTA's flattened (item, j) sequence
@@ -247,19 +250,22 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       bool ok = true;
       auto issue_s = [&](const It& it) -> bool {
         const int g = it.G & 1, s = it.G % KV_STAGES, qb = it.k & 1;
-        if (it.j == 0 && !mbar_wait(&q_full[qb], (it.k >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&kv_full[s], (it.G / KV_STAGES) & 1, abort_flag)) return false;
+        if (it.j == 0 && !mbar_wait_warp(&q_full[qb], (it.k >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&kv_full[s], (it.G / KV_STAGES) & 1, abort_flag)) return false;
         const int cs = g ? cs1 : cs0;
-        if (!mbar_wait(&s_empty[g], (cs & 1) ^ 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&s_empty[g], (cs & 1) ^ 1, abort_flag)) return false;
         if (g) ++cs1; else ++cs0;
         tc_fence_after();
         const uint32_t aQ = smem_u32(sQ + qb * TILE_BYTES);
         const uint32_t bK = smem_u32(sK + s * TILE_BYTES);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          tc_mma_bf16(tmem + S_COL + g * KT, make_sdesc_sw128(aQ + kk * 32, 16, 1024),
-                      make_sdesc_sw128(bK + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-        tc_commit(&s_full[g]);
+          for (int kk = 0; kk < HD / 16; ++kk)
+            tc_mma_bf16(tmem + S_COL + g * KT, make_sdesc_sw128(aQ + kk * 32, 16, 1024),
+                        make_sdesc_sw128(bK + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          tc_commit(&s_full[g]);
+        }
+        __syncwarp();
         return true;
       };
       if (valid(cur)) ok = issue_s(cur);
@@ -268,20 +274,24 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         if (valid(nx) && !issue_s(nx)) break;
         const int g = cur.G & 1, s = cur.G % KV_STAGES;
         const int co = g ? co1 : co0;
-        if (!mbar_wait(&p_full[g], co & 1, abort_flag)) break;
+        if (!mbar_wait_warp(&p_full[g], co & 1, abort_flag)) break;
         if (g) ++co1; else ++co0;
         tc_fence_after();
         const bool first_of_group = (cur.j < 2);          // the group's first tile of this item
         const uint32_t bV = smem_u32(sV + s * TILE_BYTES);
         // A: 16 keys of P = 8 TMEM columns per step; B: 16 rows of V, MN-major
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk)
-          tc_mma_bf16_ts(tmem + O_COL + g * HD, tmem + P_COL + g * 64 + kk * 8,
-                         make_sdesc_sw128(bV + kk * 2048, 8192, 1024), idesc_o, (kk > 0 || !first_of_group) ? 1u : 0u);
-        tc_commit(&kv_empty[s]);
-        tc_commit(&p_empty[g]);
-        if (cur.j + 2 > cur.qt) tc_commit(&o_done[g]);    // the group's last tile of this item
-        if (cur.j == cur.qt) tc_commit(&q_empty[cur.k & 1]);
+          for (int kk = 0; kk < KT / 16; ++kk)
+            tc_mma_bf16_ts(tmem + O_COL + g * HD, tmem + P_COL + g * 64 + kk * 8,
+                           make_sdesc_sw128(bV + kk * 2048, 8192, 1024), idesc_o,
+                           (kk > 0 || !first_of_group) ? 1u : 0u);
+          tc_commit(&kv_empty[s]);
+          tc_commit(&p_empty[g]);
+          if (cur.j + 2 > cur.qt) tc_commit(&o_done[g]);    // the group's last tile of this item
+          if (cur.j == cur.qt) tc_commit(&q_empty[cur.k & 1]);
+        }
+        __syncwarp();
         cur = nx;
       }
     }
@@ -654,8 +664,11 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       if (*abort_flag) tx.drain();   // copies still in flight land before the CTA leaves
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {
       // ---------------------------------------------------------------- MMA issuer
+      // the whole warp runs the loop (descriptors and counters stay warp-uniform); one elected
+      // lane issues the MMAs and commits
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc_sq = make_idesc_bf16(128, 128, false, false);   // 128x128, K=64, both K-major
       constexpr uint32_t idesc_acc = make_idesc_bf16(128, HD, false, true);    // 128x64, K=128: A from TMEM,
                                                                                // B MN-major
@@ -663,26 +676,29 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       // tiles are the A operands in MODE 0 (rows: keys) and in MODE 1 (rows: queries)
       auto issue_sd = [&](int g, int rb) -> bool {
         const int st = g % BWD_STAGES;
-        if (!mbar_wait(&t_full[st], (g / BWD_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait(sd_empty, (g & 1) ^ 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&t_full[st], (g / BWD_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait_warp(sd_empty, (g & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t a = smem_u32(sA + st * TILE_BYTES), bq = smem_u32(sB + st * TILE_BYTES);
         const uint32_t r0 = smem_u32(sRes + rb * 2 * TILE_BYTES), r1 = r0 + TILE_BYTES;
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < HD / 16; ++k) {
-          // MODE 0: S^T = K_j Q_i^T, dP^T = V_j dO_i^T;  MODE 1: S = Q_i K_j^T, dP = dO_i V_j^T
-          tc_mma_bf16(tmem + BS_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
-                      idesc_sq, k > 0 ? 1u : 0u);
-          tc_mma_bf16(tmem + BDP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024), make_sdesc_sw128(bq + k * 32, 16, 1024),
-                      idesc_sq, k > 0 ? 1u : 0u);
+          for (int k = 0; k < HD / 16; ++k) {
+            // MODE 0: S^T = K_j Q_i^T, dP^T = V_j dO_i^T;  MODE 1: S = Q_i K_j^T, dP = dO_i V_j^T
+            tc_mma_bf16(tmem + BS_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
+                        idesc_sq, k > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + BDP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024),
+                        make_sdesc_sw128(bq + k * 32, 16, 1024), idesc_sq, k > 0 ? 1u : 0u);
+          }
+          tc_commit(sd_full);
         }
-        tc_commit(sd_full);
+        __syncwarp();
         return true;
       };
       bool ok = true;
       int g = 0;
       int idx = bwd_turn_item(0);
-      if (idx < n_items) ok = mbar_wait(&r_full[0], 0, abort_flag) && issue_sd(0, 0);
+      if (idx < n_items) ok = mbar_wait_warp(&r_full[0], 0, abort_flag) && issue_sd(0, 0);
       for (int k = 0; idx < n_items && ok; ++k) {
         const BwdItem w = bwd_item<MODE>(idx, BH, n_t);
         const int n_it = w.it1 - w.it0;
@@ -694,41 +710,47 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
           if (n + 1 < n_it) {
             ok = issue_sd(g + 1, k & 1);
           } else if (nidx < n_items) {
-            ok = mbar_wait(&r_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag) && issue_sd(g + 1, (k + 1) & 1);
+            ok = mbar_wait_warp(&r_full[(k + 1) & 1], ((k + 1) >> 1) & 1, abort_flag) && issue_sd(g + 1, (k + 1) & 1);
           }
           if (!ok) break;
           // the accumulator buffer must have been read out by the epilogue of the item that
           // last used it (item k - 1 for dK/dV, k - 2 for dQ)
           if (n == 0) {
-            const bool got = (MODE == 0) ? mbar_wait(&acc_empty[0], (k & 1) ^ 1, abort_flag)
-                                         : mbar_wait(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag);
+            const bool got = (MODE == 0) ? mbar_wait_warp(&acc_empty[0], (k & 1) ^ 1, abort_flag)
+                                         : mbar_wait_warp(&acc_empty[ab], ((k >> 1) & 1) ^ 1, abort_flag);
             if (!got) { ok = false; break; }
           }
           const int st = g % BWD_STAGES;
-          if (!mbar_wait(ps_full, g & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(ps_full, g & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a = smem_u32(sA + st * TILE_BYTES), bq = smem_u32(sB + st * TILE_BYTES);
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t accum = (n > 0 || kk > 0) ? 1u : 0u;
-            // A: 16 queries (MODE 0) or keys (MODE 1) of P / dZ = 8 TMEM columns per step;
-            // B: the same 16 rows of a [128 x 64] tile, MN-major (2 KB per step)
-            if (MODE == 0) {
-              tc_mma_bf16_ts(acc0, tmem + BP_C + kk * 8, make_sdesc_sw128(bq + kk * 2048, 8192, 1024), idesc_acc,
-                             accum);                                                    // dV += P^T dO_i
-              tc_mma_bf16_ts(acc1, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
-                             accum);                                                    // dK += dZ^T Q_i
-            } else {
-              tc_mma_bf16_ts(acc0, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
-                             accum);                                                    // dQ += dZ K_j
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t accum = (n > 0 || kk > 0) ? 1u : 0u;
+              // A: 16 queries (MODE 0) or keys (MODE 1) of P / dZ = 8 TMEM columns per step;
+              // B: the same 16 rows of a [128 x 64] tile, MN-major (2 KB per step)
+              if (MODE == 0) {
+                tc_mma_bf16_ts(acc0, tmem + BP_C + kk * 8, make_sdesc_sw128(bq + kk * 2048, 8192, 1024), idesc_acc,
+                               accum);                                                    // dV += P^T dO_i
+                tc_mma_bf16_ts(acc1, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
+                               accum);                                                    // dK += dZ^T Q_i
+              } else {
+                tc_mma_bf16_ts(acc0, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
+                               accum);                                                    // dQ += dZ K_j
+              }
             }
+            tc_commit(&t_empty[st]);
+            tc_commit(ps_empty);
           }
-          tc_commit(&t_empty[st]);
-          tc_commit(ps_empty);
+          __syncwarp();
         }
         if (!ok) break;
-        tc_commit(&acc_full[ab]);
-        tc_commit(&r_empty[k & 1]);
+        if (leader) {
+          tc_commit(&acc_full[ab]);
+          tc_commit(&r_empty[k & 1]);
+        }
+        __syncwarp();
         idx = nidx;
       }
     }

@@ -338,8 +338,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         }
     }
   } else if (warp == 1) {
-    if (lane == 0 && rank == 0) {
+    if (rank == 0) {
       // ------------------------------------------------------------ MMA issuer (the leader)
+      // the whole warp runs the loop (descriptors and counters stay warp-uniform); one elected
+      // lane issues the MMAs and commits
+      const bool leader = elect_one_sync();
       constexpr uint32_t idesc = make_idesc_bf16(BMT, BN, A_MN, B_MN);
       int stage = 0;
       uint32_t phase = 0;
@@ -349,32 +352,38 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       for (int t = cl_id; t < ntiles && ok; t += n_cl) {
         int tm, tn, split, kb0, kb1;
         sched.decode(t, tm, tn, split, kb0, kb1);
-        if (CG == 2 ? !mbar_wait_cluster(&tempty_bar[acc], acc_phase ^ 1, abort_flag)
-                    : !mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag))
-          break;
+        const bool got = (CG == 2) ? mbar_wait_cluster(&tempty_bar[acc], acc_phase ^ 1, abort_flag)
+                                   : mbar_wait(&tempty_bar[acc], acc_phase ^ 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t aBase = smem_u32(smem + stage * Cfg::STAGE_BYTES);
           const uint32_t bBase = aBase + Cfg::A_BYTES;
+          if (leader) {
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t ad = A_MN ? make_sdesc_sw128(aBase + k * 2048, 8192, 1024)
-                                     : make_sdesc_sw128(aBase + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? make_sdesc_sw128(bBase + k * 2048, 8192, 1024)
-                                     : make_sdesc_sw128(bBase + k * 32, 16, 1024);
-            if (CG == 2) tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-            else tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < BK / 16; ++k) {
+              const uint64_t ad = A_MN ? make_sdesc_sw128(aBase + k * 2048, 8192, 1024)
+                                       : make_sdesc_sw128(aBase + k * 32, 16, 1024);
+              const uint64_t bd = B_MN ? make_sdesc_sw128(bBase + k * 2048, 8192, 1024)
+                                       : make_sdesc_sw128(bBase + k * 32, 16, 1024);
+              if (CG == 2) tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+              else tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            }
+            if (CG == 2) tc_commit_pair(&empty_bar[stage], 0x3);   // both CTAs' stage is free
+            else tc_commit(&empty_bar[stage]);
           }
-          if (CG == 2) tc_commit_pair(&empty_bar[stage], 0x3);   // both CTAs' stage is free
-          else tc_commit(&empty_bar[stage]);
+          __syncwarp();
           if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        if (CG == 2) tc_commit_pair(&tfull_bar[acc], 0x3);       // both halves of D are ready
-        else tc_commit(&tfull_bar[acc]);
+        if (leader) {
+          if (CG == 2) tc_commit_pair(&tfull_bar[acc], 0x3);     // both halves of D are ready
+          else tc_commit(&tfull_bar[acc]);
+        }
+        __syncwarp();
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }

@@ -263,6 +263,19 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// One lane of a converged warp (elect.sync): the warp runs an issuing role together, so that
+// the values it computes stay warp-uniform, and the elected lane issues the instructions.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+
 // Shared-memory matrix descriptor for tcgen05 (128-byte swizzle, sm_100 version field).
 //   K-major operand  : rows of 64 bf16 (128 B), 8-row groups SBO bytes apart, LBO unused (16).
 //   MN-major operand : 64-element (128 B) MN runs, 8-row K groups SBO bytes apart and
