@@ -145,11 +145,13 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
   uint64_t* q_empty = q_full + 2;                // 2
   uint64_t* kv_full = q_empty + 2;               // KV_STAGES
   uint64_t* kv_empty = kv_full + KV_STAGES;      // KV_STAGES
+  // S(G) is committed after the group's previous P.V product was issued, so its completion
+  // also means that product is done (P columns free, O stable); and the MMA issuer writes a
+  // group's next S only after that group's P is in, so its S has been read.  Neither needs a
+  // barrier of its own.
   uint64_t* s_full = kv_empty + KV_STAGES;       // 2 (per group)
-  uint64_t* s_empty = s_full + 2;                // 2
-  uint64_t* p_full = s_empty + 2;                // 2
-  uint64_t* p_empty = p_full + 2;                // 2
-  uint64_t* o_done = p_empty + 2;                // 2
+  uint64_t* p_full = s_full + 2;                 // 2
+  uint64_t* o_done = p_full + 2;                 // 2
   uint64_t* merge_full = o_done + 2;             // 1
   uint64_t* merge_empty = merge_full + 1;        // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(merge_empty + 1);
@@ -164,9 +166,7 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
       mbar_init(&p_full[i], 128);
-      mbar_init(&p_empty[i], 1);
       mbar_init(&o_done[i], 1);
     }
     for (int s = 0; s < KV_STAGES; ++s) {
@@ -245,54 +245,55 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         int bh;
         items.get(cur.t, cur.qt, bh);
       }
-      int cs0 = 0, cs1 = 0;    // S issues per group
       int co0 = 0, co1 = 0;    // O issues per group
       bool ok = true;
+      // operand descriptors of the first Q, K and V buffers; each MMA's is derived by an add
+      const uint64_t dQ0 = make_sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK0 = make_sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = make_sdesc_sw128(smem_u32(sV), 8192, 1024);
       auto issue_s = [&](const It& it) -> bool {
         const int g = it.G & 1, s = it.G % KV_STAGES, qb = it.k & 1;
         if (it.j == 0 && !mbar_wait_warp(&q_full[qb], (it.k >> 1) & 1, abort_flag)) return false;
         if (!mbar_wait_warp(&kv_full[s], (it.G / KV_STAGES) & 1, abort_flag)) return false;
-        const int cs = g ? cs1 : cs0;
-        if (!mbar_wait_warp(&s_empty[g], (cs & 1) ^ 1, abort_flag)) return false;
-        if (g) ++cs1; else ++cs0;
         tc_fence_after();
-        const uint32_t aQ = smem_u32(sQ + qb * TILE_BYTES);
-        const uint32_t bK = smem_u32(sK + s * TILE_BYTES);
+        const uint64_t aQ = sdesc_add(dQ0, qb * TILE_BYTES), bK = sdesc_add(dK0, s * TILE_BYTES);
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk)
-            tc_mma_bf16(tmem + S_COL + g * KT, make_sdesc_sw128(aQ + kk * 32, 16, 1024),
-                        make_sdesc_sw128(bK + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + S_COL + g * KT, sdesc_add(aQ, kk * 32), sdesc_add(bK, kk * 32), idesc_s,
+                        kk > 0 ? 1u : 0u);
           tc_commit(&s_full[g]);
         }
         __syncwarp();
         return true;
       };
+      // S of each group's first tile; then per tile: P.V of it and S of the group's next tile
+      It nx = next(cur);
       if (valid(cur)) ok = issue_s(cur);
+      if (ok && valid(nx)) ok = issue_s(nx);
       while (ok && valid(cur)) {
-        const It nx = next(cur);
-        if (valid(nx) && !issue_s(nx)) break;
         const int g = cur.G & 1, s = cur.G % KV_STAGES;
         const int co = g ? co1 : co0;
         if (!mbar_wait_warp(&p_full[g], co & 1, abort_flag)) break;
         if (g) ++co1; else ++co0;
         tc_fence_after();
         const bool first_of_group = (cur.j < 2);          // the group's first tile of this item
-        const uint32_t bV = smem_u32(sV + s * TILE_BYTES);
+        const uint64_t bV = sdesc_add(dV0, s * TILE_BYTES);
         // A: 16 keys of P = 8 TMEM columns per step; B: 16 rows of V, MN-major
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < KT / 16; ++kk)
-            tc_mma_bf16_ts(tmem + O_COL + g * HD, tmem + P_COL + g * 64 + kk * 8,
-                           make_sdesc_sw128(bV + kk * 2048, 8192, 1024), idesc_o,
+            tc_mma_bf16_ts(tmem + O_COL + g * HD, tmem + P_COL + g * 64 + kk * 8, sdesc_add(bV, kk * 2048), idesc_o,
                            (kk > 0 || !first_of_group) ? 1u : 0u);
           tc_commit(&kv_empty[s]);
-          tc_commit(&p_empty[g]);
           if (cur.j + 2 > cur.qt) tc_commit(&o_done[g]);    // the group's last tile of this item
           if (cur.j == cur.qt) tc_commit(&q_empty[cur.k & 1]);
         }
         __syncwarp();
+        const It n2 = next(nx);                           // the same group's next tile
+        if (valid(n2) && !issue_s(n2)) break;
         cur = nx;
+        nx = n2;
       }
     }
   } else {
@@ -327,8 +328,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
           // the true max and writes P again if it grew past the threshold
           m_ref = (diag ? s_chunk32_max<true>(srow, r) : s_chunk32_max<false>(srow, r)) * scale_log2;
         }
-        // the group's previous P.V MMA must be done: P columns free, O stable
-        if (!mbar_wait_warp(&p_empty[grp], (c & 1) ^ 1, abort_flag)) { ok = false; break; }
         // one pass: P against the current m_ref, and the tile's row max alongside
         float mx;
         sum = diag ? p_row_store<true, true>(srow, r, scale_log2, m_ref, pcol, &mx)
@@ -361,7 +360,6 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict_
         }
         l += sum;
         tc_fence_before();
-        mbar_arrive(&s_empty[grp]);
         // an O row handed over at the previous item must be read before this group's next MMA
         if (pending) {
           if (!mbar_wait_warp(merge_empty, (hcount & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -674,21 +672,24 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
                                                                                // B MN-major
       // S / dP of the CTA's g-th streamed tile, read against resident buffer rb: the resident
       // tiles are the A operands in MODE 0 (rows: keys) and in MODE 1 (rows: queries)
+      // operand descriptors of the first buffers (K-major for S / dP, MN-major for the
+      // accumulations); each MMA's is derived by an add
+      const uint64_t dA_k = make_sdesc_sw128(smem_u32(sA), 16, 1024), dA_mn = make_sdesc_sw128(smem_u32(sA), 8192, 1024);
+      const uint64_t dB_k = make_sdesc_sw128(smem_u32(sB), 16, 1024), dB_mn = make_sdesc_sw128(smem_u32(sB), 8192, 1024);
+      const uint64_t dR_k = make_sdesc_sw128(smem_u32(sRes), 16, 1024);
       auto issue_sd = [&](int g, int rb) -> bool {
         const int st = g % BWD_STAGES;
         if (!mbar_wait_warp(&t_full[st], (g / BWD_STAGES) & 1, abort_flag)) return false;
         if (!mbar_wait_warp(sd_empty, (g & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t a = smem_u32(sA + st * TILE_BYTES), bq = smem_u32(sB + st * TILE_BYTES);
-        const uint32_t r0 = smem_u32(sRes + rb * 2 * TILE_BYTES), r1 = r0 + TILE_BYTES;
+        const uint64_t a = sdesc_add(dA_k, st * TILE_BYTES), bq = sdesc_add(dB_k, st * TILE_BYTES);
+        const uint64_t r0 = sdesc_add(dR_k, rb * 2 * TILE_BYTES), r1 = sdesc_add(r0, TILE_BYTES);
         if (leader) {
 #pragma unroll
           for (int k = 0; k < HD / 16; ++k) {
             // MODE 0: S^T = K_j Q_i^T, dP^T = V_j dO_i^T;  MODE 1: S = Q_i K_j^T, dP = dO_i V_j^T
-            tc_mma_bf16(tmem + BS_C, make_sdesc_sw128(r0 + k * 32, 16, 1024), make_sdesc_sw128(a + k * 32, 16, 1024),
-                        idesc_sq, k > 0 ? 1u : 0u);
-            tc_mma_bf16(tmem + BDP_C, make_sdesc_sw128(r1 + k * 32, 16, 1024),
-                        make_sdesc_sw128(bq + k * 32, 16, 1024), idesc_sq, k > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + BS_C, sdesc_add(r0, k * 32), sdesc_add(a, k * 32), idesc_sq, k > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + BDP_C, sdesc_add(r1, k * 32), sdesc_add(bq, k * 32), idesc_sq, k > 0 ? 1u : 0u);
           }
           tc_commit(sd_full);
         }
@@ -723,7 +724,7 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
           const int st = g % BWD_STAGES;
           if (!mbar_wait_warp(ps_full, g & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a = smem_u32(sA + st * TILE_BYTES), bq = smem_u32(sB + st * TILE_BYTES);
+          const uint64_t a = sdesc_add(dA_mn, st * TILE_BYTES), bq = sdesc_add(dB_mn, st * TILE_BYTES);
           if (leader) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
@@ -731,13 +732,10 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
               // A: 16 queries (MODE 0) or keys (MODE 1) of P / dZ = 8 TMEM columns per step;
               // B: the same 16 rows of a [128 x 64] tile, MN-major (2 KB per step)
               if (MODE == 0) {
-                tc_mma_bf16_ts(acc0, tmem + BP_C + kk * 8, make_sdesc_sw128(bq + kk * 2048, 8192, 1024), idesc_acc,
-                               accum);                                                    // dV += P^T dO_i
-                tc_mma_bf16_ts(acc1, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
-                               accum);                                                    // dK += dZ^T Q_i
+                tc_mma_bf16_ts(acc0, tmem + BP_C + kk * 8, sdesc_add(bq, kk * 2048), idesc_acc, accum);   // dV += P^T dO_i
+                tc_mma_bf16_ts(acc1, tmem + BDS_C + kk * 8, sdesc_add(a, kk * 2048), idesc_acc, accum);   // dK += dZ^T Q_i
               } else {
-                tc_mma_bf16_ts(acc0, tmem + BDS_C + kk * 8, make_sdesc_sw128(a + kk * 2048, 8192, 1024), idesc_acc,
-                               accum);                                                    // dQ += dZ K_j
+                tc_mma_bf16_ts(acc0, tmem + BDS_C + kk * 8, sdesc_add(a, kk * 2048), idesc_acc, accum);   // dQ += dZ K_j
               }
             }
             tc_commit(&t_empty[st]);

@@ -344,6 +344,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       // lane issues the MMAs and commits
       const bool leader = elect_one_sync();
       constexpr uint32_t idesc = make_idesc_bf16(BMT, BN, A_MN, B_MN);
+      // operand descriptors of stage 0; each MMA's is derived by an add
+      const uint64_t dA0 = A_MN ? make_sdesc_sw128(smem_u32(smem), 8192, 1024) : make_sdesc_sw128(smem_u32(smem), 16, 1024);
+      const uint64_t dB0 = B_MN ? make_sdesc_sw128(smem_u32(smem) + Cfg::A_BYTES, 8192, 1024)
+                                : make_sdesc_sw128(smem_u32(smem) + Cfg::A_BYTES, 16, 1024);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -360,15 +364,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_warp(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t aBase = smem_u32(smem + stage * Cfg::STAGE_BYTES);
-          const uint32_t bBase = aBase + Cfg::A_BYTES;
+          const uint64_t aBase = sdesc_add(dA0, stage * Cfg::STAGE_BYTES);
+          const uint64_t bBase = sdesc_add(dB0, stage * Cfg::STAGE_BYTES);
           if (leader) {
 #pragma unroll
             for (int k = 0; k < BK / 16; ++k) {
-              const uint64_t ad = A_MN ? make_sdesc_sw128(aBase + k * 2048, 8192, 1024)
-                                       : make_sdesc_sw128(aBase + k * 32, 16, 1024);
-              const uint64_t bd = B_MN ? make_sdesc_sw128(bBase + k * 2048, 8192, 1024)
-                                       : make_sdesc_sw128(bBase + k * 32, 16, 1024);
+              const uint64_t ad = sdesc_add(aBase, A_MN ? k * 2048 : k * 32);
+              const uint64_t bd = sdesc_add(bBase, B_MN ? k * 2048 : k * 32);
               if (CG == 2) tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
               else tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
             }
