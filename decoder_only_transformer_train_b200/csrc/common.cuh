@@ -148,5 +148,22 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return d;
 }
 
+// gelu(x) and gelu'(x) for two values with paired fp32 arithmetic and the hardware tanh
+// (results rounded to bf16).  With p = (1 + t) / 2 and t = tanh(A x (1 + C x^2)):
+//   gelu(x) = x p,   gelu'(x) = p + (x / 2) A (1 - t^2)(1 + 3 C x^2) = p (1 + x A (1 - t)(1 + 3 C x^2)),
+// using 1 - t^2 = (1 - t)(1 + t): eleven paired operations and two tanh per pair.
+__device__ __forceinline__ void gelu2_and_grad_fast(float2 x, float2& g, float2& gp) {
+  const float2 one = make_float2(1.0f, 1.0f), half = make_float2(0.5f, 0.5f);
+  const float2 x2 = fmul2(x, x);
+  const float2 xa = fmul2(x, make_float2(GELU_A, GELU_A));
+  const float2 arg = fmul2(xa, ffma2(x2, make_float2(GELU_C, GELU_C), one));
+  const float2 t = make_float2(tanh_approx(arg.x), tanh_approx(arg.y));
+  const float2 p = ffma2(t, half, half);
+  g = fmul2(x, p);
+  const float2 omt = ffma2(t, make_float2(-1.0f, -1.0f), one);
+  const float2 d = ffma2(x2, make_float2(3.0f * GELU_C, 3.0f * GELU_C), one);
+  gp = fmul2(p, ffma2(fmul2(xa, omt), d, one));
+}
+
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 __host__ __device__ __forceinline__ long long cdivll(long long a, long long b) { return (a + b - 1) / b; }

@@ -473,10 +473,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int j = 0; j < 32; ++j) b[j] = (use_bias && n0 + j < ep.N) ? ep.bias[n0 + j] : 0.f;
           }
           if (kind == EPI_GELU_FWD) {
-            // gelu(u) and gelu'(u) from one tanh; gelu'(u) is what the backward needs
+            // gelu(u) and gelu'(u) from one tanh, in pairs; gelu'(u) is what the backward needs
             float gp[32], g[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) gelu_tanh_and_grad_fast(alpha * v[j] + b[j], g[j], gp[j]);
+            for (int j = 0; j < 32; j += 2) {
+              float2 gl, gd;
+              gelu2_and_grad_fast(ffma2(make_float2(alpha, alpha), make_float2(v[j], v[j + 1]), make_float2(b[j], b[j + 1])),
+                                  gl, gd);
+              g[j] = gl.x; g[j + 1] = gl.y;
+              gp[j] = gd.x; gp[j + 1] = gd.y;
+            }
             int bx = E.take();
             box_put_bf16(E.box(bx), lane, gp);
             E.store(bx, &tmOut2, n0, m_warp);
@@ -490,13 +496,22 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             box_get_bf16(E.box(bx), lane, u);
             __syncwarp();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] = alpha * v[j] * u[j];
+            for (int j = 0; j < 32; j += 2) {
+              const float2 o = fmul2(fmul2(make_float2(alpha, alpha), make_float2(v[j], v[j + 1])),
+                                     make_float2(u[j], u[j + 1]));
+              u[j] = o.x;
+              u[j + 1] = o.y;
+            }
             box_put_bf16(E.box(bx), lane, u);
             E.store(bx, &tmOut, n0, m_warp);
             if (c + depth < nch) load_chunk(c + depth);
           } else {   // EPI_STORE_ACT, EPI_CE_FWD
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = alpha * v[j] + b[j];
+            for (int j = 0; j < 32; j += 2) {
+              const float2 o = ffma2(make_float2(alpha, alpha), make_float2(v[j], v[j + 1]), make_float2(b[j], b[j + 1]));
+              v[j] = o.x;
+              v[j + 1] = o.y;
+            }
             const int bx = E.take();
             box_put_bf16(E.box(bx), lane, v);
             E.store(bx, &tmOut, n0, m_warp);
@@ -509,10 +524,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const int n1 = n0 + hh * 16;
             if (!ok || n1 >= ep.N) continue;
             float o[16];
+            if (kind == EPI_SPLITK) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float bj = (use_bias && n1 + j < ep.N) ? ep.bias[n1 + j] : 0.f;
-              o[j] = (kind == EPI_SPLITK) ? v[hh * 16 + j] : alpha * v[hh * 16 + j] + bj;
+              for (int j = 0; j < 16; ++j) o[j] = v[hh * 16 + j];
+            } else {
+              float bj[16];
+              if (use_bias && n1 + 16 <= ep.N) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float4 q4 = reinterpret_cast<const float4*>(ep.bias + n1)[i];
+                  bj[4 * i] = q4.x; bj[4 * i + 1] = q4.y; bj[4 * i + 2] = q4.z; bj[4 * i + 3] = q4.w;
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) bj[j] = (use_bias && n1 + j < ep.N) ? ep.bias[n1 + j] : 0.f;
+              }
+#pragma unroll
+              for (int j = 0; j < 16; j += 2) {
+                const float2 r2 = ffma2(make_float2(alpha, alpha), make_float2(v[hh * 16 + j], v[hh * 16 + j + 1]),
+                                        make_float2(bj[j], bj[j + 1]));
+                o[j] = r2.x;
+                o[j + 1] = r2.y;
+              }
             }
             int bx;
             if (has_in) {
@@ -522,7 +555,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               box_get_f32(E.box(bx), lane, in);
               __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 16; ++j) o[j] += in[j];
+              for (int j = 0; j < 16; j += 2) {
+                const float2 r2 = fadd2(make_float2(o[j], o[j + 1]), make_float2(in[j], in[j + 1]));
+                o[j] = r2.x;
+                o[j + 1] = r2.y;
+              }
             } else {
               bx = E.take();
             }
