@@ -228,7 +228,10 @@ def barrier(world):
 def cpu_oracle_configs():
     """Wall time of the oracle (fp32, as it stands) on the small workloads: the tiny model's
     full step (B=2, T=64: forward, backward, clip, AdamW), the 124M B=1 x T=1024 forward +
-    backward on one thread, and one 124M step on B=4 x T=1024 on all host threads."""
+    backward on one thread, one 124M step on B=4 x T=1024 on all host threads, the
+    classifier-head stress (lm_head + softmax + cross-entropy forward and backward at the
+    unpadded vocabulary 50257, timed on 1024 of its 16384 rows and scaled), and the medium
+    model's B=1 x T=1024 forward + backward."""
     import torch
     import oracle as O
     from decoder_only_transformer_train_b200 import synthetic as S
@@ -259,6 +262,31 @@ def cpu_oracle_configs():
     out["gpt2_124m_b1_fwd_bwd_1_thread_s"] = round(t1, 2)
     out["gpt2_124m_tokens_per_s_1_thread"] = round(1024 / t1, 1)
     out["gpt2_124m_b4_step_s"] = round(step(params, cfg, 4, 1024, 2), 2)
+    del params
+    # classifier head at V=50257: hidden states N(0,1), tied weight N(0,0.02), uniform targets
+    # with 1% ignored; 1024 rows of the 16384 (the oracle's cost is linear in the rows)
+    g = torch.Generator().manual_seed(7)
+    rows, V, C = 1024, 50257, 768
+    h = torch.randn(rows, C, generator=g)
+    W = torch.randn(V, C, generator=g) * 0.02
+    y = torch.randint(0, V, (rows,), generator=g)
+    y[torch.rand(rows, generator=g) < 0.01] = O.IGNORE_INDEX
+    t0 = time.perf_counter()
+    z = h @ W.t()
+    _, lse, count = O.cross_entropy_forward(z, y)
+    dz = O.cross_entropy_backward(z, y, lse, count, 1.0)
+    _ = dz @ W
+    _ = dz.t() @ h
+    out["c4_classifier_50257_s"] = round((time.perf_counter() - t0) * (16384 / rows), 2)
+    out["c4_sample"] = f"{rows} of 16384 rows, scaled"
+    del z, dz, W
+    mcfg = O.Config(n_layer=24, n_embd=1024, n_head=16)
+    mparams = O.init_params(mcfg, 1, dtype=torch.float32)
+    x, y = S.token_batch(4, 1, 1024, mcfg.vocab_size)
+    t0 = time.perf_counter()
+    _, cache = O.forward(mparams, mcfg, torch.from_numpy(x), torch.from_numpy(y))
+    O.backward(mparams, mcfg, cache)
+    out["c5_medium_b1_fwd_bwd_s"] = round(time.perf_counter() - t0, 2)
     out["threads"] = threads
     return out
 
