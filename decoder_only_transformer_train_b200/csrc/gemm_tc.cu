@@ -165,6 +165,18 @@ __device__ __forceinline__ void box_get_f32(const uint8_t* box, int r, float* v)
   }
 }
 
+// Epilogue classes, one kernel instantiation each, so that a kernel carries only its own
+// epilogue code (the fused ones compile to straight-line code for their kind; the plain
+// class covers bf16 / fp32 stores, fp32 accumulation and split-K partials at run time).
+enum EpiClass : int { EK_PLAIN = 0, EK_RESID = 1, EK_GELU_FWD = 2, EK_GELU_BWD = 3, EK_CE = 4 };
+inline int epi_class(int kind) {
+  return kind == EPI_RESID_F32 ? EK_RESID
+         : kind == EPI_GELU_FWD ? EK_GELU_FWD
+         : kind == EPI_GELU_BWD ? EK_GELU_BWD
+         : kind == EPI_CE_FWD   ? EK_CE
+                                : EK_PLAIN;
+}
+
 __device__ __forceinline__ bool kind_has_bias(int kind) {
   return kind == EPI_STORE_ACT || kind == EPI_STORE_F32 || kind == EPI_RESID_F32 || kind == EPI_GELU_FWD;
 }
@@ -233,7 +245,7 @@ struct EpiRing {
   }
 };
 
-template <int BN, bool A_MN, bool B_MN, int CG>
+template <int BN, bool A_MN, bool B_MN, int CG, int EK>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmIn,
@@ -406,7 +418,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     E.stores = 0;
     E.abort_flag = abort_flag;
     E.lane = lane;
-    const int kind = ep.kind;
+    // the fused classes fix their kind at compile time
+    const int kind = (EK == EK_RESID)      ? (int)EPI_RESID_F32
+                     : (EK == EK_GELU_FWD) ? (int)EPI_GELU_FWD
+                     : (EK == EK_GELU_BWD) ? (int)EPI_GELU_BWD
+                     : (EK == EK_CE)       ? (int)EPI_CE_FWD
+                                           : ep.kind;
     const bool out_bf16 = kind_out_bf16(kind);
     const bool use_bias = ep.bias != nullptr && kind_has_bias(kind);
     const float alpha = ep.alpha;
@@ -414,7 +431,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // accumulator (fp32, two 16-column boxes per 32-column chunk) or the GELU pre-activation
     // (bf16, one box per chunk).  The first NB boxes of them are requested before the
     // accumulator is ready; later ones as boxes retire.
-    const bool has_in = (kind == EPI_RESID_F32 || kind == EPI_ACCUM_F32 || kind == EPI_GELU_BWD);
+    const bool has_in = (EK == EK_RESID || kind == EPI_ACCUM_F32 || EK == EK_GELU_BWD);
     const CUtensorMap* in_map = (kind == EPI_ACCUM_F32) ? &tmOut : &tmIn;
     const int depth = out_bf16 ? NB : NB / 2;   // chunks loaded ahead
     int acc = 0;
@@ -446,7 +463,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       if (has_in)
         for (int c = 0; c < min(depth, nch); ++c) load_chunk(c);
       CeRowState ce{-INFINITY, 0.0f, -INFINITY, 0.0f, 0x7fffffff};
-      const int y_row = (kind == EPI_CE_FWD && m < ep.M) ? ep.targets[m] : -1;
+      const int y_row = (EK == EK_CE && m < ep.M) ? ep.targets[m] : -1;
       if (!mbar_wait_warp(&tfull_bar[acc], acc_phase, abort_flag)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll 1
@@ -459,7 +476,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         float v[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-        if (kind == EPI_CE_FWD && m < ep.M) ce_row_chunk(n0, min(32, ep.N - n0), y_row, v, ce);
+        if (EK == EK_CE && m < ep.M) ce_row_chunk(n0, min(32, ep.N - n0), y_row, v, ce);
         if (out_bf16) {
           float b[32];
           if (use_bias && n0 + 32 <= ep.N) {
@@ -472,7 +489,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
             for (int j = 0; j < 32; ++j) b[j] = (use_bias && n0 + j < ep.N) ? ep.bias[n0 + j] : 0.f;
           }
-          if (kind == EPI_GELU_FWD) {
+          if (EK == EK_GELU_FWD) {
             // gelu(u) and gelu'(u) from one tanh, in pairs; gelu'(u) is what the backward needs
             float gp[32], g[32];
 #pragma unroll
@@ -489,7 +506,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             bx = E.take();
             box_put_bf16(E.box(bx), lane, g);
             E.store(bx, &tmOut, n0, m_warp);
-          } else if (kind == EPI_GELU_BWD) {
+          } else if (EK == EK_GELU_BWD) {
             const int bx = (in_first + c) % NB;
             if (!E.wait_load(bx)) { ok = false; break; }
             float u[32];
@@ -569,7 +586,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (ok && has_in && c + depth < nch) load_chunk(c + depth);
         }
       }
-      if (kind == EPI_CE_FWD && m < ep.M) {
+      if (EK == EK_CE && m < ep.M) {
         CePartial p;
         p.max = ce.mx;
         p.sum = ce.sum;
@@ -685,11 +702,11 @@ int encode_epi_box(CUtensorMap* map, bool bf16_elems, const void* base, uint64_t
                                 CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-template <int BN, bool A_MN, bool B_MN, int CG>
+template <int BN, bool A_MN, bool B_MN, int CG, int EK>
 int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
               const CUtensorMap& tin, const CUtensorMap& tout2, TileSched sched, const EpiParams& ep, int num_sms) {
   using Cfg = TileCfg<BN, CG>;
-  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, CG>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, CG, EK>;
   // co-resident CTA groups of this kernel on the current device (its shared-memory limit set)
   const int max_groups = per_device_once((const void*)kern, [&]() -> int {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) != cudaSuccess)
@@ -735,6 +752,21 @@ int launch_tc(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, con
   }
   note_kernel_launches(1);
   return cudaGetLastError() == cudaSuccess ? 0 : -3;
+}
+
+// launch_tc for the epilogue class of ep.kind
+template <int BN, bool A_MN, bool B_MN, int CG>
+int launch_tc_ek(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tout,
+                 const CUtensorMap& tin, const CUtensorMap& tout2, TileSched sched, const EpiParams& ep, int num_sms) {
+  switch (epi_class(ep.kind)) {
+    case EK_RESID: return launch_tc<BN, A_MN, B_MN, CG, EK_RESID>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
+    case EK_GELU_FWD:
+      return launch_tc<BN, A_MN, B_MN, CG, EK_GELU_FWD>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
+    case EK_GELU_BWD:
+      return launch_tc<BN, A_MN, B_MN, CG, EK_GELU_BWD>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
+    case EK_CE: return launch_tc<BN, A_MN, B_MN, CG, EK_CE>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
+    default: return launch_tc<BN, A_MN, B_MN, CG, EK_PLAIN>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
+  }
 }
 
 }  // namespace
@@ -876,9 +908,9 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   if (rc) return rc;
 #define LAUNCH_BN(BNV, CGV)                                                                                   \
   do {                                                                                                        \
-    if (!a_mn && !b_mn) rc = launch_tc<BNV, false, false, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);   \
-    else if (!a_mn && b_mn) rc = launch_tc<BNV, false, true, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms); \
-    else rc = launch_tc<BNV, true, true, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);                    \
+    if (!a_mn && !b_mn) rc = launch_tc_ek<BNV, false, false, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);   \
+    else if (!a_mn && b_mn) rc = launch_tc_ek<BNV, false, true, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms); \
+    else rc = launch_tc_ek<BNV, true, true, CGV>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);                    \
   } while (0)
   if (CG == 1) {
     if (BN == 256) LAUNCH_BN(256, 1);
@@ -888,7 +920,7 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
     if (BN == 256) LAUNCH_BN(256, 2);
     else if (BN == 192) {
       if (b_mn) return -1;   // excluded by the tile choice
-      rc = launch_tc<192, false, false, 2>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);
+      rc = launch_tc_ek<192, false, false, 2>(st, ta, tb, tout, tin, tout2, sched, run, num_sms);
     } else LAUNCH_BN(128, 2);
   }
 #undef LAUNCH_BN
