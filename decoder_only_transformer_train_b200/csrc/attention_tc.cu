@@ -544,23 +544,6 @@ __device__ __forceinline__ int bwd_turn_item(int k) {
 // (the bias gradient of c_attn, before the bf16 rounding of dqkv): row (tile * B + b) * 4 + q,
 // columns [0, 3C), sums over the 32 rows of TMEM lane quarter q of the 128-row tile; every
 // (row, column) is written by exactly one item of one of the two kernels.
-// Column sums of one warp's 32 rows of 16 values (x[j] = row `lane`, column j): lane l returns
-// the sum of column l >> 1 (lanes l and l ^ 1 agree).  Each step halves the values a lane
-// keeps, adding its partner's half: 8 + 4 + 2 + 1 shuffles, then one for the last pair.
-__device__ __forceinline__ float warp_colsum16(float (&x)[16], int lane) {
-#pragma unroll
-  for (int s = 16, n = 16; s >= 2; s >>= 1, n >>= 1) {
-    const bool upper = (lane & s) != 0;
-#pragma unroll
-    for (int j = 0; j < n / 2; ++j) {
-      const float send = upper ? x[j] : x[j + n / 2];
-      const float keep = upper ? x[j + n / 2] : x[j];
-      x[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
-    }
-  }
-  return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
-}
-
 template <int MODE>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
 attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,

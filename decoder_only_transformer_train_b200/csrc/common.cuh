@@ -62,6 +62,23 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   return v;
 }
 
+// Column sums of one warp's 32 rows of 16 values (x[j] = row `lane`, column j): lane l returns
+// the sum of column l >> 1 (lanes l and l ^ 1 agree).  Each step halves the values a lane
+// keeps, adding its partner's half: 8 + 4 + 2 + 1 shuffles, then one for the last pair.
+__device__ __forceinline__ float warp_colsum16(float (&x)[16], int lane) {
+#pragma unroll
+  for (int s = 16, n = 16; s >= 2; s >>= 1, n >>= 1) {
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int j = 0; j < n / 2; ++j) {
+      const float send = upper ? x[j] : x[j + n / 2];
+      const float keep = upper ? x[j + n / 2] : x[j];
+      x[j] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+    }
+  }
+  return x[0] + __shfl_xor_sync(0xffffffffu, x[0], 1);
+}
+
 // ---------------------------------------------------------------- GELU (tanh form)
 // gelu(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3)))  -- the approximation GPT-2
 // used ("Karpathy's Zero to Hero, Lecture 9" notes, section "1:48:25 – 2:00:19").

@@ -16,7 +16,8 @@ enum EpiKind : int {
   EPI_ACCUM_F32 = 2,   // C(f32) += alpha*D                 (weight gradients)
   EPI_RESID_F32 = 3,   // C(f32) = aux(f32) + alpha*D + bias (residual stream)
   EPI_GELU_FWD = 4,    // u = alpha*D + bias; aux_out(act) = gelu'(u); C(act) = gelu(u)
-  EPI_GELU_BWD = 5,    // C(act) = alpha*D * aux(act)   (aux: the gelu'(u) the forward kept)
+  EPI_GELU_BWD = 5,    // C(act) = alpha*D * aux(act)   (aux: the gelu'(u) the forward kept); optional
+                       // column sums of C per 32-row group (the c_fc bias gradient's partials)
   EPI_CE_FWD = 6,      // C(act) = alpha*D (logits) + per-(row, column-tile) softmax partials
   EPI_SPLITK = 7,      // ws[split][m][n] = D   (internal: split-K partial products)
 };
@@ -48,6 +49,9 @@ struct EpiParams {
   // EPI_SPLITK
   float* ws;
   int kb_per_split;
+  // EPI_GELU_BWD (optional): column sums of C before its bf16 rounding, one fp32 row per
+  // 32-row group: colsum_part[(m / 32) * N + n] = sum over the group's rows m < M of C[m, n]
+  float* colsum_part;
 };
 
 inline EpiParams epi_make(int kind, void* C, long long ldc) {

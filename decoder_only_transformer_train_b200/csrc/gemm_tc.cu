@@ -521,6 +521,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
             box_put_bf16(E.box(bx), lane, u);
             E.store(bx, &tmOut, n0, m_warp);
+            if (ep.colsum_part != nullptr) {
+              // the warp's 32 rows summed per column (rows past M left out), 16 columns per pass
+              float* prow = ep.colsum_part + (long long)(m_warp >> 5) * ep.N;
+#pragma unroll
+              for (int h16 = 0; h16 < 2; ++h16) {
+                float x[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) x[j] = (m < ep.M) ? u[16 * h16 + j] : 0.f;
+                const float cs = warp_colsum16(x, lane);
+                const int n = n0 + 16 * h16 + (lane >> 1);
+                if ((lane & 1) == 0 && n < ep.N) prow[n] = cs;
+              }
+            }
             if (c + depth < nch) load_chunk(c + depth);
           } else {   // EPI_STORE_ACT, EPI_CE_FWD
 #pragma unroll

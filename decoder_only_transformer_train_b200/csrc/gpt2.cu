@@ -110,6 +110,7 @@ struct gpt2_ctx {
   void* dattn = nullptr;
   float* attnD = nullptr;
   float* attn_bias_part = nullptr;   // c_attn bias column sums from the attention backward
+  float* fc_bias_part = nullptr;     // c_fc bias column sums per 32 rows, from the c_proj dX GEMM
   float* ln_part = nullptr;
   int ln_blocks = 0;
   float* colsum_part = nullptr;
@@ -455,6 +456,10 @@ int backward_impl(gpt2_ctx* c) {
     e = epi_make(EPI_GELU_BWD, c->d4c, 4 * C);
     e.aux = a.fc_pre;
     e.ld_aux = 4 * C;
+    // the tensor-core path also leaves the column sums of d4C (the c_fc bias gradient) per
+    // 32-row group, so d4C is not read again for them
+    const bool fused_fc_bias = c->bf16 && c->fc_bias_part != nullptr;
+    if (fused_fc_bias) e.colsum_part = c->fc_bias_part;
     {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * 4 * Cd * Cd, 0);
       RC(gemm(c, N, 4 * C, C, c->dres_act, C, false, W(c, pi(MPROJ_W)), 4 * C, true, e));
@@ -464,7 +469,11 @@ int backward_impl(gpt2_ctx* c) {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * 4 * Cd * Cd, 0);
       RC(gemm(c, 4 * C, C, N, c->d4c, 4 * C, true, a.ln2, C, true, e));
     }
-    {
+    if (fused_fc_bias) {
+      const int rows = cdiv(N, 32);
+      PROF(PROF_BIAS, 0, 4.0 * rows * 4 * Cd);
+      RC(launch_colsum_reduce(st, c->fc_bias_part, rows, 4 * C, G(c, pi(FC_B))));
+    } else {
       PROF(PROF_BIAS, 0, A * Nd * 4 * Cd);
       RC(launch_colsum(st, c->bf16, c->d4c, 4 * C, N, 4 * C, c->colsum_part, ncs, G(c, pi(FC_B))));
     }
@@ -712,6 +721,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
   AL(dalloc(c, &c->attnD, N * H));
   if (c->bf16 && C / H == 64)
     AL(dalloc(c, &c->attn_bias_part, (size_t)attn_bwd_bias_rows(g.max_batch, g.block_size) * 3 * C));
+  if (c->bf16) AL(dalloc(c, &c->fc_bias_part, (size_t)cdiv(g.max_batch * g.block_size, 32) * 4 * C));
   c->ln_blocks = layernorm_bwd_blocks(c->num_sms);
   AL(dalloc(c, &c->ln_part, (size_t)c->ln_blocks * 3 * C));
   AL(dalloc(c, &c->colsum_part, (size_t)colsum_chunks((int)N) * 4 * C));
