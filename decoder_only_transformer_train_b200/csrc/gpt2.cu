@@ -109,8 +109,14 @@ struct gpt2_ctx {
   void* dqkv = nullptr;
   void* dattn = nullptr;
   float* attnD = nullptr;
-  float* attn_bias_part = nullptr;   // c_attn bias column sums from the attention backward
-  float* fc_bias_part = nullptr;     // c_fc bias column sums per 32 rows, from the c_proj dX GEMM
+  // Partial column sums that the backward leaves behind and one batched launch at its end
+  // reduces: per layer, the c_attn bias sums from the attention backward and the c_fc bias
+  // sums per 32 rows from the c_proj dX GEMM; per LayerNorm (ln_1 and ln_2 of each layer, then
+  // ln_f), the weight, bias and upstream Linear bias sums per LayerNorm backward block.
+  float* attn_bias_part = nullptr;
+  size_t attn_bias_stride = 0;
+  float* fc_bias_part = nullptr;
+  size_t fc_bias_stride = 0;
   float* ln_part = nullptr;
   int ln_blocks = 0;
   float* colsum_part = nullptr;
@@ -435,12 +441,24 @@ int backward_impl(gpt2_ctx* c) {
   const int lf = lnf_w_index(g);
   float* xL = c->resid + (long long)L * c->Nmax * C;
   const double ln_bwd_bytes = Nd * Cd * (4.0 * 3 + 2.0 * A) + 8.0 * Nd;   // dy, x, dres in; dres, dres_act out
+  // the parameter and bias gradients whose partial rows are reduced in one launch at the end
+  std::vector<ColsumJob> jobs;
+  jobs.reserve(8 * L + 3);
+  const size_t ln_slot = (size_t)c->ln_blocks * 3 * C;
+  // LayerNorm partial row: [dy * xhat | dy | new dres]; the last third is the bias gradient of
+  // the Linear layer that writes the residual stream there (null: none)
+  auto ln_jobs = [&](const float* part, float* dw, float* db, float* dbias) {
+    jobs.push_back(ColsumJob{part, dw, 3 * C, c->ln_blocks, C});
+    jobs.push_back(ColsumJob{part + C, db, 3 * C, c->ln_blocks, C});
+    if (dbias) jobs.push_back(ColsumJob{part + 2 * C, dbias, 3 * C, c->ln_blocks, C});
+  };
   {
     PROF(PROF_LN_BWD, 0, ln_bwd_bytes - 4.0 * Nd * Cd);
     // the new dres is d loss / d x_L: its column sums are the last mlp.c_proj bias gradient
+    float* part = c->ln_part + 2 * L * ln_slot;
     RC(launch_layernorm_bwd(st, c->bf16, c->dy, xL, c->lnf_mean, c->lnf_rstd, P(c, lf), c->dres, c->dres_act, false,
-                            c->ln_part, c->ln_blocks, G(c, lf), G(c, lf + 1), G(c, param_index(g, L - 1, MPROJ_B)), N,
-                            C));
+                            part, c->ln_blocks, N, C));
+    ln_jobs(part, G(c, lf), G(c, lf + 1), G(c, param_index(g, L - 1, MPROJ_B)));
   }
   const int ncs = colsum_chunks(N);
   for (int l = L - 1; l >= 0; --l) {
@@ -459,7 +477,8 @@ int backward_impl(gpt2_ctx* c) {
     // the tensor-core path also leaves the column sums of d4C (the c_fc bias gradient) per
     // 32-row group, so d4C is not read again for them
     const bool fused_fc_bias = c->bf16 && c->fc_bias_part != nullptr;
-    if (fused_fc_bias) e.colsum_part = c->fc_bias_part;
+    float* fc_part = fused_fc_bias ? c->fc_bias_part + l * c->fc_bias_stride : nullptr;
+    if (fused_fc_bias) e.colsum_part = fc_part;
     {
       PROF(PROF_GEMM_BWD, 2.0 * Nd * 4 * Cd * Cd, 0);
       RC(gemm(c, N, 4 * C, C, c->dres_act, C, false, W(c, pi(MPROJ_W)), 4 * C, true, e));
@@ -470,9 +489,7 @@ int backward_impl(gpt2_ctx* c) {
       RC(gemm(c, 4 * C, C, N, c->d4c, 4 * C, true, a.ln2, C, true, e));
     }
     if (fused_fc_bias) {
-      const int rows = cdiv(N, 32);
-      PROF(PROF_BIAS, 0, 4.0 * rows * 4 * Cd);
-      RC(launch_colsum_reduce(st, c->fc_bias_part, rows, 4 * C, G(c, pi(FC_B))));
+      jobs.push_back(ColsumJob{fc_part, G(c, pi(FC_B)), 4 * C, cdiv(N, 32), 4 * C});
     } else {
       PROF(PROF_BIAS, 0, A * Nd * 4 * Cd);
       RC(launch_colsum(st, c->bf16, c->d4c, 4 * C, N, 4 * C, c->colsum_part, ncs, G(c, pi(FC_B))));
@@ -485,9 +502,10 @@ int backward_impl(gpt2_ctx* c) {
     {
       PROF(PROF_LN_BWD, 0, ln_bwd_bytes);
       // the new dres is d loss / d x1: its column sums are this layer's attn.c_proj bias gradient
+      float* part = c->ln_part + (2 * l + 1) * ln_slot;
       RC(launch_layernorm_bwd(st, c->bf16, c->dy, a.x1, a.ln2_mean, a.ln2_rstd, P(c, pi(LN2_W)), c->dres,
-                              c->dres_act, true, c->ln_part, c->ln_blocks, G(c, pi(LN2_W)), G(c, pi(LN2_B)),
-                              G(c, pi(PROJ_B)), N, C));
+                              c->dres_act, true, part, c->ln_blocks, N, C));
+      ln_jobs(part, G(c, pi(LN2_W)), G(c, pi(LN2_B)), G(c, pi(PROJ_B)));
     }
     // ---- attention: x1 = x + attn(ln1 Wqkv^T + bqkv) Wp^T + bp
     e = epi_make(EPI_ACCUM_F32, G(c, pi(PROJ_W)), C);
@@ -503,10 +521,11 @@ int backward_impl(gpt2_ctx* c) {
     // the tensor-core path also leaves the column sums of dqkv (the c_attn bias gradient) per
     // 32-row group, so dqkv is not read again for them
     const bool fused_qkv_bias = c->attn_bias_part != nullptr;
+    float* qkv_part = fused_qkv_bias ? c->attn_bias_part + l * c->attn_bias_stride : nullptr;
     {
       PROF(PROF_ATTN_BWD, 4.0 * B * (double)T * T * Cd, 0);
       RC(launch_attn_bwd(st, c->bf16, a.qkv, a.attn, c->dattn, a.attn_lse, c->attnD, c->dqkv, B, T, H, hd,
-                         fused_qkv_bias ? c->attn_bias_part : nullptr));
+                         qkv_part));
     }
     e = epi_make(EPI_ACCUM_F32, G(c, pi(ATTN_W)), C);
     {
@@ -514,9 +533,7 @@ int backward_impl(gpt2_ctx* c) {
       RC(gemm(c, 3 * C, C, N, c->dqkv, 3 * C, true, a.ln1, C, true, e));
     }
     if (fused_qkv_bias) {
-      const int rows = attn_bwd_bias_rows(B, T);
-      PROF(PROF_BIAS, 0, 4.0 * rows * 3 * Cd);
-      RC(launch_colsum_reduce(st, c->attn_bias_part, rows, 3 * C, G(c, pi(ATTN_B))));
+      jobs.push_back(ColsumJob{qkv_part, G(c, pi(ATTN_B)), 3 * C, attn_bwd_bias_rows(B, T), 3 * C});
     } else {
       PROF(PROF_BIAS, 0, A * Nd * 3 * Cd);
       RC(launch_colsum(st, c->bf16, c->dqkv, 3 * C, N, 3 * C, c->colsum_part, ncs, G(c, pi(ATTN_B))));
@@ -530,9 +547,17 @@ int backward_impl(gpt2_ctx* c) {
       PROF(PROF_LN_BWD, 0, ln_bwd_bytes);
       // the new dres is d loss / d x_l: the previous layer's mlp.c_proj bias gradient
       float* db_prev = (l > 0) ? G(c, param_index(g, l - 1, MPROJ_B)) : nullptr;
+      float* part = c->ln_part + 2 * l * ln_slot;
       RC(launch_layernorm_bwd(st, c->bf16, c->dy, x, a.ln1_mean, a.ln1_rstd, P(c, pi(LN1_W)), c->dres, c->dres_act,
-                              true, c->ln_part, c->ln_blocks, G(c, pi(LN1_W)), G(c, pi(LN1_B)), db_prev, N, C));
+                              true, part, c->ln_blocks, N, C));
+      ln_jobs(part, G(c, pi(LN1_W)), G(c, pi(LN1_B)), db_prev);
     }
+  }
+  {
+    double bytes = 0;
+    for (const ColsumJob& j : jobs) bytes += 4.0 * j.rows * j.ncols;
+    PROF(PROF_BIAS, 0, bytes);
+    RC(launch_colsum_batch(st, jobs.data(), (int)jobs.size()));
   }
   // token + position embedding
   {
@@ -719,11 +744,16 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, gpt2_ctx** out) {
   AL(dalloc_bytes(c, &c->dqkv, N * 3 * C * A));
   AL(dalloc_bytes(c, &c->dattn, N * C * A));
   AL(dalloc(c, &c->attnD, N * H));
-  if (c->bf16 && C / H == 64)
-    AL(dalloc(c, &c->attn_bias_part, (size_t)attn_bwd_bias_rows(g.max_batch, g.block_size) * 3 * C));
-  if (c->bf16) AL(dalloc(c, &c->fc_bias_part, (size_t)cdiv(g.max_batch * g.block_size, 32) * 4 * C));
+  if (c->bf16 && C / H == 64) {
+    c->attn_bias_stride = (size_t)attn_bwd_bias_rows(g.max_batch, g.block_size) * 3 * C;
+    AL(dalloc(c, &c->attn_bias_part, L * c->attn_bias_stride));
+  }
+  if (c->bf16) {
+    c->fc_bias_stride = (size_t)cdiv(g.max_batch * g.block_size, 32) * 4 * C;
+    AL(dalloc(c, &c->fc_bias_part, L * c->fc_bias_stride));
+  }
   c->ln_blocks = layernorm_bwd_blocks(c->num_sms);
-  AL(dalloc(c, &c->ln_part, (size_t)c->ln_blocks * 3 * C));
+  AL(dalloc(c, &c->ln_part, (2 * L + 1) * (size_t)c->ln_blocks * 3 * C));
   AL(dalloc(c, &c->colsum_part, (size_t)colsum_chunks((int)N) * 4 * C));
   AL(dalloc(c, &c->enc_sorted, N));
   AL(dalloc(c, &c->enc_seg, encoder_bwd_seg_words((int)N)));

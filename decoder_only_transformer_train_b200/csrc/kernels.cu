@@ -208,44 +208,6 @@ __global__ void __launch_bounds__(256, 2) ln_bwd_kernel(const ActT* __restrict__
   }
 }
 
-// Block: 32 columns x 32 row groups.  Row group r sums partial rows r, r+32, r+64, ... in
-// that order (8 loads in flight: one batch for the 2-per-SM partial rows of a B200), then the
-// 32 group sums are added in group order, so the result does not depend on timing.
-constexpr int LNP_GROUPS = 32;
-__global__ void __launch_bounds__(32 * LNP_GROUPS) ln_param_reduce_kernel(const float* __restrict__ part, int nblocks,
-                                                                         int C, float* __restrict__ dw,
-                                                                         float* __restrict__ db,
-                                                                         float* __restrict__ dbias_out) {
-  __shared__ float red[LNP_GROUPS][33];
-  const int lane = threadIdx.x & 31, r = threadIdx.x >> 5;
-  const int c = blockIdx.x * 32 + lane;
-  const int ncols = dbias_out ? 3 * C : 2 * C;
-  const long long ld = 3LL * C;
-  float s = 0.f;
-  if (c < ncols) {
-    for (int b0 = r; b0 < nblocks; b0 += LNP_GROUPS * 8) {
-      float v[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int b = b0 + LNP_GROUPS * i;
-        v[i] = (b < nblocks) ? part[(long long)b * ld + c] : 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) s += v[i];
-    }
-  }
-  red[r][lane] = s;
-  __syncthreads();
-  if (r == 0 && c < ncols) {
-    float t = 0.f;
-#pragma unroll
-    for (int i = 0; i < LNP_GROUPS; ++i) t += red[i][lane];
-    if (c < C) dw[c] += t;
-    else if (c < 2 * C) db[c - C] += t;
-    else dbias_out[c - 2 * C] += t;
-  }
-}
-
 // ================================================================ bias gradients
 // out[n] += sum_m x[m, n] (bias gradients), in a fixed order: partial sums over row chunks,
 // then the chunks added in order.
@@ -292,23 +254,24 @@ __global__ void __launch_bounds__(1024) colsum_rows_kernel(const T* __restrict__
     for (int i = 0; i < VEC; ++i) part[(long long)blockIdx.x * N + g * VEC + i] = s[i];
   }
 }
-// out[n] += sum_k part[k][n] in a fixed order.  Block: 32 columns x 32 chunk groups; group g
-// adds chunks g, g + 32, ... in order (8 loads in flight: one batch for up to 256 chunks),
-// then the 32 group sums are added in group order.
+// out[n] += sum_k part[k * ld + n] (k < rows, n < ncols) in a fixed order.  Block: 32 columns
+// x 32 row groups; group g adds rows g, g + 32, ... in order (8 loads in flight: one batch for
+// up to 256 rows), then the 32 group sums are added in group order, so the result does not
+// depend on timing.
 constexpr int CSR_GROUPS = 32;
-__global__ void __launch_bounds__(32 * CSR_GROUPS) colsum_reduce_kernel(const float* __restrict__ part, int nchunks,
-                                                                       int N, float* __restrict__ out) {
+__device__ __forceinline__ void colsum_fixed_order(const float* __restrict__ part, long long ld, int rows, int ncols,
+                                                   int col0, float* __restrict__ out) {
   __shared__ float red[CSR_GROUPS][33];
   const int lane = threadIdx.x & 31, gr = threadIdx.x >> 5;
-  const int n = blockIdx.x * 32 + lane;
+  const int n = col0 + lane;
   float s = 0.f;
-  if (n < N) {
-    for (int k0 = gr; k0 < nchunks; k0 += CSR_GROUPS * 8) {
+  if (n < ncols) {
+    for (int k0 = gr; k0 < rows; k0 += CSR_GROUPS * 8) {
       float v[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int k = k0 + CSR_GROUPS * i;
-        v[i] = (k < nchunks) ? part[(long long)k * N + n] : 0.f;
+        v[i] = (k < rows) ? part[(long long)k * ld + n] : 0.f;
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) s += v[i];
@@ -316,12 +279,38 @@ __global__ void __launch_bounds__(32 * CSR_GROUPS) colsum_reduce_kernel(const fl
   }
   red[gr][lane] = s;
   __syncthreads();
-  if (gr == 0 && n < N) {
+  if (gr == 0 && n < ncols) {
     float t = 0.f;
 #pragma unroll
     for (int i = 0; i < CSR_GROUPS; ++i) t += red[i][lane];
     out[n] += t;
   }
+}
+__global__ void __launch_bounds__(32 * CSR_GROUPS) colsum_reduce_kernel(const float* __restrict__ part, int nchunks,
+                                                                       int N, float* __restrict__ out) {
+  colsum_fixed_order(part, N, nchunks, N, blockIdx.x * 32, out);
+}
+// Many independent reductions in one launch (the gradients of the LayerNorm parameters and of
+// the biases, whose partial rows the backward leaves behind): job j owns blocks
+// [block0[j], block0[j + 1]), one per 32 of its columns.  The table is a kernel parameter, read
+// in place.
+constexpr int CSB_MAX_JOBS = 100;
+struct ColsumBatchArgs {
+  ColsumJob job[CSB_MAX_JOBS];
+  int block0[CSB_MAX_JOBS + 1];
+  int njobs;
+};
+static_assert(sizeof(ColsumBatchArgs) <= 4000, "kernel parameters are limited to 4 KB");
+__global__ void __launch_bounds__(32 * CSR_GROUPS) colsum_batch_kernel(const __grid_constant__ ColsumBatchArgs a) {
+  const int bx = blockIdx.x;
+  int lo = 0, hi = a.njobs - 1;
+  while (lo < hi) {   // the last job whose first block is at or before this one
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.block0[mid] <= bx) lo = mid;
+    else hi = mid - 1;
+  }
+  const ColsumJob& j = a.job[lo];
+  colsum_fixed_order(j.part, j.ld, j.rows, j.ncols, (bx - a.block0[lo]) * 32, j.out);
 }
 
 // ================================================================ cross-entropy
@@ -1293,15 +1282,12 @@ int layernorm_bwd_blocks(int num_sms) { return 2 * num_sms; }
 
 int launch_layernorm_bwd(cudaStream_t st, bool is_bf16, const void* dy, const float* x, const float* mean,
                          const float* rstd, const float* w, float* dres, void* dres_act, bool accumulate, float* part,
-                         int nblocks, float* dw, float* db, float* dbias_out, int N, int C) {
+                         int nblocks, int N, int C) {
   int rc = is_bf16 ? ln_bwd_dispatch<bf16>(st, reinterpret_cast<const bf16*>(dy), x, mean, rstd, w, dres,
                                            reinterpret_cast<bf16*>(dres_act), accumulate, part, nblocks, N, C)
                    : ln_bwd_dispatch<float>(st, reinterpret_cast<const float*>(dy), x, mean, rstd, w, dres,
                                             reinterpret_cast<float*>(dres_act), accumulate, part, nblocks, N, C);
   if (rc) return rc;
-  ln_param_reduce_kernel<<<cdiv(dbias_out ? 3 * C : 2 * C, 32), 32 * LNP_GROUPS, 0, st>>>(part, nblocks, C, dw, db,
-                                                                                         dbias_out);
-  note_kernel_launches(1);
   return ok();
 }
 
@@ -1325,10 +1311,24 @@ int launch_colsum(cudaStream_t st, bool is_bf16, const void* x, long long ldx, i
   return ok();
 }
 
-int launch_colsum_reduce(cudaStream_t st, const float* part, int rows, int N, float* out) {
-  if (rows <= 0 || N <= 0) return -4;
-  colsum_reduce_kernel<<<cdiv(N, 32), 32 * CSR_GROUPS, 0, st>>>(part, rows, N, out);
-  note_kernel_launches(1);
+int launch_colsum_batch(cudaStream_t st, const ColsumJob* jobs, int njobs) {
+  for (int j = 0; j < njobs; ++j)
+    if (jobs[j].part == nullptr || jobs[j].out == nullptr || jobs[j].rows <= 0 || jobs[j].ncols <= 0 ||
+        jobs[j].ld < jobs[j].ncols)
+      return -4;
+  for (int first = 0; first < njobs; first += CSB_MAX_JOBS) {
+    ColsumBatchArgs a;
+    a.njobs = njobs - first < CSB_MAX_JOBS ? njobs - first : CSB_MAX_JOBS;
+    int blocks = 0;
+    for (int j = 0; j < a.njobs; ++j) {
+      a.job[j] = jobs[first + j];
+      a.block0[j] = blocks;
+      blocks += cdiv(a.job[j].ncols, 32);
+    }
+    a.block0[a.njobs] = blocks;
+    colsum_batch_kernel<<<blocks, 32 * CSR_GROUPS, 0, st>>>(a);
+    note_kernel_launches(1);
+  }
   return ok();
 }
 

@@ -21,11 +21,12 @@ int launch_encoder_fwd(cudaStream_t st, const int* tok, const float* wte, const 
 int launch_layernorm_fwd(cudaStream_t st, bool bf16, const float* x, const float* w, const float* b, void* y,
                          float* mean, float* rstd, int N, int C);
 // dy: the gradient of the LayerNorm output, of the activation type (bf16 in bf16 mode, as the
-// bf16 product that makes it returns it).  dbias_out (may be null): receives the column sums of
-// the new dres rows.
+// bf16 product that makes it returns it).  part: nblocks rows of 3C floats, each the column
+// sums over this block's rows of [dy * xhat | dy | new dres] (the weight, bias and upstream
+// Linear bias gradients), left for launch_colsum_batch.
 int launch_layernorm_bwd(cudaStream_t st, bool bf16, const void* dy, const float* x, const float* mean,
                          const float* rstd, const float* w, float* dres, void* dres_act, bool accumulate,
-                         float* part, int nblocks, float* dw, float* db, float* dbias_out, int N, int C);
+                         float* part, int nblocks, int N, int C);
 int layernorm_bwd_blocks(int num_sms);
 int launch_colsum(cudaStream_t st, bool bf16, const void* x, long long ldx, int M, int N, float* part, int nchunks,
                   float* out);
@@ -60,7 +61,7 @@ int launch_attn_fwd(cudaStream_t st, bool bf16, const void* qkv, void* out, floa
                     int hd);
 // bias_part (may be null; the bf16 head-size-64 path only): column sums of dqkv per 32-row
 // lane quarter of each 128-row tile, attn_bwd_bias_rows(B, T) rows of 3C floats, to be
-// reduced by launch_colsum_reduce into the c_attn bias gradient.
+// reduced by launch_colsum_batch into the c_attn bias gradient.
 int launch_attn_bwd(cudaStream_t st, bool bf16, const void* qkv, const void* out, const void* dout,
                     const float* lse, float* Dbuf, void* dqkv, int B, int T, int H, int hd,
                     float* bias_part = nullptr);
@@ -68,8 +69,17 @@ int launch_attn_fwd_tc(cudaStream_t st, const void* qkv, void* out, float* lse, 
 int launch_attn_bwd_tc(cudaStream_t st, const void* qkv, const void* dout, const float* lse, const float* Dbuf,
                        void* dqkv, int B, int T, int H, int hd, float* bias_part);
 inline int attn_bwd_bias_rows(int B, int T) { return (T + 127) / 128 * B * 4; }
-// out[n] += sum over rows k of part[k * N + n], in a fixed order
-int launch_colsum_reduce(cudaStream_t st, const float* part, int rows, int N, float* out);
+// One fixed-order column reduction: out[n] += sum over k < rows of part[k * ld + n], n < ncols.
+struct ColsumJob {
+  const float* part;
+  float* out;
+  int ld;
+  int rows;
+  int ncols;
+};
+// Runs every job, up to 100 per launch; each output element gets one add of its sum, whose
+// order of terms is fixed.  Jobs must not write overlapping outputs.
+int launch_colsum_batch(cudaStream_t st, const ColsumJob* jobs, int njobs);
 int read_and_clear_device_error(int* code);
 // Host-side values computed once per (key, device) under a lock: a process may drive several
 // GPUs, from several threads, and a kernel attribute set on one device is unset on the others.
