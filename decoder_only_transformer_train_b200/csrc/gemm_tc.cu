@@ -167,14 +167,16 @@ __device__ __forceinline__ void box_get_f32(const uint8_t* box, int r, float* v)
 
 // Epilogue classes, one kernel instantiation each, so that a kernel carries only its own
 // epilogue code (the fused ones compile to straight-line code for their kind; the plain
-// class covers bf16 / fp32 stores, fp32 accumulation and split-K partials at run time).
-enum EpiClass : int { EK_PLAIN = 0, EK_RESID = 1, EK_GELU_FWD = 2, EK_GELU_BWD = 3, EK_CE = 4 };
+// class is the bf16 store with bias, the fp32 class covers fp32 stores, fp32 accumulation
+// and split-K partials at run time).
+enum EpiClass : int { EK_PLAIN = 0, EK_RESID = 1, EK_GELU_FWD = 2, EK_GELU_BWD = 3, EK_CE = 4, EK_F32 = 5 };
 inline int epi_class(int kind) {
   return kind == EPI_RESID_F32 ? EK_RESID
          : kind == EPI_GELU_FWD ? EK_GELU_FWD
          : kind == EPI_GELU_BWD ? EK_GELU_BWD
          : kind == EPI_CE_FWD   ? EK_CE
-                                : EK_PLAIN;
+         : kind == EPI_STORE_ACT ? EK_PLAIN
+                                 : EK_F32;
 }
 
 __device__ __forceinline__ bool kind_has_bias(int kind) {
@@ -423,8 +425,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                      : (EK == EK_GELU_FWD) ? (int)EPI_GELU_FWD
                      : (EK == EK_GELU_BWD) ? (int)EPI_GELU_BWD
                      : (EK == EK_CE)       ? (int)EPI_CE_FWD
+                     : (EK == EK_PLAIN)    ? (int)EPI_STORE_ACT
                                            : ep.kind;
-    const bool out_bf16 = kind_out_bf16(kind);
+    const bool out_bf16 = (EK != EK_F32) && kind_out_bf16(kind);
     const bool use_bias = ep.bias != nullptr && kind_has_bias(kind);
     const float alpha = ep.alpha;
     // inputs read into the staging boxes and overwritten there by the result: residual or
@@ -778,7 +781,8 @@ int launch_tc_ek(cudaStream_t st, const CUtensorMap& ta, const CUtensorMap& tb, 
     case EK_GELU_BWD:
       return launch_tc<BN, A_MN, B_MN, CG, EK_GELU_BWD>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
     case EK_CE: return launch_tc<BN, A_MN, B_MN, CG, EK_CE>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
-    default: return launch_tc<BN, A_MN, B_MN, CG, EK_PLAIN>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
+    case EK_PLAIN: return launch_tc<BN, A_MN, B_MN, CG, EK_PLAIN>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
+    default: return launch_tc<BN, A_MN, B_MN, CG, EK_F32>(st, ta, tb, tout, tin, tout2, sched, ep, num_sms);
   }
 }
 
