@@ -20,6 +20,7 @@
 //                 next MMA.  At the end of an item the two groups' (m_ref, l, O) are merged.
 #include <math.h>
 #include <stdlib.h>
+#include <type_traits>
 #include "sm100.cuh"
 #include "kernels.h"
 
@@ -856,32 +857,48 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
             tc_fence_before();
             mbar_arrive(sd_empty);
           }
+          // P and dZ of the 16 columns, with the causal mask only on the diagonal tile: the two
+          // cases are separate code, so the other tiles carry no mask arithmetic
+          auto pairs = [&](auto diag_tag) {
+            constexpr bool DG = decltype(diag_tag)::value;
 #pragma unroll
-          for (int d = 0; d < 16; d += 2) {
-            const int c = c0 + 16 * hf + d;
-            float2 nl, nd;
-            if (MODE == 0) {
-              nl = *reinterpret_cast<const float2*>(vec + 16 * hf + d);
-              nd = *reinterpret_cast<const float2*>(vec + 32 + 16 * hf + d);
-            } else {
-              nl = make_float2(nl1, nl1);
-              nd = make_float2(nd1, nd1);
-            }
-            const float2 x = ffma2(make_float2(__uint_as_float(us[d]), __uint_as_float(us[d + 1])), sc, nl);
-            float2 pp = all_masked ? make_float2(0.f, 0.f) : make_float2(ex2(x.x), ex2(x.y));
-            if (diag) {
+            for (int d = 0; d < 16; d += 4) {
+              float4 nl4, nd4;   // the scalars of the 4 columns d .. d + 3
               if (MODE == 0) {
-                if (c < r) pp.x = 0.f;
-                if (c + 1 < r) pp.y = 0.f;
+                nl4 = *reinterpret_cast<const float4*>(vec + 16 * hf + d);
+                nd4 = *reinterpret_cast<const float4*>(vec + 32 + 16 * hf + d);
               } else {
-                if (c > r) pp.x = 0.f;
-                if (c + 1 > r) pp.y = 0.f;
+                nl4 = make_float4(nl1, nl1, nl1, nl1);
+                nd4 = make_float4(nd1, nd1, nd1, nd1);
+              }
+#pragma unroll
+              for (int e = 0; e < 4; e += 2) {
+                const int j = d + e;
+                const float2 nl = e ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+                const float2 nd = e ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+                const float2 x = ffma2(make_float2(__uint_as_float(us[j]), __uint_as_float(us[j + 1])), sc, nl);
+                float2 pp;
+                if constexpr (DG) {
+                  const int c = c0 + 16 * hf + j;
+                  pp = all_masked ? make_float2(0.f, 0.f) : make_float2(ex2(x.x), ex2(x.y));
+                  if (MODE == 0) {
+                    if (c < r) pp.x = 0.f;
+                    if (c + 1 < r) pp.y = 0.f;
+                  } else {
+                    if (c > r) pp.x = 0.f;
+                    if (c + 1 > r) pp.y = 0.f;
+                  }
+                } else {
+                  pp = make_float2(ex2(x.x), ex2(x.y));
+                }
+                const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[j]), __uint_as_float(ud[j + 1])), nd));
+                pw[8 * hf + (j >> 1)] = pack_bf16x2(pp.x, pp.y);
+                dw[8 * hf + (j >> 1)] = pack_bf16x2(gz.x, gz.y);
               }
             }
-            const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[d]), __uint_as_float(ud[d + 1])), nd));
-            pw[8 * hf + (d >> 1)] = pack_bf16x2(pp.x, pp.y);
-            dw[8 * hf + (d >> 1)] = pack_bf16x2(gz.x, gz.y);
-          }
+          };
+          if (diag) pairs(std::true_type{});
+          else pairs(std::false_type{});
         }
         // the previous tile's MMAs must be done reading P / dZ in TMEM
         if (!mbar_wait_warp(ps_empty, (g & 1) ^ 1, abort_flag)) { ok = false; break; }

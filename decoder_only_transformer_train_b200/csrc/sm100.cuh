@@ -292,10 +292,13 @@ __device__ __forceinline__ uint64_t make_sdesc_sw128(uint32_t saddr, uint32_t lb
 
 // The descriptor of an operand `bytes` further on in shared memory: the start-address field
 // holds address >> 4 in the low 14 bits, and shared-memory addresses stay below 256 KB, so
-// adding bytes >> 4 to the whole descriptor never carries into the other fields.  Issuing
-// roles build a base descriptor per buffer once and derive each MMA's from it, which keeps
-// the per-MMA work to one add.
-__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+// adding bytes >> 4 to the low word never carries into the other fields.  Issuing roles build
+// a base descriptor per buffer once and derive each MMA's from it, which keeps the per-MMA
+// work to one 32-bit add.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = static_cast<uint32_t>(d) + (bytes >> 4);
+  return (d & 0xFFFFFFFF00000000ull) | lo;
+}
 
 // ---------------------------------------------------------------- CTA pairs (cta_group::2)
 // Two CTAs of a cluster share one tcgen05.mma: the leader (rank 0) issues it, each CTA
