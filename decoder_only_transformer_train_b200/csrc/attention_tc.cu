@@ -568,8 +568,9 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
   uint64_t* t_full = r_empty + 2;                        // [BWD_STAGES]
   uint64_t* t_empty = t_full + BWD_STAGES;               // [BWD_STAGES]
   uint64_t* sd_full = t_empty + BWD_STAGES;              // S and dP in TMEM
-  uint64_t* sd_empty = sd_full + 1;                      // S and dP read out
-  uint64_t* ps_full = sd_empty + 1;                      // P and dZ written to TMEM
+  uint64_t* s_empty = sd_full + 1;                       // S read out
+  uint64_t* dp_empty = s_empty + 1;                      // dP read out
+  uint64_t* ps_full = dp_empty + 1;                      // P and dZ written to TMEM
   uint64_t* ps_empty = ps_full + 1;                      // P and dZ consumed by the MMAs
   uint64_t* acc_full = ps_empty + 1;                     // [2] an item's accumulation done
   uint64_t* acc_empty = acc_full + 2;                    // [2] an item's accumulators read out
@@ -594,7 +595,8 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       mbar_init(&t_empty[i], 1);
     }
     mbar_init(sd_full, 1);
-    mbar_init(sd_empty, 512);
+    mbar_init(s_empty, 512);
+    mbar_init(dp_empty, 512);
     mbar_init(ps_full, 512);
     mbar_init(ps_empty, 1);
     *abort_flag = 0;
@@ -670,17 +672,24 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
       auto issue_sd = [&](int g, int rb) -> bool {
         const int st = g % BWD_STAGES;
         if (!mbar_wait_warp(&t_full[st], (g / BWD_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait_warp(sd_empty, (g & 1) ^ 1, abort_flag)) return false;
+        // S goes as soon as the elementwise warps have read the previous S, dP once they have
+        // read the previous dP (its second half comes after their first half's arithmetic)
+        if (!mbar_wait_warp(s_empty, (g & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
         const uint64_t a = sdesc_add(dA_k, st * TILE_BYTES), bq = sdesc_add(dB_k, st * TILE_BYTES);
         const uint64_t r0 = sdesc_add(dR_k, rb * 2 * TILE_BYTES), r1 = sdesc_add(r0, TILE_BYTES);
         if (leader) {
 #pragma unroll
-          for (int k = 0; k < HD / 16; ++k) {
-            // MODE 0: S^T = K_j Q_i^T, dP^T = V_j dO_i^T;  MODE 1: S = Q_i K_j^T, dP = dO_i V_j^T
+          for (int k = 0; k < HD / 16; ++k)   // MODE 0: S^T = K_j Q_i^T;  MODE 1: S = Q_i K_j^T
             tc_mma_bf16(tmem + BS_C, sdesc_add(r0, k * 32), sdesc_add(a, k * 32), idesc_sq, k > 0 ? 1u : 0u);
+        }
+        __syncwarp();
+        if (!mbar_wait_warp(dp_empty, (g & 1) ^ 1, abort_flag)) return false;
+        tc_fence_after();
+        if (leader) {
+#pragma unroll
+          for (int k = 0; k < HD / 16; ++k)   // MODE 0: dP^T = V_j dO_i^T;  MODE 1: dP = dO_i V_j^T
             tc_mma_bf16(tmem + BDP_C, sdesc_add(r1, k * 32), sdesc_add(bq, k * 32), idesc_sq, k > 0 ? 1u : 0u);
-          }
           tc_commit(sd_full);
         }
         __syncwarp();
@@ -842,69 +851,73 @@ attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_cons
         // and its scores need no exponentials.
         const bool diag = (t == w.tile);
         const bool all_masked = diag && ((MODE == 0) ? (part < q) : (part > q));
-        // the thread's 32 columns in two halves of 16: S and dP of a half read from TMEM (the
-        // wait for them also keeps the compiler from hoisting the next half's work, which bounds
-        // the registers live at once), P and dZ computed; the S / dP buffer is released after
-        // the second half's read
-        uint32_t pw[16], dw[16];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t us[16], ud[16];
-          tmem_ld16(tmem + lane_off + BS_C + c0 + 16 * hf, us);
-          tmem_ld16(tmem + lane_off + BDP_C + c0 + 16 * hf, ud);
-          tmem_wait_ld_regs16x2(us, ud);
-          if (hf == 1) {
-            tc_fence_before();
-            mbar_arrive(sd_empty);
-          }
-          // P and dZ of the 16 columns, with the causal mask only on the diagonal tile: the two
+        // The thread's 32 columns: all of S and the first 16 of dP come from TMEM first, and S
+        // is released at once; dP's second half is read (and released) after the first half's
+        // P and dZ are computed and stored.  Holding 64 of the 96 registers at most.
+        auto pairs = [&](auto diag_tag, const uint32_t (&us)[32], const uint32_t (&ud)[16], int hf, uint32_t (&pw)[8],
+                         uint32_t (&dw)[8]) {
+          // P and dZ of 16 columns, with the causal mask only on the diagonal tile: the two
           // cases are separate code, so the other tiles carry no mask arithmetic
-          auto pairs = [&](auto diag_tag) {
-            constexpr bool DG = decltype(diag_tag)::value;
+          constexpr bool DG = decltype(diag_tag)::value;
 #pragma unroll
-            for (int d = 0; d < 16; d += 4) {
-              float4 nl4, nd4;   // the scalars of the 4 columns d .. d + 3
-              if (MODE == 0) {
-                nl4 = *reinterpret_cast<const float4*>(vec + 16 * hf + d);
-                nd4 = *reinterpret_cast<const float4*>(vec + 32 + 16 * hf + d);
-              } else {
-                nl4 = make_float4(nl1, nl1, nl1, nl1);
-                nd4 = make_float4(nd1, nd1, nd1, nd1);
-              }
-#pragma unroll
-              for (int e = 0; e < 4; e += 2) {
-                const int j = d + e;
-                const float2 nl = e ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
-                const float2 nd = e ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-                const float2 x = ffma2(make_float2(__uint_as_float(us[j]), __uint_as_float(us[j + 1])), sc, nl);
-                float2 pp;
-                if constexpr (DG) {
-                  const int c = c0 + 16 * hf + j;
-                  pp = all_masked ? make_float2(0.f, 0.f) : make_float2(ex2(x.x), ex2(x.y));
-                  if (MODE == 0) {
-                    if (c < r) pp.x = 0.f;
-                    if (c + 1 < r) pp.y = 0.f;
-                  } else {
-                    if (c > r) pp.x = 0.f;
-                    if (c + 1 > r) pp.y = 0.f;
-                  }
-                } else {
-                  pp = make_float2(ex2(x.x), ex2(x.y));
-                }
-                const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[j]), __uint_as_float(ud[j + 1])), nd));
-                pw[8 * hf + (j >> 1)] = pack_bf16x2(pp.x, pp.y);
-                dw[8 * hf + (j >> 1)] = pack_bf16x2(gz.x, gz.y);
-              }
+          for (int d = 0; d < 16; d += 4) {
+            float4 nl4, nd4;   // the scalars of the 4 columns d .. d + 3
+            if (MODE == 0) {
+              nl4 = *reinterpret_cast<const float4*>(vec + 16 * hf + d);
+              nd4 = *reinterpret_cast<const float4*>(vec + 32 + 16 * hf + d);
+            } else {
+              nl4 = make_float4(nl1, nl1, nl1, nl1);
+              nd4 = make_float4(nd1, nd1, nd1, nd1);
             }
-          };
-          if (diag) pairs(std::true_type{});
-          else pairs(std::false_type{});
-        }
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+              const int j = d + e;
+              const float2 nl = e ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+              const float2 nd = e ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+              const float2 x = ffma2(make_float2(__uint_as_float(us[16 * hf + j]), __uint_as_float(us[16 * hf + j + 1])),
+                                     sc, nl);
+              float2 pp;
+              if constexpr (DG) {
+                const int c = c0 + 16 * hf + j;
+                pp = all_masked ? make_float2(0.f, 0.f) : make_float2(ex2(x.x), ex2(x.y));
+                if (MODE == 0) {
+                  if (c < r) pp.x = 0.f;
+                  if (c + 1 < r) pp.y = 0.f;
+                } else {
+                  if (c > r) pp.x = 0.f;
+                  if (c + 1 > r) pp.y = 0.f;
+                }
+              } else {
+                pp = make_float2(ex2(x.x), ex2(x.y));
+              }
+              const float2 gz = fmul2(pp, fadd2(make_float2(__uint_as_float(ud[j]), __uint_as_float(ud[j + 1])), nd));
+              pw[j >> 1] = pack_bf16x2(pp.x, pp.y);
+              dw[j >> 1] = pack_bf16x2(gz.x, gz.y);
+            }
+          }
+        };
+        uint32_t us[32], ud[16], pw[8], dw[8];
+        tmem_ld32(tmem + lane_off + BS_C + c0, us);
+        tmem_ld16(tmem + lane_off + BDP_C + c0, ud);
+        tmem_wait_ld_regs(us);
+        tmem_wait_ld_regs16(ud);
+        tc_fence_before();
+        mbar_arrive(s_empty);
+        if (diag) pairs(std::true_type{}, us, ud, 0, pw, dw);
+        else pairs(std::false_type{}, us, ud, 0, pw, dw);
         // the previous tile's MMAs must be done reading P / dZ in TMEM
         if (!mbar_wait_warp(ps_empty, (g & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (MODE == 0) tmem_st16(tmem + lane_off + BP_C + (c0 >> 1), pw);
-        tmem_st16(tmem + lane_off + BDS_C + (c0 >> 1), dw);
+        if (MODE == 0) tmem_st8(tmem + lane_off + BP_C + (c0 >> 1), pw);
+        tmem_st8(tmem + lane_off + BDS_C + (c0 >> 1), dw);
+        tmem_ld16(tmem + lane_off + BDP_C + c0 + 16, ud);
+        tmem_wait_ld_regs16(ud);
+        tc_fence_before();
+        mbar_arrive(dp_empty);
+        if (diag) pairs(std::true_type{}, us, ud, 1, pw, dw);
+        else pairs(std::false_type{}, us, ud, 1, pw, dw);
+        if (MODE == 0) tmem_st8(tmem + lane_off + BP_C + (c0 >> 1) + 8, pw);
+        tmem_st8(tmem + lane_off + BDS_C + (c0 >> 1) + 8, dw);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(ps_full);
