@@ -238,6 +238,24 @@ def test_medium_width_bf16_step_matches_oracle():
     _check_argmax(r["argmax_gpu"], r["logits_ref"])
 
 
+# Fourteen layers of head size 64: the backward then leaves more parameter-gradient partials
+# (LayerNorm weights and biases, the c_attn, c_fc and both c_proj biases: 3 + 8 * 13 + 7 = 114
+# reductions) than one launch of the batched fixed-order reduction takes (100), so the
+# reduction runs as two launches.
+DEEP = O.Config(n_layer=14, n_embd=128, n_head=2, block_size=64, vocab_size=512, padded_vocab_size=512)
+
+
+def test_deep_bf16_step_matches_oracle():
+    r = _run_step(DEEP, BD.GPT2_BF16, B=2, T=64)
+    assert abs(r["losses"][0] - r["loss_ref"]) < 2e-2
+    errs = _per_tensor(r["grads_gpu"], r["grads_ref"], DEEP)
+    assert max(errs.values()) < 2e-2, {k: v for k, v in errs.items() if v >= 2e-2}
+    # the LayerNorm and bias gradients come only from the batched reduction
+    small = {k: v for k, v in errs.items() if k.endswith(("ln_1.weight", "ln_1.bias", "ln_2.weight", "ln_2.bias",
+                                                             "c_attn.bias", "c_fc.bias", "c_proj.bias"))}
+    assert len(small) >= 7 * DEEP.n_layer, sorted(small)[:8]
+
+
 # The GPT-3 context length with the 124M model's head size ("Karpathy's Zero to Hero, Lecture 9"
 # notes, "3:41:50 – 3:53:37 Results: one epoch and an overnight run": T = 2048 to match GPT-3):
 # 16 key tiles per query row in the attention kernels, a 2048-row position table.
