@@ -28,7 +28,6 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;             // 64 bf16 = one 128-byte swizzle row
 constexpr int NUM_THREADS = 320;
-constexpr int EPI_THREADS = 256;
 
 constexpr int BOX_BYTES = 2048;     // one epilogue staging box: 32 rows x 64 bytes
 
@@ -678,6 +677,40 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(float* __restrict__ 
   }
 }
 
+// The same with two consecutive float4 per thread (N % 8 == 0), every load of both issued
+// before the adds, and one thread per pair: for the two-way splits of the weight gradients
+// that is six 16-byte loads in flight per thread and a single pass over the grid.
+__global__ void __launch_bounds__(256) splitk_reduce8_kernel(float* __restrict__ C, long long ldc,
+                                                             const float* __restrict__ ws, int M, int Mpad, int N,
+                                                             int splits, float alpha) {
+  const int n8 = N >> 3;
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= (long long)M * n8) return;
+  const long long per_split = (long long)Mpad * N;
+  const int m = (int)(i / n8), q = (int)(i - (long long)m * n8);
+  const float* src = ws + (long long)m * N + 8 * q;
+  float4* dst = reinterpret_cast<float4*>(C + (long long)m * ldc + 8 * q);
+  float4 v[8][2];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    if (k < splits) {
+      v[k][0] = __ldcs(reinterpret_cast<const float4*>(src + k * per_split));
+      v[k][1] = __ldcs(reinterpret_cast<const float4*>(src + k * per_split) + 1);
+    }
+  float4 c0 = dst[0], c1 = dst[1];
+  float4 a0 = v[0][0], a1 = v[0][1];
+#pragma unroll
+  for (int k = 1; k < 8; ++k)
+    if (k < splits) {
+      a0.x += v[k][0].x; a0.y += v[k][0].y; a0.z += v[k][0].z; a0.w += v[k][0].w;
+      a1.x += v[k][1].x; a1.y += v[k][1].y; a1.z += v[k][1].z; a1.w += v[k][1].w;
+    }
+  c0.x += alpha * a0.x; c0.y += alpha * a0.y; c0.z += alpha * a0.z; c0.w += alpha * a0.w;
+  c1.x += alpha * a1.x; c1.y += alpha * a1.y; c1.z += alpha * a1.z; c1.w += alpha * a1.w;
+  dst[0] = c0;
+  dst[1] = c1;
+}
+
 typedef CUresult (*PFN_tmapEncodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                          const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                          CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -946,7 +979,13 @@ int gemm_bf16_tc(cudaStream_t st, int M, int N, int K, const void* A, long long 
   }
 #undef LAUNCH_BN
   if (rc) return rc;
-  if (split) {
+  if (split && N % 8 == 0 && ep.ldc % 8 == 0) {
+    const long long total = (long long)M * (N / 8);
+    splitk_reduce8_kernel<<<(unsigned)cdivll(total, 256), 256, 0, st>>>(reinterpret_cast<float*>(ep.C), ep.ldc, ws,
+                                                                       M, Mpad, N, sched.splits, ep.alpha);
+    note_kernel_launches(1);
+    if (cudaGetLastError() != cudaSuccess) return -3;
+  } else if (split) {
     const long long total = (long long)M * (N / 4);
     const int threads = 256;
     long long nb = cdivll(total, threads);
