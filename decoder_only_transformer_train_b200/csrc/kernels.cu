@@ -292,8 +292,7 @@ __global__ void __launch_bounds__(32 * CSR_GROUPS) colsum_reduce_kernel(const fl
 }
 // Many independent reductions in one launch (the gradients of the LayerNorm parameters and of
 // the biases, whose partial rows the backward leaves behind): job j owns blocks
-// [block0[j], block0[j + 1]), one per 32 of its columns.  The table is a kernel parameter, read
-// in place.
+// [block0[j], block0[j + 1]).  The table is a kernel parameter, read in place.
 constexpr int CSB_MAX_JOBS = 100;
 struct ColsumBatchArgs {
   ColsumJob job[CSB_MAX_JOBS];
@@ -301,22 +300,11 @@ struct ColsumBatchArgs {
   int njobs;
 };
 static_assert(sizeof(ColsumBatchArgs) <= 4000, "kernel parameters are limited to 4 KB");
-__global__ void __launch_bounds__(32 * CSR_GROUPS) colsum_batch_kernel(const __grid_constant__ ColsumBatchArgs a) {
-  const int bx = blockIdx.x;
-  int lo = 0, hi = a.njobs - 1;
-  while (lo < hi) {   // the last job whose first block is at or before this one
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.block0[mid] <= bx) lo = mid;
-    else hi = mid - 1;
-  }
-  const ColsumJob& j = a.job[lo];
-  colsum_fixed_order(j.part, j.ld, j.rows, j.ncols, (bx - a.block0[lo]) * 32, j.out);
-}
-// The same with 16-byte accesses, for jobs whose columns, row stride and pointers are
-// 16-byte multiples: a block takes 128 columns (a float4 per lane) x 16 row groups; group g
-// adds rows g, g + 16, ... in order (8 loads in flight), then the 16 group sums are added in
-// group order.  A block moves 4x the bytes of the scalar form, so far fewer, longer blocks
-// keep HBM busy.
+// With 16-byte accesses (columns, row stride and pointers are 16-byte multiples): a block
+// takes 128 columns of one job (a float4 per lane) x 16 row groups; group g adds rows g,
+// g + 16, ... in order (8 loads in flight), then the 16 group sums are added in group order,
+// so the result does not depend on timing.  Blocks this wide keep HBM busy where 32-column
+// blocks of 6 us each were latency-bound.
 constexpr int CSB4_GROUPS = 16;
 __global__ void __launch_bounds__(32 * CSB4_GROUPS) colsum_batch4_kernel(const __grid_constant__ ColsumBatchArgs a) {
   __shared__ float4 red[CSB4_GROUPS][32];
@@ -1376,12 +1364,10 @@ int launch_colsum_batch(cudaStream_t st, const ColsumJob* jobs, int njobs) {
     if (jobs[j].part == nullptr || jobs[j].out == nullptr || jobs[j].rows <= 0 || jobs[j].ncols <= 0 ||
         jobs[j].ld < jobs[j].ncols)
       return -4;
-  // the 16-byte form when every job allows it
-  bool vec = true;
   for (int j = 0; j < njobs; ++j)
-    vec = vec && jobs[j].ncols % 4 == 0 && jobs[j].ld % 4 == 0 && reinterpret_cast<uintptr_t>(jobs[j].part) % 16 == 0 &&
-          reinterpret_cast<uintptr_t>(jobs[j].out) % 16 == 0;
-  const int cols_per_block = vec ? 128 : 32;
+    if (jobs[j].ncols % 4 != 0 || jobs[j].ld % 4 != 0 || reinterpret_cast<uintptr_t>(jobs[j].part) % 16 != 0 ||
+        reinterpret_cast<uintptr_t>(jobs[j].out) % 16 != 0)
+      return -1;
   for (int first = 0; first < njobs; first += CSB_MAX_JOBS) {
     ColsumBatchArgs a;
     a.njobs = njobs - first < CSB_MAX_JOBS ? njobs - first : CSB_MAX_JOBS;
@@ -1389,11 +1375,10 @@ int launch_colsum_batch(cudaStream_t st, const ColsumJob* jobs, int njobs) {
     for (int j = 0; j < a.njobs; ++j) {
       a.job[j] = jobs[first + j];
       a.block0[j] = blocks;
-      blocks += cdiv(a.job[j].ncols, cols_per_block);
+      blocks += cdiv(a.job[j].ncols, 128);
     }
     a.block0[a.njobs] = blocks;
-    if (vec) colsum_batch4_kernel<<<blocks, 32 * CSB4_GROUPS, 0, st>>>(a);
-    else colsum_batch_kernel<<<blocks, 32 * CSR_GROUPS, 0, st>>>(a);
+    colsum_batch4_kernel<<<blocks, 32 * CSB4_GROUPS, 0, st>>>(a);
     note_kernel_launches(1);
   }
   return ok();

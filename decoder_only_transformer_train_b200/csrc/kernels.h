@@ -78,7 +78,8 @@ struct ColsumJob {
   int ncols;
 };
 // Runs every job, up to 100 per launch; each output element gets one add of its sum, whose
-// order of terms is fixed.  Jobs must not write overlapping outputs.
+// order of terms is fixed.  Jobs must not write overlapping outputs; their column counts and
+// row strides must be multiples of 4 floats and their pointers 16-byte aligned (-1 if not).
 int launch_colsum_batch(cudaStream_t st, const ColsumJob* jobs, int njobs);
 int read_and_clear_device_error(int* code);
 // Host-side values computed once per (key, device) under a lock: a process may drive several
