@@ -308,7 +308,7 @@ int gpt2op_classifier_fwd_bwd(void* stream, const void* h, const void* W, const 
 #define GPT2_PROF_LN_FWD 6
 #define GPT2_PROF_LN_BWD 7
 #define GPT2_PROF_CE 8          /* softmax finalisation, loss, logit gradient */
-#define GPT2_PROF_BIAS 9        /* bias-gradient column sums */
+#define GPT2_PROF_BIAS 9        /* LayerNorm and bias gradients summed from partial rows */
 #define GPT2_PROF_EMBED 10      /* embedding gather and its backward */
 #define GPT2_PROF_OPTIM 11      /* global norm and AdamW */
 int gpt2_profile_start(gpt2_ctx* ctx);
